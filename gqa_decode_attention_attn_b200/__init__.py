@@ -1,0 +1,256 @@
+"""B200 (sm_100a) decode-time grouped-query attention.
+
+Thin Python binding over the C ABI in ``include/gqa_decode.h``
+(``lib/libgqa_decode_b200.so``).  This module only marshals torch tensors into
+pointers and sizes; every step of the computation runs in the library's CUDA
+kernels.  There is no fallback: if the library is missing or a CUDA device is
+absent, calls raise.
+
+    out = gqa_decode(q, k_cache, v_cache, block_table, seq_lens)
+
+q [B, Hq, D] bf16; caches [num_blocks, Hkv, block_size, D] bf16 (paged, with
+block_table [B, max_blocks] int32) or [B, Hkv, capacity, D] (block_table=None);
+seq_lens [B] int32 -- all on the same CUDA device.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libgqa_decode_b200.so")
+
+GQA_OK = 0
+GQA_ERR_WORKSPACE_TOO_SMALL = 3
+DEV_BAD_BLOCK = 1
+DEV_BAD_LENGTH = 2
+DEV_TIMEOUT = 4
+
+EXPORTED = ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states", "gqa_merge_states",
+            "gqa_status", "gqa_decode_host_buffer_bytes", "gqa_decode_host", "gqa_error_string")
+
+_lib = None
+
+
+class GqaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn}: {error_string(code)} (code {code})")
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python -m gqa_decode_attention_attn_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.gqa_decode_workspace_size.argtypes = [I, I, I, I, I, ctypes.POINTER(SZ)]
+    lib.gqa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, SZ, P]
+    lib.gqa_decode_states.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, SZ, P]
+    lib.gqa_merge_states.argtypes = [P, P, P, I, I, I, P, P, P]
+    lib.gqa_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint)]
+    lib.gqa_decode_host_buffer_bytes.argtypes = [I, I, I, I, I, I, I, I]
+    lib.gqa_decode_host_buffer_bytes.restype = SZ
+    lib.gqa_decode_host.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, SZ, P, SZ, P]
+    lib.gqa_error_string.argtypes = [I]
+    lib.gqa_error_string.restype = ctypes.c_char_p
+    for name in ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states",
+                 "gqa_merge_states", "gqa_status", "gqa_decode_host"):
+        getattr(lib, name).restype = I
+    _lib = lib
+    return lib
+
+
+def error_string(code: int) -> str:
+    return load_library().gqa_error_string(int(code)).decode()
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != GQA_OK:
+        raise GqaError(fn, rc)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _shape(q, k_cache, block_table):
+    if q.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError("q must be [B, Hq, D] and caches [blocks, Hkv, block_size, D]")
+    B, Hq, D = q.shape
+    nb, Hkv, bs, D2 = k_cache.shape
+    if D2 != D:
+        raise ValueError("head_dim of q and the cache differ")
+    mb = 0 if block_table is None else block_table.shape[1]
+    return B, Hq, Hkv, D, bs, mb, nb
+
+
+def _require(t: torch.Tensor, name: str, dtype, device) -> None:
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def workspace_size(B: int, Hq: int, Hkv: int, D: int, device: int | None = None) -> int:
+    lib = load_library()
+    dev = torch.cuda.current_device() if device is None else int(device)
+    out = ctypes.c_size_t(0)
+    _check("gqa_decode_workspace_size", lib.gqa_decode_workspace_size(B, Hq, Hkv, D, dev,
+                                                                      ctypes.byref(out)))
+    return out.value
+
+
+class Workspace:
+    """A zero-initialised device workspace that grows on demand (one per device and
+    stream; calls sharing it must not overlap on the GPU)."""
+
+    def __init__(self, device=None):
+        self.device = torch.device("cuda", torch.cuda.current_device() if device is None
+                                   else torch.device(device).index)
+        self.buf = torch.zeros(0, dtype=torch.uint8, device=self.device)
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf.numel() < nbytes:
+            self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
+        return self.buf
+
+    def status(self, stream=None) -> int:
+        """Device status bits since the last call (synchronises the stream)."""
+        lib = load_library()
+        v = ctypes.c_uint(0)
+        _check("gqa_status", lib.gqa_status(_ptr(self.buf), _stream_ptr(stream), ctypes.byref(v)))
+        return v.value
+
+
+_workspaces: dict = {}
+
+
+def default_workspace(device) -> Workspace:
+    key = (torch.device(device).index, torch.cuda.current_stream(device).cuda_stream)
+    if key not in _workspaces:
+        _workspaces[key] = Workspace(device)
+    return _workspaces[key]
+
+
+def gqa_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+               block_table: Optional[torch.Tensor], seq_lens: torch.Tensor,
+               out: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+               workspace: Optional[Workspace] = None, stream=None) -> torch.Tensor:
+    """Decode attention; returns out [B, Hq, D] bf16 (see include/gqa_decode.h)."""
+    lib = load_library()
+    B, Hq, Hkv, D, bs, mb, nb = _shape(q, k_cache, block_table)
+    dev = q.device
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _require(t, n, torch.bfloat16, dev)
+    _require(seq_lens, "seq_lens", torch.int32, dev)
+    if block_table is not None:
+        _require(block_table, "block_table", torch.int32, dev)
+    if out is None:
+        out = torch.empty_like(q)
+    _require(out, "out", torch.bfloat16, dev)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    ws = default_workspace(dev) if workspace is None else workspace
+    buf = ws.get(workspace_size(B, Hq, Hkv, D, dev.index))
+    with torch.cuda.device(dev):
+        rc = lib.gqa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                            _ptr(seq_lens), _ptr(out), B, Hq, Hkv, D, bs, scale, mb, nb,
+                            _ptr(buf), buf.numel(), _stream_ptr(stream))
+    _check("gqa_decode", rc)
+    return out
+
+
+def gqa_decode_states(q, k_cache, v_cache, block_table, kv_begin, kv_end, scale=None,
+                      workspace: Optional[Workspace] = None, stream=None):
+    """Partial states over [kv_begin[b], kv_end[b]): (acc [B,Hq,D], m [B,Hq], l [B,Hq]) fp32,
+    natural-log units, acc not normalised."""
+    lib = load_library()
+    B, Hq, Hkv, D, bs, mb, nb = _shape(q, k_cache, block_table)
+    dev = q.device
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _require(t, n, torch.bfloat16, dev)
+    _require(kv_begin, "kv_begin", torch.int32, dev)
+    _require(kv_end, "kv_end", torch.int32, dev)
+    if block_table is not None:
+        _require(block_table, "block_table", torch.int32, dev)
+    acc = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    m = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    l = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    ws = default_workspace(dev) if workspace is None else workspace
+    buf = ws.get(workspace_size(B, Hq, Hkv, D, dev.index))
+    with torch.cuda.device(dev):
+        rc = lib.gqa_decode_states(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                   _ptr(kv_begin), _ptr(kv_end), _ptr(acc), _ptr(m), _ptr(l),
+                                   B, Hq, Hkv, D, bs, scale, mb, nb, _ptr(buf), buf.numel(),
+                                   _stream_ptr(stream))
+    _check("gqa_decode_states", rc)
+    return acc, m, l
+
+
+def gqa_merge_states(acc: torch.Tensor, m: torch.Tensor, l: torch.Tensor, stream=None):
+    """Merge S partial states: acc [S, N, D], m/l [S, N] fp32 -> (out [N, D] bf16, lse [N])."""
+    lib = load_library()
+    S, N, D = acc.shape
+    dev = acc.device
+    _require(acc, "acc", torch.float32, dev)
+    _require(m, "m", torch.float32, dev)
+    _require(l, "l", torch.float32, dev)
+    if m.shape != (S, N) or l.shape != (S, N):
+        raise ValueError("m and l must be [S, N]")
+    out = torch.empty((N, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((N,), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.gqa_merge_states(_ptr(acc), _ptr(m), _ptr(l), S, N, D, _ptr(out), _ptr(lse),
+                                  _stream_ptr(stream))
+    _check("gqa_merge_states", rc)
+    return out, lse
+
+
+class HostDecoder:
+    """gqa_decode over HOST tensors: each call copies the inputs host->device, runs the
+    kernel and copies the output back (the C ABI's gqa_decode_host)."""
+
+    def __init__(self, B, Hq, Hkv, D, block_size, max_blocks, num_blocks, paged, device=None):
+        lib = load_library()
+        self.dims = (B, Hq, Hkv, D, block_size, max_blocks, num_blocks)
+        self.paged = bool(paged)
+        self.device = torch.device("cuda", torch.cuda.current_device() if device is None
+                                   else torch.device(device).index)
+        nbytes = lib.gqa_decode_host_buffer_bytes(B, Hq, Hkv, D, block_size, max_blocks,
+                                                  num_blocks, int(paged))
+        self.dbuf = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        self.ws = Workspace(self.device)
+        self.wsbuf = self.ws.get(workspace_size(B, Hq, Hkv, D, self.device.index))
+
+    def h2d_bytes(self, q, k_cache, v_cache, block_table, seq_lens) -> int:
+        n = q.numel() * 2 + k_cache.numel() * 2 + v_cache.numel() * 2 + seq_lens.numel() * 4
+        return n + (0 if block_table is None else block_table.numel() * 4)
+
+    def __call__(self, q, k_cache, v_cache, block_table, seq_lens, out, scale=None, stream=None):
+        lib = load_library()
+        B, Hq, Hkv, D, bs, mb, nb = self.dims
+        scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+        with torch.cuda.device(self.device):
+            rc = lib.gqa_decode_host(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                     _ptr(seq_lens), _ptr(out), B, Hq, Hkv, D, bs, scale, mb, nb,
+                                     _ptr(self.dbuf), self.dbuf.numel(), _ptr(self.wsbuf),
+                                     self.wsbuf.numel(), _stream_ptr(stream))
+        _check("gqa_decode_host", rc)
+        return out

@@ -1,0 +1,397 @@
+// api.cu -- the C ABI declared in include/gqa_decode.h: argument checks,
+// per-device launch geometry, workspace carving and kernel dispatch.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "decode_simt.cuh"
+#include "gqa_decode.h"
+#include "merge_states.cuh"
+
+namespace gqa {
+namespace {
+
+constexpr int MAX_DEVICES = 64;
+constexpr size_t STATUS_BYTES = 256;
+constexpr float LOG2E = 1.4426950408889634f;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Query heads per chunk for the CUDA-core kernel: the next power of two >= G,
+// capped at 8 (larger groups run as several chunks).
+int head_chunk(int G)
+{
+    int gc = 1;
+    while (gc < G && gc < 8)
+        gc <<= 1;
+    return gc;
+}
+
+using KernelFn = void (*)(Params);
+
+template <int D, int GC, bool ST>
+KernelFn simt_fn()
+{
+    return gqa_decode_simt_kernel<D, GC, ST>;
+}
+
+struct Variant {
+    KernelFn fn;
+    int threads;
+    size_t smem_max;                  // shared memory at the largest batch
+    size_t (*smem)(int B);
+    int slot_floats;
+};
+
+template <int D, int GC, bool ST>
+Variant make_variant()
+{
+    using C = SimtCfg<D, GC>;
+    return Variant{simt_fn<D, GC, ST>(), C::THREADS, C::smem_bytes(GQA_MAX_BATCH), &C::smem_bytes,
+                   C::SLOT_FLOATS};
+}
+
+template <bool ST>
+bool pick_gc(int D, int GC, Variant &v)
+{
+#define GQA_CASE(DD, GG)                       \
+    if (D == DD && GC == GG) {                 \
+        v = make_variant<DD, GG, ST>();        \
+        return true;                           \
+    }
+    GQA_CASE(64, 1) GQA_CASE(64, 2) GQA_CASE(64, 4) GQA_CASE(64, 8)
+    GQA_CASE(128, 1) GQA_CASE(128, 2) GQA_CASE(128, 4) GQA_CASE(128, 8)
+    GQA_CASE(256, 1) GQA_CASE(256, 2) GQA_CASE(256, 4) GQA_CASE(256, 8)
+#undef GQA_CASE
+    return false;
+}
+
+bool pick_variant(int D, int G, bool states, Variant &v)
+{
+    const int gc = head_chunk(G);
+    return states ? pick_gc<true>(D, gc, v) : pick_gc<false>(D, gc, v);
+}
+
+// Per-device cache: SM count and, per kernel, resident CTAs per SM.
+struct DeviceGeom {
+    int sms = 0;
+    bool ready = false;
+};
+std::mutex g_mu;
+DeviceGeom g_dev[MAX_DEVICES];
+struct FnGeom {
+    KernelFn fn;
+    int device;
+    int ctas_per_sm;
+};
+FnGeom g_fn[256];
+int g_nfn = 0;
+
+int current_device(int &dev)
+{
+    return cudaGetDevice(&dev) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+// Persistent grid for a kernel on a device: SMs x resident CTAs per SM.
+int persistent_ctas(const Variant &v, int dev, int &ctas)
+{
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (dev < 0 || dev >= MAX_DEVICES)
+        return GQA_ERR_UNSUPPORTED;
+    if (!g_dev[dev].ready) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return GQA_ERR_CUDA;
+        g_dev[dev].sms = sms;
+        g_dev[dev].ready = true;
+    }
+    for (int i = 0; i < g_nfn; ++i) {
+        if (g_fn[i].fn == v.fn && g_fn[i].device == dev) {
+            ctas = g_dev[dev].sms * g_fn[i].ctas_per_sm;
+            return GQA_OK;
+        }
+    }
+    int prev = -1;
+    if (cudaGetDevice(&prev) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    int per_sm = 0;
+    cudaError_t e = cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)v.smem_max);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.fn, v.threads, v.smem_max);
+    if (prev != dev)
+        cudaSetDevice(prev);
+    if (e != cudaSuccess || per_sm < 1)
+        return GQA_ERR_CUDA;
+    if (g_nfn < 256)
+        g_fn[g_nfn++] = FnGeom{v.fn, dev, per_sm};
+    ctas = g_dev[dev].sms * per_sm;
+    return GQA_OK;
+}
+
+struct WorkspaceLayout {
+    size_t counters_off, slots_off, total;
+};
+
+WorkspaceLayout layout_for(int B, int Hq, int ctas, int slot_floats)
+{
+    WorkspaceLayout w;
+    w.counters_off = STATUS_BYTES;
+    w.slots_off = align_up(w.counters_off + sizeof(int) * (size_t)B * Hq, 256);
+    w.total = align_up(w.slots_off + sizeof(float) * 2 * (size_t)ctas * slot_floats, 256);
+    return w;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int check_shape(int B, int Hq, int Hkv, int D, int block_size, const int32_t *block_table,
+                int max_blocks, int num_blocks, float scale)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || block_size <= 0 || Hq % Hkv != 0)
+        return GQA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale))
+        return GQA_ERR_INVALID_ARG;
+    if (block_table && (max_blocks <= 0 || num_blocks <= 0))
+        return GQA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128 && D != 256)
+        return GQA_ERR_UNSUPPORTED;
+    if (B > GQA_MAX_BATCH)
+        return GQA_ERR_UNSUPPORTED;
+    return GQA_OK;
+}
+
+int run_decode(bool states, const void *q, const void *k_cache, const void *v_cache,
+               const int32_t *block_table, const int32_t *seq_lens, const int32_t *kv_begin,
+               const int32_t *kv_end, void *out, float *acc, float *m, float *l, int B, int Hq,
+               int Hkv, int D, int block_size, float scale, int max_blocks, int num_blocks,
+               void *workspace, size_t workspace_bytes, void *stream)
+{
+    int rc = check_shape(B, Hq, Hkv, D, block_size, block_table, max_blocks, num_blocks, scale);
+    if (rc)
+        return rc;
+    if (!q || !k_cache || !v_cache || !workspace)
+        return GQA_ERR_INVALID_ARG;
+    if (states ? (!kv_begin || !kv_end || !acc || !m || !l) : (!seq_lens || !out))
+        return GQA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || (out && !aligned16(out)))
+        return GQA_ERR_MISALIGNED;
+    const int G = Hq / Hkv;
+    Variant v;
+    if (!pick_variant(D, G, states, v))
+        return GQA_ERR_UNSUPPORTED;
+    int dev = 0;
+    if ((rc = current_device(dev)))
+        return rc;
+    int ctas = 0;
+    if ((rc = persistent_ctas(v, dev, ctas)))
+        return rc;
+    const WorkspaceLayout w = layout_for(B, Hq, ctas, v.slot_floats);
+    if (workspace_bytes < w.total)
+        return GQA_ERR_WORKSPACE_TOO_SMALL;
+    if (B == 0)
+        return GQA_OK;
+
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    Params p{};
+    p.q = static_cast<const uint16_t *>(q);
+    p.k = static_cast<const uint16_t *>(k_cache);
+    p.v = static_cast<const uint16_t *>(v_cache);
+    p.block_table = block_table;
+    p.seq_lens = seq_lens;
+    p.kv_begin = kv_begin;
+    p.kv_end = kv_end;
+    p.out = static_cast<uint16_t *>(out);
+    p.st_acc = acc;
+    p.st_m = m;
+    p.st_l = l;
+    p.status = reinterpret_cast<unsigned *>(ws);
+    p.counters = reinterpret_cast<int *>(ws + w.counters_off);
+    p.slots = reinterpret_cast<float *>(ws + w.slots_off);
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = G;
+    p.block_size = block_size;
+    p.max_blocks = block_table ? max_blocks : 1;
+    p.num_blocks = block_table ? num_blocks : B;
+    p.hch = (G + head_chunk(G) - 1) / head_chunk(G);
+    p.capacity = block_table ? (int64_t)max_blocks * block_size : (int64_t)block_size;
+    p.qscale = scale * LOG2E;
+
+    v.fn<<<ctas, v.threads, v.smem(B), static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace gqa
+
+using namespace gqa;
+
+extern "C" {
+
+int gqa_decode_workspace_size(int B, int Hq, int Hkv, int D, int device, size_t *bytes)
+{
+    if (!bytes)
+        return GQA_ERR_INVALID_ARG;
+    int rc = check_shape(B, Hq, Hkv, D, 1, nullptr, 0, 0, 1.0f);
+    if (rc)
+        return rc;
+    size_t best = 0;
+    for (int states = 0; states < 2; ++states) {
+        Variant v;
+        if (!pick_variant(D, Hq / Hkv, states != 0, v))
+            return GQA_ERR_UNSUPPORTED;
+        int ctas = 0;
+        if ((rc = persistent_ctas(v, device, ctas)))
+            return rc;
+        const size_t t = layout_for(B, Hq, ctas, v.slot_floats).total;
+        best = t > best ? t : best;
+    }
+    *bytes = best;
+    return GQA_OK;
+}
+
+int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+               const int32_t *seq_lens, void *out, int B, int Hq, int Hkv, int D, int block_size,
+               float scale, int max_blocks_per_seq, int num_blocks, void *workspace,
+               size_t workspace_bytes, void *stream)
+{
+    return run_decode(false, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, out,
+                      nullptr, nullptr, nullptr, B, Hq, Hkv, D, block_size, scale,
+                      max_blocks_per_seq, num_blocks, workspace, workspace_bytes, stream);
+}
+
+int gqa_decode_states(const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_table, const int32_t *kv_begin, const int32_t *kv_end,
+                      float *acc, float *m, float *l, int B, int Hq, int Hkv, int D,
+                      int block_size, float scale, int max_blocks_per_seq, int num_blocks,
+                      void *workspace, size_t workspace_bytes, void *stream)
+{
+    return run_decode(true, q, k_cache, v_cache, block_table, nullptr, kv_begin, kv_end, nullptr,
+                      acc, m, l, B, Hq, Hkv, D, block_size, scale, max_blocks_per_seq, num_blocks,
+                      workspace, workspace_bytes, stream);
+}
+
+int gqa_merge_states(const float *acc, const float *m, const float *l, int S, int N, int D,
+                     void *out, float *lse, void *stream)
+{
+    if (S < 0 || N < 0 || D <= 0)
+        return GQA_ERR_INVALID_ARG;
+    if (N == 0)
+        return GQA_OK;
+    if (!out || (S > 0 && (!acc || !m || !l)))
+        return GQA_ERR_INVALID_ARG;
+    const int blocks = (N + MERGE_WARPS - 1) / MERGE_WARPS;
+    merge_states_kernel<<<blocks, MERGE_WARPS * 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        acc, m, l, S, N, D, static_cast<uint16_t *>(out), lse);
+    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+int gqa_status(void *workspace, void *stream, unsigned *device_error)
+{
+    if (!workspace || !device_error)
+        return GQA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned v = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    if (cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    if (v && cudaMemset(workspace, 0, sizeof v) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    *device_error = v;
+    return GQA_OK;
+}
+
+struct HostLayout {
+    size_t q, k, v, bt, lens, out, total;
+};
+
+static HostLayout host_layout(int B, int Hq, int Hkv, int D, int block_size, int max_blocks,
+                              int num_blocks, int paged)
+{
+    HostLayout h;
+    const size_t nb = paged ? (size_t)num_blocks : (size_t)B;
+    const size_t qbytes = (size_t)B * Hq * D * 2;
+    const size_t kv = nb * Hkv * (size_t)block_size * D * 2;
+    h.q = 0;
+    h.k = align_up(h.q + qbytes, 256);
+    h.v = align_up(h.k + kv, 256);
+    h.bt = align_up(h.v + kv, 256);
+    h.lens = align_up(h.bt + (paged ? (size_t)B * max_blocks * 4 : 0), 256);
+    h.out = align_up(h.lens + (size_t)B * 4, 256);
+    h.total = align_up(h.out + qbytes, 256);
+    return h;
+}
+
+size_t gqa_decode_host_buffer_bytes(int B, int Hq, int Hkv, int D, int block_size,
+                                    int max_blocks_per_seq, int num_blocks, int paged)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || block_size <= 0)
+        return 0;
+    return host_layout(B, Hq, Hkv, D, block_size, max_blocks_per_seq, num_blocks, paged).total;
+}
+
+int gqa_decode_host(const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_table, const int32_t *seq_lens, void *out, int B, int Hq,
+                    int Hkv, int D, int block_size, float scale, int max_blocks_per_seq,
+                    int num_blocks, void *device_buffer, size_t device_buffer_bytes,
+                    void *workspace, size_t workspace_bytes, void *stream)
+{
+    int rc = check_shape(B, Hq, Hkv, D, block_size, block_table, max_blocks_per_seq, num_blocks,
+                         scale);
+    if (rc)
+        return rc;
+    if (!q || !k_cache || !v_cache || !seq_lens || !out || !device_buffer)
+        return GQA_ERR_INVALID_ARG;
+    const int paged = block_table != nullptr;
+    const HostLayout h =
+        host_layout(B, Hq, Hkv, D, block_size, max_blocks_per_seq, num_blocks, paged);
+    if (device_buffer_bytes < h.total)
+        return GQA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned char *dbuf = static_cast<unsigned char *>(device_buffer);
+    const size_t nb = paged ? (size_t)num_blocks : (size_t)B;
+    const size_t qbytes = (size_t)B * Hq * D * 2;
+    const size_t kv = nb * Hkv * (size_t)block_size * D * 2;
+    bool ok = cudaMemcpyAsync(dbuf + h.q, q, qbytes, cudaMemcpyHostToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(dbuf + h.k, k_cache, kv, cudaMemcpyHostToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(dbuf + h.v, v_cache, kv, cudaMemcpyHostToDevice, s) == cudaSuccess;
+    if (paged)
+        ok = ok && cudaMemcpyAsync(dbuf + h.bt, block_table, (size_t)B * max_blocks_per_seq * 4,
+                                   cudaMemcpyHostToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(dbuf + h.lens, seq_lens, (size_t)B * 4, cudaMemcpyHostToDevice,
+                               s) == cudaSuccess;
+    if (!ok)
+        return GQA_ERR_CUDA;
+    rc = gqa_decode(dbuf + h.q, dbuf + h.k, dbuf + h.v,
+                    paged ? reinterpret_cast<const int32_t *>(dbuf + h.bt) : nullptr,
+                    reinterpret_cast<const int32_t *>(dbuf + h.lens), dbuf + h.out, B, Hq, Hkv, D,
+                    block_size, scale, max_blocks_per_seq, num_blocks, workspace, workspace_bytes,
+                    stream);
+    if (rc)
+        return rc;
+    if (cudaMemcpyAsync(out, dbuf + h.out, qbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    return cudaStreamSynchronize(s) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+const char *gqa_error_string(int code)
+{
+    switch (code) {
+    case GQA_OK: return "ok";
+    case GQA_ERR_INVALID_ARG: return "invalid argument";
+    case GQA_ERR_UNSUPPORTED: return "unsupported shape (D must be 64, 128 or 256; B <= 4096)";
+    case GQA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case GQA_ERR_MISALIGNED: return "bf16 tensor not 16-byte aligned";
+    case GQA_ERR_CUDA: return "CUDA runtime error";
+    default: return "unknown error";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,165 @@
+/*
+ * gqa_decode.h -- C ABI of the B200 (sm_100a) decode-attention library
+ * (libgqa_decode_b200.so).
+ *
+ * Operation (Attention co-design for long-context inference, sections
+ * "Difference between prefill and decode" and "FlashAttention and GEMM shapes";
+ * LeanAttention decode tiles digest, sections "Prefill and decode have different
+ * shapes" and "Exact softmax that merges piece by piece"):
+ *
+ *   for every request b < B and query head h < Hq, with G = Hq / Hkv and
+ *   KV head kvh = h / G,
+ *       out[b, h, :] = softmax_t( scale * q[b, h, :] . K[b, kvh, t, :] ) V[b, kvh, t, :]
+ *   over the cached tokens 0 <= t < seq_lens[b].  One query token per head;
+ *   every cached key is visible (no mask inside a single decode query).
+ *
+ * Data types and layouts (all row-major, innermost index last):
+ *   q, out         bf16 [B, Hq, D]
+ *   k_cache,
+ *   v_cache        bf16 [num_blocks, Hkv, block_size, D]   (paged pool)
+ *                  bf16 [B, Hkv, block_size, D]            (block_table == NULL:
+ *                       contiguous cache, block_size = per-request capacity)
+ *   block_table    int32 [B, max_blocks_per_seq]; logical block j of request b
+ *                  is physical block block_table[b * max_blocks_per_seq + j]
+ *                  (Essential LLM optimization techniques (2), section
+ *                  "PagedAttention", Figure 6-13); entries past a request's
+ *                  last block are never read.
+ *   seq_lens       int32 [B]
+ *   bf16 values are passed as their 16-bit patterns; accumulation is fp32.
+ *
+ * Pointers: unless a function says otherwise, every pointer is a DEVICE pointer
+ * on the current CUDA device, borrowed for the duration of the call (and of the
+ * asynchronous work it enqueues); the library never frees or retains it.
+ * q, k_cache, v_cache and out must be 16-byte aligned.  `stream` is a
+ * cudaStream_t passed as void* (NULL = legacy default stream).
+ *
+ * Errors: every entry point returns GQA_OK (0) or a positive GQA_ERR_* code
+ * after checking its arguments on the host; nothing is enqueued on error.
+ * Problems only the device can see (a block id outside [0, num_blocks), a
+ * length above the capacity, a bounded wait that ran out) never fault or trap:
+ * the kernel skips the offending reads, writes NaN to the affected output rows
+ * and ORs a GQA_DEV_* bit into a status word inside the workspace, which
+ * gqa_status() reads back.
+ */
+#ifndef GQA_DECODE_H
+#define GQA_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GQA_API __attribute__((visibility("default")))
+#else
+#define GQA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Host-side return codes. */
+#define GQA_OK 0
+#define GQA_ERR_INVALID_ARG 1         /* null pointer, negative size, Hq % Hkv != 0, ... */
+#define GQA_ERR_UNSUPPORTED 2         /* D not in {64, 128, 256}, B above GQA_MAX_BATCH, ... */
+#define GQA_ERR_WORKSPACE_TOO_SMALL 3 /* workspace_bytes below gqa_decode_workspace_size() */
+#define GQA_ERR_MISALIGNED 4          /* a bf16 tensor not 16-byte aligned */
+#define GQA_ERR_CUDA 5                /* a CUDA runtime call failed (launch, copy, ...) */
+
+/* Device-side status bits (gqa_status). */
+#define GQA_DEV_BAD_BLOCK 1u   /* a block-table entry outside [0, num_blocks) */
+#define GQA_DEV_BAD_LENGTH 2u  /* a length < 0 or above the cache capacity */
+#define GQA_DEV_TIMEOUT 4u     /* a bounded wait inside the kernel gave up */
+
+#define GQA_MAX_BATCH 4096
+
+/*
+ * Bytes of device workspace gqa_decode / gqa_decode_states need for this shape
+ * on `device` (independent of the lengths).  The workspace holds a status word,
+ * one ticket counter per (request, KV head, head chunk) and two partial softmax
+ * states per persistent CTA.  It must be zero-filled once when allocated; every
+ * call leaves the counters at zero again.  Calls that share one workspace must
+ * not overlap on the GPU (use one stream, or one workspace per stream).
+ */
+GQA_API int gqa_decode_workspace_size(int B, int Hq, int Hkv, int D, int device, size_t *bytes);
+
+/*
+ * Decode attention for one layer and one decode step (the operation above).
+ * Stream-K schedule: the context of every (request, KV head) is cut into
+ * fixed-size tiles; tiles are ordered (request, KV head, tile) and every
+ * persistent CTA takes one contiguous run of that global order, so long
+ * requests spread over many SMs (LeanAttention decode tiles digest, sections
+ * "Exact softmax that merges piece by piece" and "Hardware-sized work units").
+ * A (request, KV head) split across CTAs is finished by whichever CTA arrives
+ * last, which merges the partial states exactly; no CTA ever waits on another.
+ *
+ *   block_table        NULL for a contiguous cache
+ *   max_blocks_per_seq row stride of block_table (ignored when it is NULL)
+ *   num_blocks         pool size, for bounds checks (ignored when block_table is NULL)
+ *   scale              softmax scale, usually 1/sqrt(D)
+ */
+GQA_API int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
+               const int32_t *block_table, const int32_t *seq_lens, void *out,
+               int B, int Hq, int Hkv, int D, int block_size, float scale,
+               int max_blocks_per_seq, int num_blocks,
+               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Partial softmax states of every query row over the key range
+ * [kv_begin[b], kv_end[b]) of request b (both int32 [B], device):
+ *   m[b, h]      = max_t s_t                      (natural-log units)
+ *   l[b, h]      = sum_t exp(s_t - m)
+ *   acc[b, h, :] = sum_t exp(s_t - m) V_t         (not normalised)
+ * acc is fp32 [B, Hq, D]; m and l are fp32 [B, Hq].  An empty range gives
+ * m = -inf, l = 0, acc = 0.  Feeding the states of disjoint ranges that cover
+ * [0, L_b) to gqa_merge_states reproduces gqa_decode (LeanAttention decode tiles
+ * digest, section "Exact softmax that merges piece by piece").
+ */
+GQA_API int gqa_decode_states(const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_table, const int32_t *kv_begin,
+                      const int32_t *kv_end, float *acc, float *m, float *l,
+                      int B, int Hq, int Hkv, int D, int block_size, float scale,
+                      int max_blocks_per_seq, int num_blocks,
+                      void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Exact merge of S partial states per row (LeanAttention decode tiles digest,
+ * section "Exact softmax that merges piece by piece"):
+ *   m* = max_i m_i,  w_i = exp(m_i - m*) (0 when m_i = -inf),
+ *   out = bf16( sum_i w_i acc_i / sum_i w_i l_i ),  lse = m* + log(sum_i w_i l_i).
+ * acc fp32 [S, N, D]; m, l fp32 [S, N]; out bf16 [N, D]; lse fp32 [N] or NULL.
+ * Pieces are combined in index order, so the result does not depend on timing.
+ * A row whose pieces are all empty gives out = 0 and lse = -inf.
+ */
+GQA_API int gqa_merge_states(const float *acc, const float *m, const float *l, int S, int N, int D,
+                     void *out, float *lse, void *stream);
+
+/*
+ * Synchronises `stream`, returns the device status bits accumulated in
+ * `workspace` since the last call in *device_error (0 = clean), and clears them.
+ */
+GQA_API int gqa_status(void *workspace, void *stream, unsigned *device_error);
+
+/*
+ * gqa_decode with HOST buffers: copies q, k_cache, v_cache, block_table and
+ * seq_lens from host memory into `device_buffer` (at least
+ * gqa_decode_host_buffer_bytes() bytes, device), runs gqa_decode, copies out
+ * back to host memory and synchronises the stream.  Pinned host memory gives
+ * asynchronous, full-bandwidth copies.  Same shapes and errors as gqa_decode.
+ */
+GQA_API size_t gqa_decode_host_buffer_bytes(int B, int Hq, int Hkv, int D, int block_size,
+                                    int max_blocks_per_seq, int num_blocks, int paged);
+GQA_API int gqa_decode_host(const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_table, const int32_t *seq_lens, void *out,
+                    int B, int Hq, int Hkv, int D, int block_size, float scale,
+                    int max_blocks_per_seq, int num_blocks,
+                    void *device_buffer, size_t device_buffer_bytes,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* Human-readable text for a GQA_ERR_* code. */
+GQA_API const char *gqa_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_DECODE_H */

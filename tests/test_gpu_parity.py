@@ -1,0 +1,279 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Bar: max-abs error <= 1e-2 and relative RMS error <= 2e-3 per case over all
+outputs; index handling (block tables, lengths) bit-exact, checked through
+poisoned slots that must never be read and through permutation invariance.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from gpu_util import as_f64, parity
+from workloads import make_problem
+
+pytestmark = pytest.mark.gpu
+
+gq = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_lib():
+    global gq
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    import gqa_decode_attention_attn_b200 as mod
+    mod.load_library()
+    gq = mod
+    yield
+
+
+def run(p, out=None, workspace=None):
+    d = p.to("cuda")
+    return gq.gqa_decode(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens, out=out,
+                         scale=p.scale, workspace=workspace)
+
+
+def ref(p, rows=None):
+    return oracle.gqa_decode(p.q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, p.scale,
+                             rows=rows)
+
+
+# --------------------------------------------------------------------- small, many shapes
+
+SMALL = [
+    # B, Hq, Hkv, D, lens, block_size
+    (1, 4, 1, 128, [512], None),
+    (3, 8, 2, 128, [1, 63, 200], None),
+    (2, 8, 8, 128, [64, 65], None),                     # G = 1 (MHA)
+    (2, 8, 1, 128, [129, 7], None),                     # G = 8 (MQA)
+    (2, 6, 2, 128, [100, 33], None),                    # G = 3 (padded head chunk)
+    (2, 12, 2, 128, [300, 5], 16),                      # G = 6
+    (2, 24, 2, 64, [333, 129], 16),                     # G = 12: two head chunks
+    (1, 32, 2, 128, [1000], 64),                        # G = 16
+    (1, 64, 1, 128, [777], 64),                         # G = 64
+    (4, 8, 2, 64, [128, 127, 129, 1], 16),
+    (3, 4, 2, 256, [31, 32, 95], 8),
+    (2, 16, 4, 256, [500, 1], 32),
+    (5, 8, 4, 128, [0, 17, 0, 250, 64], 16),            # empty requests
+    (2, 4, 1, 128, [70, 70], 1),                        # one-token pages
+    (2, 4, 2, 128, [101, 55], 3),                       # pages not a power of two
+    (2, 4, 2, 128, [1000, 999], 100),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"B{c[0]}_Hq{c[1]}_Hkv{c[2]}_D{c[3]}_bs{c[5]}")
+def test_small_shapes(case):
+    B, Hq, Hkv, D, lens, bs = case
+    p = make_problem("small", B, Hq, Hkv, D, lens, seed=100 + sum(lens) + D, block_size=bs,
+                     spare_blocks=3 if bs else 0, capacity=None if bs else max(lens) + 5)
+    out = run(p)
+    torch.cuda.synchronize()
+    parity(out, ref(p), str(case))
+
+
+def test_empty_batch_and_all_empty_requests():
+    p = make_problem("empty", 3, 4, 1, 128, [0, 0, 0], seed=5, block_size=16)
+    out = run(p)
+    assert torch.all(out.float() == 0)
+    p = make_problem("empty0", 0, 4, 1, 128, [], seed=5)
+    assert run(p).numel() == 0
+
+
+def test_single_key_returns_value_row():
+    p = make_problem("one", 2, 8, 2, 128, [1, 1], seed=6)
+    out = run(p).cpu()
+    for b in range(2):
+        for h in range(8):
+            assert torch.equal(out[b, h], p.v_cache[b, h // 4, 0])
+
+
+# --------------------------------------------------------------------- the five workloads
+
+FULL = ["tiny", "llama3_8b", "long_256k"] + [f"sweep_{a}_{b}_{c}" for a, b, c in workloads.SWEEP]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_workload_full_parity(name):
+    p = workloads.workload(name)
+    out = run(p)
+    torch.cuda.synchronize()
+    parity(out, ref(p), name)
+
+
+def test_varlen_paged_sampled_rows():
+    """Full-size variable-length paged batch: every output is finite (poisoned slots and
+    unused table entries never read); sampled requests (shortest, longest, random)
+    match the oracle row by row."""
+    p = workloads.workload("varlen_paged")
+    out = run(p)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    lens = p.seq_lens.tolist()
+    pick = sorted({int(np.argmin(lens)), int(np.argmax(lens)), 7, 31, 50})
+    for b in pick:
+        r = ref(p, rows=(b * p.Hq, (b + 1) * p.Hq))
+        parity(out[b], r, f"varlen request {b} (L={lens[b]})")
+
+
+# --------------------------------------------------------------------- invariants
+
+def test_paging_permutation_bit_identical():
+    """Renaming physical blocks leaves the GPU result bit-identical (the schedule
+    depends only on the lengths)."""
+    lens = [3000, 17, 1025]
+    p = make_problem("perm", 3, 16, 4, 128, lens, seed=7, block_size=16, spare_blocks=5)
+    a = run(p).cpu()
+    perm = torch.randperm(p.num_blocks, generator=torch.Generator().manual_seed(8))
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(p.num_blocks)
+    p.k_cache = p.k_cache[inv].contiguous()
+    p.v_cache = p.v_cache[inv].contiguous()
+    valid = p.block_table >= 0
+    p.block_table[valid] = perm[p.block_table[valid].long()].to(torch.int32)
+    b = run(p).cpu()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_deterministic_repeat():
+    p = workloads.workload("tiny")
+    d = p.to("cuda")
+    outs = [gq.gqa_decode(d.q, d.k_cache, d.v_cache, None, d.seq_lens).clone() for _ in range(3)]
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+
+
+def test_contiguous_equals_paged():
+    lens = [700, 300]
+    p = make_problem("paged", 2, 8, 2, 128, lens, seed=9, block_size=64)
+    cap = max(lens)
+    kc = torch.full((2, 2, cap, 128), float("nan"), dtype=torch.bfloat16)
+    vc = kc.clone()
+    for b, L in enumerate(lens):
+        t = torch.arange(L)
+        blk = p.block_table[b, t // 64].long()
+        kc[b, :, :L] = p.k_cache[blk, :, t % 64].transpose(0, 1)
+        vc[b, :, :L] = p.v_cache[blk, :, t % 64].transpose(0, 1)
+    a = run(p).cpu()
+    c = workloads.Problem("contig", p.q, kc, vc, None, p.seq_lens, p.scale)
+    b = run(c).cpu()
+    parity(b, as_f64(a), "contiguous vs paged")
+
+
+# --------------------------------------------------------------------- states and merge
+
+def test_states_split_merge_matches_decode_and_oracle():
+    lens = [2000, 513, 64]
+    p = make_problem("split", 3, 16, 4, 128, lens, seed=10, block_size=16)
+    d = p.to("cuda")
+    full = gq.gqa_decode(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens, scale=p.scale)
+    cuts = [[0, 1, 700, 2000], [0, 300, 301, 513], [0, 0, 64, 64]]
+    pieces = []
+    for s in range(3):
+        b0 = torch.tensor([c[s] for c in cuts], dtype=torch.int32, device="cuda")
+        b1 = torch.tensor([c[s + 1] for c in cuts], dtype=torch.int32, device="cuda")
+        pieces.append(gq.gqa_decode_states(d.q, d.k_cache, d.v_cache, d.block_table, b0, b1,
+                                           scale=p.scale))
+        # states against the oracle's states
+        acc, m, l = oracle.gqa_decode_states(p.q, p.k_cache, p.v_cache, p.block_table,
+                                             b0.cpu(), b1.cpu(), p.scale)
+        gm = as_f64(pieces[-1][1])
+        fin = np.isfinite(m)
+        assert np.array_equal(fin, np.isfinite(gm))
+        assert np.allclose(gm[fin], m[fin], rtol=1e-5, atol=1e-5)
+        ga, gl = as_f64(pieces[-1][0]), as_f64(pieces[-1][2])
+        # compare normalised pieces (acc / l) where non-empty
+        nz = l > 0
+        assert np.allclose(gl[nz], l[nz], rtol=1e-4)
+        parity(torch.from_numpy((ga[nz] / gl[nz][:, None])), acc[nz] / l[nz][:, None],
+               f"piece {s}")
+    acc = torch.stack([x[0] for x in pieces]).reshape(3, -1, 128)
+    m = torch.stack([x[1] for x in pieces]).reshape(3, -1)
+    l = torch.stack([x[2] for x in pieces]).reshape(3, -1)
+    merged, lse = gq.gqa_merge_states(acc, m, l)
+    torch.cuda.synchronize()
+    r = ref(p)
+    parity(merged.view(3, 16, 128), r, "merged vs oracle")
+    parity(merged.view(3, 16, 128), as_f64(full), "merged vs gqa_decode")
+
+
+def test_merge_states_against_oracle():
+    g = torch.Generator().manual_seed(11)
+    S, N, D = 5, 37, 128
+    acc = torch.randn((S, N, D), generator=g) * 3
+    m = torch.randn((S, N), generator=g) * 4
+    l = torch.rand((S, N), generator=g) + 0.1
+    m[1, :10] = -math.inf
+    l[1, :10] = 0
+    acc[1, :10] = 0
+    m[:, 36] = -math.inf
+    l[:, 36] = 0
+    acc[:, 36] = 0
+    out, lse = gq.gqa_merge_states(acc.cuda(), m.cuda(), l.cuda())
+    torch.cuda.synchronize()
+    r_out, r_lse = oracle.merge_states(acc.double().numpy(), m.double().numpy(),
+                                       l.double().numpy())
+    parity(out, r_out, "merge_states")
+    gl = lse.cpu().double().numpy()
+    assert gl[36] == -np.inf
+    assert np.allclose(gl[:36], r_lse[:36], rtol=1e-6, atol=1e-5)
+
+
+# --------------------------------------------------------------------- errors, no faults
+
+def test_bad_block_id_sets_status_and_nan_rows():
+    lens = [100, 90]
+    p = make_problem("badblk", 2, 4, 1, 128, lens, seed=12, block_size=16)
+    p.block_table[1, 2] = p.num_blocks + 1000          # out of the pool: must not be read
+    ws = gq.Workspace("cuda")
+    out = run(p, workspace=ws)
+    st = ws.status()
+    assert st & gq.DEV_BAD_BLOCK
+    o = out.cpu().float()
+    assert torch.isnan(o[1]).all()
+    r = ref(make_problem("badblk", 2, 4, 1, 128, lens, seed=12, block_size=16))
+    parity(out[0], r[0], "unaffected request")
+    assert ws.status() == 0                             # cleared by the read
+
+
+def test_length_above_capacity_sets_status():
+    p = make_problem("badlen", 2, 4, 1, 128, [10, 20], seed=13, block_size=16)
+    p.seq_lens[0] = 10 ** 6
+    ws = gq.Workspace("cuda")
+    out = run(p, workspace=ws)
+    assert ws.status() & gq.DEV_BAD_LENGTH
+    assert torch.isnan(out[0].float()).all()
+    assert torch.isfinite(out[1].float()).all()
+
+
+def test_workspace_too_small_is_an_error():
+    p = make_problem("ws", 1, 4, 1, 128, [10], seed=14).to("cuda")
+    ws = gq.Workspace("cuda")
+    ws.buf = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    ws.get = lambda n: ws.buf
+    with pytest.raises(gq.GqaError) as e:
+        gq.gqa_decode(p.q, p.k_cache, p.v_cache, None, p.seq_lens, workspace=ws)
+    assert e.value.code == gq.GQA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_max_batch():
+    B = 4096
+    lens = [(i * 37) % 300 for i in range(B)]
+    p = make_problem("maxb", B, 8, 2, 64, lens, seed=15, block_size=16)
+    out = run(p)
+    torch.cuda.synchronize()
+    rows = (1000 * 8, 1100 * 8)
+    parity(out.view(-1, 64)[rows[0]:rows[1]], ref(p, rows=rows), "B=4096 sample")
+
+
+def test_host_buffer_entry_point():
+    p = make_problem("host", 2, 8, 2, 128, [300, 77], seed=16, block_size=16)
+    dec = gq.HostDecoder(p.B, p.Hq, p.Hkv, p.D, p.block_size, p.max_blocks, p.num_blocks, True)
+    pin = lambda t: t.pin_memory()
+    out = torch.empty_like(p.q).pin_memory()
+    dec(pin(p.q), pin(p.k_cache), pin(p.v_cache), pin(p.block_table), pin(p.seq_lens), out,
+        scale=p.scale)
+    parity(out, ref(p), "host-buffer call")
