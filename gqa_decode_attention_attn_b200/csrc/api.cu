@@ -138,11 +138,17 @@ struct WorkspaceLayout {
     size_t counters_off, slots_off, total;
 };
 
-WorkspaceLayout layout_for(int B, int Hq, int ctas, int slot_floats)
+// Fixed layout: [status | ticket counters for the largest shape | partial-state
+// slots].  The counters never move, so whatever shape a call has, each counter it
+// touches is either still zero from allocation or was reset by the call that last
+// used it; slots of one call can never alias counters of another.
+constexpr size_t COUNTERS_BYTES = sizeof(int) * (size_t)GQA_MAX_BATCH * GQA_MAX_QHEADS;
+
+WorkspaceLayout layout_for(int ctas, int slot_floats)
 {
     WorkspaceLayout w;
     w.counters_off = STATUS_BYTES;
-    w.slots_off = align_up(w.counters_off + sizeof(int) * (size_t)B * Hq, 256);
+    w.slots_off = w.counters_off + COUNTERS_BYTES;
     w.total = align_up(w.slots_off + sizeof(float) * 2 * (size_t)ctas * slot_floats, 256);
     return w;
 }
@@ -156,11 +162,11 @@ int check_shape(int B, int Hq, int Hkv, int D, int block_size, const int32_t *bl
         return GQA_ERR_INVALID_ARG;
     if (!std::isfinite(scale))
         return GQA_ERR_INVALID_ARG;
-    if (block_table && (max_blocks <= 0 || num_blocks <= 0))
+    if (block_table && (max_blocks <= 0 || num_blocks < 0))
         return GQA_ERR_INVALID_ARG;
     if (D != 64 && D != 128 && D != 256)
         return GQA_ERR_UNSUPPORTED;
-    if (B > GQA_MAX_BATCH)
+    if (B > GQA_MAX_BATCH || Hq > GQA_MAX_QHEADS)
         return GQA_ERR_UNSUPPORTED;
     return GQA_OK;
 }
@@ -174,7 +180,11 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     int rc = check_shape(B, Hq, Hkv, D, block_size, block_table, max_blocks, num_blocks, scale);
     if (rc)
         return rc;
-    if (!q || !k_cache || !v_cache || !workspace)
+    if (B == 0)
+        return GQA_OK;
+    // An empty pool (num_blocks == 0) is never read: its caches may be null.
+    const bool empty_pool = block_table && num_blocks == 0;
+    if (!q || !workspace || (!empty_pool && (!k_cache || !v_cache)))
         return GQA_ERR_INVALID_ARG;
     if (states ? (!kv_begin || !kv_end || !acc || !m || !l) : (!seq_lens || !out))
         return GQA_ERR_INVALID_ARG;
@@ -190,11 +200,9 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     int ctas = 0;
     if ((rc = persistent_ctas(v, dev, ctas)))
         return rc;
-    const WorkspaceLayout w = layout_for(B, Hq, ctas, v.slot_floats);
+    const WorkspaceLayout w = layout_for(ctas, v.slot_floats);
     if (workspace_bytes < w.total)
         return GQA_ERR_WORKSPACE_TOO_SMALL;
-    if (B == 0)
-        return GQA_OK;
 
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     Params p{};
@@ -222,6 +230,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     p.hch = (G + head_chunk(G) - 1) / head_chunk(G);
     p.capacity = block_table ? (int64_t)max_blocks * block_size : (int64_t)block_size;
     p.qscale = scale * LOG2E;
+    p.timeline = nullptr;
 
     v.fn<<<ctas, v.threads, v.smem(B), static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
@@ -249,7 +258,7 @@ int gqa_decode_workspace_size(int B, int Hq, int Hkv, int D, int device, size_t 
         int ctas = 0;
         if ((rc = persistent_ctas(v, device, ctas)))
             return rc;
-        const size_t t = layout_for(B, Hq, ctas, v.slot_floats).total;
+        const size_t t = layout_for(ctas, v.slot_floats).total;
         best = t > best ? t : best;
     }
     *bytes = best;
@@ -302,7 +311,8 @@ int gqa_status(void *workspace, void *stream, unsigned *device_error)
         return GQA_ERR_CUDA;
     if (cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
         return GQA_ERR_CUDA;
-    if (v && cudaMemset(workspace, 0, sizeof v) != cudaSuccess)
+    // After a device error some tickets may be left mid-count: clear them too.
+    if (v && cudaMemset(workspace, 0, STATUS_BYTES + COUNTERS_BYTES) != cudaSuccess)
         return GQA_ERR_CUDA;
     *device_error = v;
     return GQA_OK;

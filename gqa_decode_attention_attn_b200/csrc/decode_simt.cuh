@@ -1,18 +1,22 @@
 // decode_simt.cuh -- persistent stream-K decode-attention kernel, CUDA-core
 // arithmetic (used when few query heads share a KV head, so that q.K^T is too
-// thin to be a dense contraction).
+// thin to be a dense contraction: G query heads give M = G rows).
 //
 // Per CTA: one producer warp and NC consumer warps.
 //   producer  walks the CTA's run of tiles and, for each tile, issues bulk
 //             asynchronous copies (one per page piece) of the K and V rows into a
 //             STAGES-deep shared-memory ring; completion is counted in bytes on a
 //             "full" mbarrier, and consumers hand slots back on an "empty" one.
-//   consumers split every tile's T tokens evenly.  A warp reads a token row with
-//             16-byte loads, D/8 lanes per token; every KV row is loaded once from
-//             HBM and reused by all GC query heads of the chunk.  q.k partial dots
-//             are reduced across the token's lanes with butterfly shuffles, then
-//             the online softmax (running max m, running sum l, in log2 units)
-//             rescales the fp32 accumulators and adds p * V.
+//   consumers split every tile's T tokens evenly.  A warp reads token rows with
+//             16-byte shared loads, D/8 lanes per token; every KV row is loaded
+//             once from HBM and reused by all GC query heads of the chunk.
+//             BMM1: packed fp32 FMAs (two lanes of math per instruction) give
+//             per-lane partial dots, which a transposed butterfly reduces across
+//             the token's lanes so that each lane ends with whole scores.
+//             Online softmax: running max m and sum l per head, in log2 units
+//             (scale * log2 e is folded into q), one SFU exponential per score;
+//             the fp32 accumulators are rescaled only when a maximum moved.
+//             BMM2: packed FMAs of p * V into fp32 accumulators.
 //   epilogue  at the end of a segment piece the NC warp states are merged in
 //             shared memory; a whole segment writes bf16 output directly, a
 //             partial one stores (acc, m, l) in its workspace slot and takes a
@@ -40,16 +44,24 @@ struct SimtCfg {
     static constexpr int TPW = 32 / LPT;               // tokens per warp step
     static constexpr int TOKW = T / NC;                // tokens per warp per tile
     static constexpr int STEPS = TOKW / TPW;           // warp steps per tile
+    static constexpr int NV = STEPS * GC;              // partial dots per lane
+    static constexpr int NF = NV >= LPT ? NV / LPT : 1;  // whole scores per lane
+    static constexpr int REP = NV >= LPT ? 1 : LPT / NV; // lanes sharing one score
+    static constexpr int NS = TOKW * GC;               // scores per warp per tile
+    static constexpr int NSL = (NS + 31) / 32;         // scores per lane (softmax)
     static constexpr int TILE_ELEMS = T * D;
     static constexpr int SCRATCH_PER_WARP = GC * D + ((2 * GC + 3) / 4) * 4;  // 16-byte multiple
+    static constexpr int PSCR_PER_WARP = ((NS + GC + 3) / 4) * 4;              // scores + alphas
     static constexpr size_t RING_BYTES = 2ull * STAGES * TILE_ELEMS * sizeof(uint16_t);
     static constexpr size_t BAR_OFF = RING_BYTES;
     static constexpr size_t FLAG_OFF = BAR_OFF + 2 * STAGES * sizeof(uint64_t);
     static constexpr size_t SCRATCH_OFF = FLAG_OFF + 32 * sizeof(int);
-    static constexpr size_t PREFIX_OFF = SCRATCH_OFF + (size_t)NC * SCRATCH_PER_WARP * sizeof(float);
+    static constexpr size_t PSCR_OFF = SCRATCH_OFF + (size_t)NC * SCRATCH_PER_WARP * sizeof(float);
+    static constexpr size_t PREFIX_OFF = PSCR_OFF + (size_t)NC * PSCR_PER_WARP * sizeof(float);
     static constexpr int SLOT_FLOATS = GC * (D + 2);   // one partial state
     static size_t smem_bytes(int B) { return PREFIX_OFF + (size_t)(B + 1) * sizeof(int); }
     static_assert(STEPS >= 1 && TOKW % TPW == 0, "tile must split evenly over warps");
+    static_assert(32 % GC == 0 && GC <= 8, "head chunk must divide the warp");
     static_assert(2 * STAGES <= 24, "flag area");
 };
 
@@ -71,6 +83,32 @@ __device__ __forceinline__ void write_result(const Params &p, int64_t row, int d
     }
 }
 
+// Transposed butterfly: NV partial sums per lane, reduced across the LPT lanes of
+// a token.  While a lane still holds two or more values, each level hands half of
+// them to the partner and keeps the other half (one shuffle per kept value);
+// afterwards plain butterflies finish.  Lane s (= lane % LPT) ends with the NF
+// whole sums of flat indices NF * (s / REP) + j.
+template <int LPT, int NV>
+__device__ __forceinline__ void transpose_reduce(float (&v)[NV], int lane)
+{
+#pragma unroll
+    for (int lvl = 0; (LPT >> (lvl + 1)) >= 1; ++lvl) {
+        const int m = LPT >> (lvl + 1);
+        const int n = NV >> lvl;
+        if (n >= 2) {
+            const bool upper = (lane & m) != 0;
+#pragma unroll
+            for (int j = 0; j < n / 2; ++j) {
+                const float send = upper ? v[j] : v[j + n / 2];
+                const float keep = upper ? v[j + n / 2] : v[j];
+                v[j] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+            }
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+        }
+    }
+}
+
 template <int D, int GC, bool STATES>
 __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
     gqa_decode_simt_kernel(const Params p)
@@ -87,10 +125,12 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
     int *last_flag = stage_bad + 25;
     int *poison_flag = stage_bad + 26;
     float *scratch = reinterpret_cast<float *>(smem + C::SCRATCH_OFF);
+    float *pscr = reinterpret_cast<float *>(smem + C::PSCR_OFF);
     int *prefix = reinterpret_cast<int *>(smem + C::PREFIX_OFF);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = p.B;
+    const uint64_t t_start = global_timer_ns();
 
     if (tid == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
@@ -146,23 +186,40 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
         for (int e = tid; e < p.Hq * D; e += C::THREADS)
             write_result<STATES>(p, (int64_t)b * p.Hq + e / D, e % D, D, 0.f, -INFINITY, 0.f, bad);
     }
-    if (start >= end)
+    if (start >= end) {
+        if (p.timeline && tid == 0) {
+            unsigned sm;
+            asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+            unsigned long long *rec = p.timeline + 4 * c;
+            rec[0] = t_start;
+            rec[1] = global_timer_ns();
+            rec[2] = sm;
+            rec[3] = 0;
+        }
         return;
+    }
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         const uint64_t pol = l2_evict_first_policy();
+        TileIter it;
+        it.init(start, prefix, B, units, p.hch);
+        int cur_b = -1;
+        int64_t begin = 0, len = 0;
         int64_t k = 0;
         for (int64_t i = start; i < end; ++i, ++k) {
+            if (i > start)
+                it.next(prefix, B, p.Hkv, p.hch);
             const int s = (int)(k % C::STAGES);
             const uint32_t ph = (uint32_t)((k / C::STAGES) & 1);
             if (k >= C::STAGES && !bounded_wait(&empty[s], ph ^ 1u, abort_flag, p.status))
                 break;
-            const Tile t = locate_tile(i, prefix, B, units, p.hch);
-            int64_t begin, len;
-            request_range<STATES>(p, t.b, begin, len);
-            const int64_t tok0 = begin + (int64_t)t.j * C::T;
-            const int64_t n = min((int64_t)C::T, len - (int64_t)t.j * C::T);
+            if (it.b != cur_b) {
+                cur_b = it.b;
+                request_range<STATES>(p, cur_b, begin, len);
+            }
+            const int64_t tok0 = begin + (int64_t)it.j * C::T;
+            const int64_t n = min((int64_t)C::T, len - (int64_t)it.j * C::T);
             const int64_t bs = p.block_size;
             const int64_t pg0 = tok0 / bs, pg1 = (tok0 + n - 1) / bs;
             const int npieces = (int)(pg1 - pg0 + 1);
@@ -170,7 +227,7 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
             bool bad = false;
             for (int pc = lane; pc < npieces; pc += 32) {
                 const int64_t pg = pg0 + pc;
-                const int64_t blk = p.block_table ? p.block_table[(int64_t)t.b * p.max_blocks + pg] : t.b;
+                const int64_t blk = p.block_table ? p.block_table[(int64_t)it.b * p.max_blocks + pg] : it.b;
                 if (p.block_table && (blk < 0 || blk >= p.num_blocks)) {
                     bad = true;
                 } else {
@@ -192,11 +249,11 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
             __syncwarp();
             for (int pc = lane; pc < npieces; pc += 32) {
                 const int64_t pg = pg0 + pc;
-                const int64_t blk = p.block_table ? p.block_table[(int64_t)t.b * p.max_blocks + pg] : t.b;
+                const int64_t blk = p.block_table ? p.block_table[(int64_t)it.b * p.max_blocks + pg] : it.b;
                 if (p.block_table && (blk < 0 || blk >= p.num_blocks))
                     continue;
                 const int64_t a = max(tok0, pg * bs), z = min(tok0 + n, (pg + 1) * bs);
-                const int64_t src = ((blk * p.Hkv + t.kvh) * bs + (a - pg * bs)) * D;
+                const int64_t src = ((blk * p.Hkv + it.kvh) * bs + (a - pg * bs)) * D;
                 const int64_t dst = (int64_t)s * C::TILE_ELEMS + (a - tok0) * D;
                 const uint32_t nb = (uint32_t)((z - a) * D * 2);
                 bulk_copy_g2s(kring + dst, p.k + src, nb, &full[s], pol);
@@ -220,41 +277,44 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
     const int cw = warp - 1;               // consumer warp index
     const int ctid = tid - 32;             // consumer thread index
     const int grp = lane / C::LPT;         // token slot inside a warp step
-    const int d0 = (lane % C::LPT) * 8;    // this lane's 8 dimensions
+    const int sub = lane % C::LPT;
+    const int d0 = sub * 8;                // this lane's 8 dimensions
     const int G = p.G;
+    float *ps = pscr + cw * C::PSCR_PER_WARP;  // this warp's scores / probabilities
+    float *alpha_s = ps + C::NS;
 
-    float qf[GC][8], acc[GC][8], m[GC], l[GC];
+    float2 q2[GC][4], acc[GC][4];
+    float m_h = -INFINITY, l_h = 0.f;      // running max / sum of head (lane % GC)
     bool poisoned = false;
-    Tile cur{};
+    TileIter it, cur;
+    it.init(start, prefix, B, units, p.hch);
+    cur = it;
     int64_t piece_first = start;
     int64_t k = 0;
 
     for (int64_t i = start; i < end; ++i, ++k) {
-        const Tile t = locate_tile(i, prefix, B, units, p.hch);
-        if (i == start || t.seg0 != cur.seg0) {
-            cur = t;
+        if (i > start)
+            it.next(prefix, B, p.Hkv, p.hch);
+        if (i == start || it.seg0 != cur.seg0) {
+            cur = it;
             piece_first = i;
             poisoned = false;
+            m_h = -INFINITY;
+            l_h = 0.f;
 #pragma unroll
             for (int g = 0; g < GC; ++g) {
-                const int hg = t.hc * GC + g;  // head inside the group
+                const int hg = it.hc * GC + g;  // head inside the group
                 uint4 w = make_uint4(0, 0, 0, 0);
                 if (hg < G)
                     w = __ldg(reinterpret_cast<const uint4 *>(
-                        p.q + (((int64_t)t.b * p.Hq + (int64_t)t.kvh * G + hg) * D + d0)));
+                        p.q + (((int64_t)it.b * p.Hq + (int64_t)it.kvh * G + hg) * D + d0)));
                 const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    float lo, hi;
-                    bf16x2_to_float2(ww[j], lo, hi);
-                    qf[g][2 * j] = lo * p.qscale;
-                    qf[g][2 * j + 1] = hi * p.qscale;
+                    const float2 f = bf16x2_to_float2(ww[j]);
+                    q2[g][j] = make_float2(f.x * p.qscale, f.y * p.qscale);
+                    acc[g][j] = make_float2(0.f, 0.f);
                 }
-                m[g] = -INFINITY;
-                l[g] = 0.f;
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    acc[g][j] = 0.f;
             }
         }
 
@@ -268,121 +328,153 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
             const int n = stage_n[s];
             const uint16_t *Ks = kring + s * C::TILE_ELEMS;
             const uint16_t *Vs = vring + s * C::TILE_ELEMS;
+            const int tok_base = cw * C::TOKW;  // this warp's first token in the tile
 
-            float sc[C::STEPS][GC];
-            bool valid[C::STEPS];
+            // BMM1: partial dots over this lane's 8 dimensions.
+            float part[C::NV];
 #pragma unroll
             for (int st = 0; st < C::STEPS; ++st) {
-                const int tt = cw * C::TOKW + st * C::TPW + grp;
-                valid[st] = tt < n;
+                const int tt = tok_base + st * C::TPW + grp;
                 uint4 w = make_uint4(0, 0, 0, 0);
-                if (valid[st])
+                if (tt < n)
                     w = *reinterpret_cast<const uint4 *>(Ks + tt * D + d0);
-                float kf[8];
-                bf16x2_to_float2(w.x, kf[0], kf[1]);
-                bf16x2_to_float2(w.y, kf[2], kf[3]);
-                bf16x2_to_float2(w.z, kf[4], kf[5]);
-                bf16x2_to_float2(w.w, kf[6], kf[7]);
+                const float2 k0 = bf16x2_to_float2(w.x), k1 = bf16x2_to_float2(w.y);
+                const float2 k2 = bf16x2_to_float2(w.z), k3 = bf16x2_to_float2(w.w);
 #pragma unroll
                 for (int g = 0; g < GC; ++g) {
-                    float a = 0.f;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        a = fmaf(qf[g][j], kf[j], a);
-                    sc[st][g] = a;
+                    float2 a = __fmul2_rn(q2[g][0], k0);
+                    a = __ffma2_rn(q2[g][1], k1, a);
+                    a = __ffma2_rn(q2[g][2], k2, a);
+                    a = __ffma2_rn(q2[g][3], k3, a);
+                    part[st * GC + g] = a.x + a.y;
                 }
             }
-            // Full dot products: butterfly over the LPT lanes of each token.
+            transpose_reduce<C::LPT, C::NV>(part, lane);
+            // Scores to shared memory in (token, head) order.
+            if (sub % C::REP == 0) {
 #pragma unroll
-            for (int o = C::LPT / 2; o >= 1; o >>= 1)
-#pragma unroll
-                for (int st = 0; st < C::STEPS; ++st)
-#pragma unroll
-                    for (int g = 0; g < GC; ++g)
-                        sc[st][g] += __shfl_xor_sync(0xffffffffu, sc[st][g], o);
-            // Online softmax over this warp's tokens of the tile (scores become
-            // probabilities in place).
-#pragma unroll
-            for (int g = 0; g < GC; ++g) {
-                float mx = -INFINITY;
-#pragma unroll
-                for (int st = 0; st < C::STEPS; ++st)
-                    if (valid[st])
-                        mx = fmaxf(mx, sc[st][g]);
-#pragma unroll
-                for (int o = C::LPT; o < 32; o <<= 1)
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                const float mnew = fmaxf(m[g], mx);
-                const float muse = mnew == -INFINITY ? 0.f : mnew;
-                const float alpha = exp2f(m[g] - muse);
-                float ps = 0.f;
-#pragma unroll
-                for (int st = 0; st < C::STEPS; ++st) {
-                    sc[st][g] = valid[st] ? exp2f(sc[st][g] - muse) : 0.f;
-                    ps += sc[st][g];
+                for (int j = 0; j < C::NF; ++j) {
+                    const int f = C::NF * (sub / C::REP) + j;
+                    ps[((f / GC) * C::TPW + grp) * GC + (f % GC)] = part[j];
                 }
-                l[g] = l[g] * alpha + ps;
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    acc[g][j] *= alpha;
-                m[g] = mnew;
             }
+            __syncwarp();
+
+            // Online softmax.  Lane handles scores sigma = lane + 32 r; all of them
+            // belong to head lane % GC.
+            float sc[C::NSL];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int r = 0; r < C::NSL; ++r) {
+                const int sg = lane + 32 * r;
+                const bool ok = sg < C::NS && tok_base + sg / GC < n;
+                sc[r] = ok ? ps[sg] : -INFINITY;
+                mx = fmaxf(mx, sc[r]);
+            }
+#pragma unroll
+            for (int o = GC; o < 32; o <<= 1)
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const float m_new = fmaxf(m_h, mx);
+            const float m_use = m_new == -INFINITY ? 0.f : m_new;
+            const float alpha = fast_exp2(m_h - m_use);
+            float lsum = 0.f;
+#pragma unroll
+            for (int r = 0; r < C::NSL; ++r) {
+                const int sg = lane + 32 * r;
+                const float pr = fast_exp2(sc[r] - m_use);  // exp2(-inf) = 0
+                lsum += pr;
+                if (sg < C::NS)
+                    ps[sg] = pr;
+            }
+            l_h = l_h * alpha + lsum;
+            m_h = m_new;
+            const bool rescale = __any_sync(0xffffffffu, alpha != 1.f);
+            if (rescale && lane < GC)
+                alpha_s[lane] = alpha;
+            __syncwarp();
+            if (rescale) {
+#pragma unroll
+                for (int g = 0; g < GC; ++g) {
+                    const float a = alpha_s[g];
+                    const float2 a2 = make_float2(a, a);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        acc[g][j] = __fmul2_rn(acc[g][j], a2);
+                }
+            }
+            // BMM2: acc += p * V over this lane's tokens and dimensions.
 #pragma unroll
             for (int st = 0; st < C::STEPS; ++st) {
-                if (!valid[st])
+                const int tl = st * C::TPW + grp;  // token inside this warp's share
+                if (tok_base + tl >= n)
                     continue;
-                const int tt = cw * C::TOKW + st * C::TPW + grp;
-                const uint4 w = *reinterpret_cast<const uint4 *>(Vs + tt * D + d0);
-                float vf[8];
-                bf16x2_to_float2(w.x, vf[0], vf[1]);
-                bf16x2_to_float2(w.y, vf[2], vf[3]);
-                bf16x2_to_float2(w.z, vf[4], vf[5]);
-                bf16x2_to_float2(w.w, vf[6], vf[7]);
+                const uint4 w = *reinterpret_cast<const uint4 *>(Vs + (tok_base + tl) * D + d0);
+                const float2 v0 = bf16x2_to_float2(w.x), v1 = bf16x2_to_float2(w.y);
+                const float2 v2 = bf16x2_to_float2(w.z), v3 = bf16x2_to_float2(w.w);
+                float pv[GC];
+                if constexpr (GC % 4 == 0) {
 #pragma unroll
-                for (int g = 0; g < GC; ++g)
+                    for (int g = 0; g < GC; g += 4) {
+                        const float4 f = *reinterpret_cast<const float4 *>(ps + tl * GC + g);
+                        pv[g] = f.x;
+                        pv[g + 1] = f.y;
+                        pv[g + 2] = f.z;
+                        pv[g + 3] = f.w;
+                    }
+                } else {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        acc[g][j] = fmaf(sc[st][g], vf[j], acc[g][j]);
+                    for (int g = 0; g < GC; ++g)
+                        pv[g] = ps[tl * GC + g];
+                }
+#pragma unroll
+                for (int g = 0; g < GC; ++g) {
+                    const float2 pp = make_float2(pv[g], pv[g]);
+                    acc[g][0] = __ffma2_rn(pp, v0, acc[g][0]);
+                    acc[g][1] = __ffma2_rn(pp, v1, acc[g][1]);
+                    acc[g][2] = __ffma2_rn(pp, v2, acc[g][2]);
+                    acc[g][3] = __ffma2_rn(pp, v3, acc[g][3]);
+                }
             }
         }
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&empty[s]);
 
-        const bool piece_end = (i + 1 == end) || (i + 1 == t.seg0 + t.nb);
+        const bool piece_end = (i + 1 == end) || (i + 1 == it.seg0 + it.nb);
         if (!piece_end)
             continue;
 
         // ------------------------------------------------------------ epilogue
-        // Token slots of a warp share m; add their l and acc.
+        // Lanes of one head share m; add their l.  Token slots of a warp share m;
+        // add their accumulators.
+        float l_tot = l_h;
 #pragma unroll
-        for (int g = 0; g < GC; ++g) {
+        for (int o = GC; o < 32; o <<= 1)
+            l_tot += __shfl_xor_sync(0xffffffffu, l_tot, o);
 #pragma unroll
-            for (int o = C::LPT; o < 32; o <<= 1) {
-                l[g] += __shfl_xor_sync(0xffffffffu, l[g], o);
+        for (int g = 0; g < GC; ++g)
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    acc[g][j] += __shfl_xor_sync(0xffffffffu, acc[g][j], o);
-            }
-        }
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int o = C::LPT; o < 32; o <<= 1) {
+                    acc[g][j].x += __shfl_xor_sync(0xffffffffu, acc[g][j].x, o);
+                    acc[g][j].y += __shfl_xor_sync(0xffffffffu, acc[g][j].y, o);
+                }
         float *mine = scratch + cw * C::SCRATCH_PER_WARP;
         if (grp == 0) {
 #pragma unroll
             for (int g = 0; g < GC; ++g) {
                 float4 *dst = reinterpret_cast<float4 *>(mine + g * D + d0);
-                dst[0] = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
-                dst[1] = make_float4(acc[g][4], acc[g][5], acc[g][6], acc[g][7]);
+                dst[0] = make_float4(acc[g][0].x, acc[g][0].y, acc[g][1].x, acc[g][1].y);
+                dst[1] = make_float4(acc[g][2].x, acc[g][2].y, acc[g][3].x, acc[g][3].y);
             }
         }
-        if (lane == 0) {
-#pragma unroll
-            for (int g = 0; g < GC; ++g) {
-                mine[GC * D + g] = m[g];
-                mine[GC * D + GC + g] = l[g];
-            }
-            if (poisoned)
-                atomicOr(poison_flag, 1);
+        if (lane < GC) {
+            mine[GC * D + lane] = m_h;
+            mine[GC * D + GC + lane] = l_tot;
         }
+        if (lane == 0 && poisoned)
+            atomicOr(poison_flag, 1);
         named_barrier_sync(1, C::NC * 32);
 
         const bool pois = *reinterpret_cast<volatile int *>(poison_flag) != 0;
@@ -405,7 +497,7 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
             for (int w = 0; w < C::NC; ++w) {
                 const float *sw = scratch + w * C::SCRATCH_PER_WARP;
                 const float mw = sw[GC * D + g];
-                const float wt = mw == -INFINITY ? 0.f : exp2f(mw - ms);
+                const float wt = mw == -INFINITY ? 0.f : fast_exp2(mw - ms);
                 a = fmaf(wt, sw[g * D + d], a);
                 ls = fmaf(wt, sw[GC * D + GC + g], ls);
             }
@@ -434,30 +526,57 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
                 __threadfence();
                 const int64_t seg1 = cur.seg0 + cur.nb;
                 const int64_t c0 = tile_owner(cur.seg0, W, P), c1 = tile_owner(seg1 - 1, W, P);
-                for (int e = ctid; e < GC * D; e += C::NC * 32) {
-                    const int g = e / D, d = e - (e / D) * D;
-                    if (g >= rows)
-                        continue;
+                // Pass 1: common maximum per head (thread g < GC), via shared memory.
+                float *mstar = scratch;  // the warp states are no longer needed
+                if (ctid < GC) {
                     float ms = -INFINITY;
+                    RunWalker rw(c0, W, P);
                     for (int64_t cc = c0; cc <= c1; ++cc) {
-                        const int64_t s0 = run_start(cc, W, P);
-                        if (s0 == run_start(cc + 1, W, P))
+                        const int64_t s0 = rw.start();
+                        rw.next();
+                        if (s0 == rw.start())
                             continue;
                         const float *sl = p.slots + (2 * cc + (s0 < cur.seg0 ? 1 : 0)) * (int64_t)C::SLOT_FLOATS;
-                        ms = fmaxf(ms, __ldcg(sl + GC * D + g));
+                        ms = fmaxf(ms, __ldcg(sl + GC * D + ctid));
                     }
-                    float a = 0.f, ls = 0.f;
-                    for (int64_t cc = c0; cc <= c1; ++cc) {
-                        const int64_t s0 = run_start(cc, W, P);
-                        if (s0 == run_start(cc + 1, W, P))
+                    mstar[ctid] = ms;
+                }
+                named_barrier_sync(1, C::NC * 32);
+                // Pass 2: weighted sums, pieces in CTA order.
+                constexpr int EPT = (GC * D + C::NC * 32 - 1) / (C::NC * 32);
+                float a[EPT], ls[EPT];
+#pragma unroll
+                for (int x = 0; x < EPT; ++x) {
+                    a[x] = 0.f;
+                    ls[x] = 0.f;
+                }
+                RunWalker rw(c0, W, P);
+                for (int64_t cc = c0; cc <= c1; ++cc) {
+                    const int64_t s0 = rw.start();
+                    rw.next();
+                    if (s0 == rw.start())
+                        continue;
+                    const float *sl = p.slots + (2 * cc + (s0 < cur.seg0 ? 1 : 0)) * (int64_t)C::SLOT_FLOATS;
+#pragma unroll
+                    for (int x = 0; x < EPT; ++x) {
+                        const int e = ctid + x * C::NC * 32;
+                        if (e >= GC * D)
                             continue;
-                        const float *sl = p.slots + (2 * cc + (s0 < cur.seg0 ? 1 : 0)) * (int64_t)C::SLOT_FLOATS;
+                        const int g = e / D, d = e - (e / D) * D;
                         const float mw = __ldcg(sl + GC * D + g);
-                        const float wt = mw == -INFINITY ? 0.f : exp2f(mw - ms);
-                        a = fmaf(wt, __ldcg(sl + g * D + d), a);
-                        ls = fmaf(wt, __ldcg(sl + GC * D + GC + g), ls);
+                        const float wt = mw == -INFINITY ? 0.f : fast_exp2(mw - mstar[g]);
+                        a[x] = fmaf(wt, __ldcg(sl + g * D + d), a[x]);
+                        ls[x] = fmaf(wt, __ldcg(sl + GC * D + GC + g), ls[x]);
                     }
-                    write_result<STATES>(p, row0 + g, d, D, a, ms, ls, ls != ls);
+                }
+#pragma unroll
+                for (int x = 0; x < EPT; ++x) {
+                    const int e = ctid + x * C::NC * 32;
+                    if (e >= GC * D)
+                        continue;
+                    const int g = e / D, d = e - (e / D) * D;
+                    if (g < rows)
+                        write_result<STATES>(p, row0 + g, d, D, a[x], mstar[g], ls[x], ls[x] != ls[x]);
                 }
                 if (ctid == 0)
                     p.counters[vseg] = 0;
@@ -466,6 +585,16 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
             *poison_flag = 0;
         }
         named_barrier_sync(1, C::NC * 32);
+    }
+
+    if (p.timeline && ctid == 0) {
+        unsigned sm;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+        unsigned long long *rec = p.timeline + 4 * c;
+        rec[0] = t_start;
+        rec[1] = global_timer_ns();
+        rec[2] = sm;
+        rec[3] = (unsigned long long)(end - start);
     }
 }
 

@@ -91,3 +91,22 @@ __device__ __forceinline__ void bf16x2_to_float2(uint32_t w, float &lo, float &h
 }
 
 }  // namespace gqa
+
+namespace gqa {
+
+// 2^x with the SFU's approximate exponential (ex2.approx.ftz.f32, PTX ISA):
+// relative error about 2^-22; results below 2^-126 flush to zero.
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Two bf16 values packed in a 32-bit word -> float2 (exact).
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w)
+{
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+}  // namespace gqa

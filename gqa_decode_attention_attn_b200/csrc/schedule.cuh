@@ -46,39 +46,83 @@ struct Params {
     int hch;                      // head chunks per KV head
     int64_t capacity;             // tokens a request can hold
     float qscale;                 // scale * log2(e): scores are kept in log2 units
+    unsigned long long *timeline; // optional [grid][4]: start ns, end ns, SM id, tiles
 };
 
-// Global tile index i -> segment coordinates.  prefix[b] = sum of n_b' (b' < b)
-// lives in shared memory; units = Hkv * hch segments per request.
-struct Tile {
+// Walks the global tile order one tile at a time.  prefix[b] = sum of n_b'
+// (b' < b) lives in shared memory; units = Hkv * hch segments per request.  Only
+// init() divides; next() is increments and compares.
+struct TileIter {
     int b, kvh, hc;
     int j;         // tile index inside the segment
     int nb;        // tiles in the segment
     int64_t seg0;  // global index of the segment's first tile
+
+    __device__ __forceinline__ void init(int64_t i, const int *prefix, int B, int64_t units,
+                                         int hch)
+    {
+        int lo = 0, hi = B;  // units*prefix[lo] <= i < units*prefix[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (units * prefix[mid] <= i)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        b = lo;
+        nb = prefix[lo + 1] - prefix[lo];
+        const int64_t local = i - units * prefix[lo];
+        const int64_t vs = local / nb;
+        j = (int)(local - vs * nb);
+        kvh = (int)(vs / hch);
+        hc = (int)(vs - (int64_t)kvh * hch);
+        seg0 = units * prefix[lo] + vs * nb;
+    }
+
+    // Advance to the next tile; the caller guarantees one exists.
+    __device__ __forceinline__ void next(const int *prefix, int B, int Hkv, int hch)
+    {
+        if (++j < nb)
+            return;
+        j = 0;
+        seg0 += nb;
+        if (++hc < hch)
+            return;
+        hc = 0;
+        if (++kvh < Hkv)
+            return;
+        kvh = 0;
+        do {
+            ++b;
+        } while (b < B - 1 && prefix[b + 1] == prefix[b]);
+        nb = prefix[b + 1] - prefix[b];
+    }
 };
 
-__device__ __forceinline__ Tile locate_tile(int64_t i, const int *prefix, int B, int64_t units,
-                                            int hch)
-{
-    int lo = 0, hi = B;  // units*prefix[lo] <= i < units*prefix[hi]
-    while (hi - lo > 1) {
-        int mid = (lo + hi) >> 1;
-        if (units * prefix[mid] <= i)
-            lo = mid;
-        else
-            hi = mid;
+// run_start(c) = floor(c * W / P) for consecutive c without dividing:
+// (q, r) tracks the quotient and remainder of c * W by P.
+struct RunWalker {
+    int64_t q, r, qw, rw, P;
+    __device__ __forceinline__ RunWalker(int64_t c, int64_t W, int64_t P_)
+    {
+        P = P_;
+        qw = W / P;
+        rw = W - qw * P;
+        const int64_t cw = c * W;
+        q = cw / P;
+        r = cw - q * P;
     }
-    Tile t;
-    t.b = lo;
-    t.nb = prefix[lo + 1] - prefix[lo];
-    int64_t local = i - units * prefix[lo];
-    int64_t vs = local / t.nb;
-    t.j = (int)(local - vs * t.nb);
-    t.kvh = (int)(vs / hch);
-    t.hc = (int)(vs - (int64_t)t.kvh * hch);
-    t.seg0 = units * prefix[lo] + vs * t.nb;
-    return t;
-}
+    __device__ __forceinline__ int64_t start() const { return q; }
+    __device__ __forceinline__ void next()
+    {
+        q += qw;
+        r += rw;
+        if (r >= P) {
+            r -= P;
+            ++q;
+        }
+    }
+};
 
 // First tile of CTA c, and the CTA whose run holds tile i.
 __device__ __forceinline__ int64_t run_start(int64_t c, int64_t W, int64_t P)

@@ -60,7 +60,7 @@ extern "C" {
 /* Host-side return codes. */
 #define GQA_OK 0
 #define GQA_ERR_INVALID_ARG 1         /* null pointer, negative size, Hq % Hkv != 0, ... */
-#define GQA_ERR_UNSUPPORTED 2         /* D not in {64, 128, 256}, B above GQA_MAX_BATCH, ... */
+#define GQA_ERR_UNSUPPORTED 2         /* D not in {64, 128, 256}, B or Hq above the maxima */
 #define GQA_ERR_WORKSPACE_TOO_SMALL 3 /* workspace_bytes below gqa_decode_workspace_size() */
 #define GQA_ERR_MISALIGNED 4          /* a bf16 tensor not 16-byte aligned */
 #define GQA_ERR_CUDA 5                /* a CUDA runtime call failed (launch, copy, ...) */
@@ -70,15 +70,19 @@ extern "C" {
 #define GQA_DEV_BAD_LENGTH 2u  /* a length < 0 or above the cache capacity */
 #define GQA_DEV_TIMEOUT 4u     /* a bounded wait inside the kernel gave up */
 
-#define GQA_MAX_BATCH 4096
+#define GQA_MAX_BATCH 4096   /* requests per call */
+#define GQA_MAX_QHEADS 256   /* query heads per request */
 
 /*
  * Bytes of device workspace gqa_decode / gqa_decode_states need for this shape
- * on `device` (independent of the lengths).  The workspace holds a status word,
- * one ticket counter per (request, KV head, head chunk) and two partial softmax
- * states per persistent CTA.  It must be zero-filled once when allocated; every
- * call leaves the counters at zero again.  Calls that share one workspace must
- * not overlap on the GPU (use one stream, or one workspace per stream).
+ * on `device` (independent of the lengths; a few MiB).  The workspace holds a
+ * status word, ticket counters at a fixed offset (room for GQA_MAX_BATCH x
+ * GQA_MAX_QHEADS) and two partial softmax states per persistent CTA.  It must be
+ * zero-filled once when allocated; every completed call leaves the counters at
+ * zero again, so one workspace serves calls of any shape in turn.  After
+ * gqa_status reports a device error it re-zeroes the counters itself.  Calls
+ * that share one workspace must not overlap on the GPU (use one stream, or one
+ * workspace per stream).
  */
 GQA_API int gqa_decode_workspace_size(int B, int Hq, int Hkv, int D, int device, size_t *bytes);
 

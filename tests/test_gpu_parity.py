@@ -201,11 +201,13 @@ def test_states_split_merge_matches_decode_and_oracle():
 
 
 def test_merge_states_against_oracle():
+    # States shaped like real attention pieces: normalised outputs of O(0.1),
+    # normalisers in [1, 100], maxima spread over a few units.
     g = torch.Generator().manual_seed(11)
     S, N, D = 5, 37, 128
-    acc = torch.randn((S, N, D), generator=g) * 3
+    l = torch.rand((S, N), generator=g) * 99 + 1
+    acc = torch.randn((S, N, D), generator=g) * 0.1 * l[..., None]
     m = torch.randn((S, N), generator=g) * 4
-    l = torch.rand((S, N), generator=g) + 0.1
     m[1, :10] = -math.inf
     l[1, :10] = 0
     acc[1, :10] = 0
@@ -257,6 +259,21 @@ def test_workspace_too_small_is_an_error():
     with pytest.raises(gq.GqaError) as e:
         gq.gqa_decode(p.q, p.k_cache, p.v_cache, None, p.seq_lens, workspace=ws)
     assert e.value.code == gq.GQA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_workspace_reused_across_shapes():
+    """One workspace serves calls of different shapes in turn (counters stay at zero
+    between calls)."""
+    ws = gq.Workspace("cuda")
+    shapes = [("a", 1, 4, 1, 128, [512], None), ("b", 16, 32, 8, 128, [3000] * 16, None),
+              ("c", 2, 8, 2, 64, [900, 17], 16), ("d", 64, 8, 8, 128, [300] * 64, 16),
+              ("a", 1, 4, 1, 128, [512], None)]
+    for name, B, Hq, Hkv, D, lens, bs in shapes:
+        p = make_problem(name, B, Hq, Hkv, D, lens, seed=B + D, block_size=bs)
+        out = run(p, workspace=ws)
+        torch.cuda.synchronize()
+        parity(out, ref(p), f"shape {name}")
+    assert ws.status() == 0
 
 
 def test_max_batch():
