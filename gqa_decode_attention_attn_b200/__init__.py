@@ -31,7 +31,9 @@ DEV_BAD_LENGTH = 2
 DEV_TIMEOUT = 4
 
 EXPORTED = ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states", "gqa_merge_states",
-            "gqa_status", "gqa_decode_host_buffer_bytes", "gqa_decode_host", "gqa_error_string")
+            "gqa_status", "gqa_decode_host_buffer_bytes", "gqa_decode_host", "gqa_error_string",
+            "gqa_decode_noalloc")
+GQA_ERR_SCRATCH_LIMIT = 6
 
 _lib = None
 
@@ -254,3 +256,25 @@ class HostDecoder:
                                      self.wsbuf.numel(), _stream_ptr(stream))
         _check("gqa_decode_host", rc)
         return out
+
+
+def gqa_decode_noalloc(q, k_cache, v_cache, block_table, seq_lens, out=None, scale=None,
+                       stream=None):
+    """gqa_decode for callers that cannot allocate device memory: the library uses
+    its own fixed 8 MiB device scratch instead of a workspace.  Calls on one device
+    share that scratch, so they must not overlap on the GPU.  (`out` is allocated
+    here only when the caller passes none.)"""
+    lib = load_library()
+    fn = lib.gqa_decode_noalloc
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    fn.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P]
+    fn.restype = I
+    B, Hq, Hkv, D, bs, mb, nb = _shape(q, k_cache, block_table)
+    if out is None:
+        out = torch.empty_like(q)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    with torch.cuda.device(q.device):
+        rc = fn(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+                _ptr(out), B, Hq, Hkv, D, bs, scale, mb, nb, _stream_ptr(stream))
+    _check("gqa_decode_noalloc", rc)
+    return out

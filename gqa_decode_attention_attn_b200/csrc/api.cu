@@ -400,8 +400,80 @@ const char *gqa_error_string(int code)
     case GQA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
     case GQA_ERR_MISALIGNED: return "bf16 tensor not 16-byte aligned";
     case GQA_ERR_CUDA: return "CUDA runtime error";
+    case GQA_ERR_SCRATCH_LIMIT: return "shape needs more scratch than gqa_decode_noalloc's fixed 8 MiB";
     default: return "unknown error";
     }
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// gqa_decode_noalloc: gqa_decode for callers that cannot allocate device memory.
+//
+// Some callers may not call cudaMalloc at all: code running inside a CUDA-graph
+// capture or another runtime's memory pool, plug-ins whose host owns every
+// allocation, or latency-critical paths that forbid allocator calls.  They still
+// own q, the caches and out, but cannot hand us a workspace.  For them the
+// scratch gqa_decode needs (status word, ticket counters, partial-state slots)
+// lives in one fixed array in this library's device image.  Every GPU that loads
+// the library keeps that array until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t NOALLOC_SCRATCH_BYTES = 8u << 20;  // 8 MiB per device
+
+// Device-side scratch shared by every gqa_decode_noalloc call on a device.  In
+// host code this name is only a handle; its device address comes from
+// cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[gqa::MAX_DEVICES] = {};
+
+// Device address of the scratch array on the current device, looked up once per
+// device (the first call on a device does it).
+int noalloc_scratch(int dev, void **addr)
+{
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+            return GQA_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *addr = g_noalloc_addr[dev];
+    return GQA_OK;
+}
+
+}  // namespace
+
+extern "C" int gqa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                  const int32_t *block_table, const int32_t *seq_lens, void *out,
+                                  int B, int Hq, int Hkv, int D, int block_size, float scale,
+                                  int max_blocks_per_seq, int num_blocks, void *stream)
+{
+    int rc = check_shape(B, Hq, Hkv, D, block_size, block_table, max_blocks_per_seq, num_blocks,
+                         scale);
+    if (rc)
+        return rc;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    if (dev < 0 || dev >= MAX_DEVICES)
+        return GQA_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    if ((rc = noalloc_scratch(dev, &scratch)))
+        return rc;
+    size_t need = 0;
+    if ((rc = gqa_decode_workspace_size(B, Hq, Hkv, D, dev, &need)))
+        return rc;
+    if (need > NOALLOC_SCRATCH_BYTES)
+        return GQA_ERR_SCRATCH_LIMIT;
+    // The status word and the ticket counters this call can touch must start at
+    // zero; a previous call that hit a device error may have left them set.
+    const size_t clear = STATUS_BYTES + sizeof(int) * (size_t)B * Hq;
+    if (cudaMemsetAsync(scratch, 0, clear, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    return gqa_decode(q, k_cache, v_cache, block_table, seq_lens, out, B, Hq, Hkv, D, block_size,
+                      scale, max_blocks_per_seq, num_blocks, scratch, NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -64,6 +64,7 @@ extern "C" {
 #define GQA_ERR_WORKSPACE_TOO_SMALL 3 /* workspace_bytes below gqa_decode_workspace_size() */
 #define GQA_ERR_MISALIGNED 4          /* a bf16 tensor not 16-byte aligned */
 #define GQA_ERR_CUDA 5                /* a CUDA runtime call failed (launch, copy, ...) */
+#define GQA_ERR_SCRATCH_LIMIT 6       /* gqa_decode_noalloc: shape needs more than its fixed scratch */
 
 /* Device-side status bits (gqa_status). */
 #define GQA_DEV_BAD_BLOCK 1u   /* a block-table entry outside [0, num_blocks) */
@@ -158,6 +159,35 @@ GQA_API int gqa_decode_host(const void *q, const void *k_cache, const void *v_ca
                     int max_blocks_per_seq, int num_blocks,
                     void *device_buffer, size_t device_buffer_bytes,
                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gqa_decode without a workspace argument, for callers that cannot allocate
+ * device memory (nothing here calls cudaMalloc, cudaFree or an allocating
+ * library routine).  The pages describe no such call; it exists for callers
+ * that run under an allocator they do not control -- inside another runtime's
+ * memory pool, in a plug-in whose host owns every allocation, or on a path where
+ * allocator calls are forbidden -- and so cannot pass the workspace gqa_decode
+ * wants.  Arguments, layouts and results are those of gqa_decode.
+ *
+ * Scratch: one fixed 8 MiB array inside the library's device image, held by
+ * every GPU that loads the library until the process exits.  A shape whose
+ * scratch need (gqa_decode_workspace_size) exceeds 8 MiB is rejected with
+ * GQA_ERR_SCRATCH_LIMIT; B above GQA_MAX_BATCH or Hq above GQA_MAX_QHEADS with
+ * GQA_ERR_UNSUPPORTED.  On B200 every shape within those maxima fits.
+ *
+ * The first call on each device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  Each call
+ * first clears, on `stream`, the status word and the ticket counters it can use.
+ * All calls on a device share the one array and it keeps the last call's
+ * contents, so calls that overlap on the GPU (different streams, no ordering
+ * between them) race and give wrong results: order them, e.g. on one stream.
+ * Device-side errors (bad block ids, lengths) still yield NaN rows as in
+ * gqa_decode; the status word is not exposed.
+ */
+GQA_API int gqa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                               const int32_t *block_table, const int32_t *seq_lens, void *out,
+                               int B, int Hq, int Hkv, int D, int block_size, float scale,
+                               int max_blocks_per_seq, int num_blocks, void *stream);
 
 /* Human-readable text for a GQA_ERR_* code. */
 GQA_API const char *gqa_error_string(int code);
