@@ -231,6 +231,15 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     p.capacity = block_table ? (int64_t)max_blocks * block_size : (int64_t)block_size;
     p.qscale = scale * LOG2E;
     p.timeline = nullptr;
+    // Magic number for t / block_size (t < 2^31): see page_of().
+    {
+        int l = 0;
+        while ((1ll << l) < block_size)
+            ++l;
+        const uint64_t m = ((((uint64_t)1 << l) - (uint64_t)block_size) << 32) / (uint64_t)block_size + 1;
+        p.bs_magic = (uint32_t)m;
+        p.bs_shift = l;
+    }
 
     v.fn<<<ctas, v.threads, v.smem(B), static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;

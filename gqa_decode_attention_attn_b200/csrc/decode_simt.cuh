@@ -205,65 +205,83 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
         TileIter it;
         it.init(start, prefix, B, units, p.hch);
         int cur_b = -1;
-        int64_t begin = 0, len = 0;
-        int64_t k = 0;
+        int begin = 0, len = 0;
+        int k = 0;
         for (int64_t i = start; i < end; ++i, ++k) {
             if (i > start)
                 it.next(prefix, B, p.Hkv, p.hch);
-            const int s = (int)(k % C::STAGES);
+            const int s = k % C::STAGES;
             const uint32_t ph = (uint32_t)((k / C::STAGES) & 1);
             if (k >= C::STAGES && !bounded_wait(&empty[s], ph ^ 1u, abort_flag, p.status))
                 break;
             if (it.b != cur_b) {
                 cur_b = it.b;
-                request_range<STATES>(p, cur_b, begin, len);
+                int64_t b0, l0;
+                request_range<STATES>(p, cur_b, b0, l0);
+                begin = (int)b0;
+                len = (int)l0;
             }
-            const int64_t tok0 = begin + (int64_t)it.j * C::T;
-            const int64_t n = min((int64_t)C::T, len - (int64_t)it.j * C::T);
-            const int64_t bs = p.block_size;
-            const int64_t pg0 = tok0 / bs, pg1 = (tok0 + n - 1) / bs;
-            const int npieces = (int)(pg1 - pg0 + 1);
-            uint32_t bytes = 0;
+            // Tokens [tok0, tok0 + n) of the request; one copy per page piece.
+            const int tok0 = begin + it.j * C::T;
+            const int n = min(C::T, len - it.j * C::T);
+            const int bs = p.block_size;
+            const int pg0 = page_of(p, tok0);
+            const int npieces = page_of(p, tok0 + n - 1) - pg0 + 1;
+            const int32_t *row = p.block_table ? p.block_table + (int64_t)it.b * p.max_blocks : nullptr;
+            // Pass 1: block ids and their bounds; bytes only need a sum when some
+            // piece is skipped.
+            int64_t blk0 = it.b;
             bool bad = false;
             for (int pc = lane; pc < npieces; pc += 32) {
-                const int64_t pg = pg0 + pc;
-                const int64_t blk = p.block_table ? p.block_table[(int64_t)it.b * p.max_blocks + pg] : it.b;
-                if (p.block_table && (blk < 0 || blk >= p.num_blocks)) {
+                const int64_t blk = row ? row[pg0 + pc] : it.b;
+                if (pc == lane)
+                    blk0 = blk;
+                if (row && (blk < 0 || blk >= p.num_blocks))
                     bad = true;
-                } else {
-                    const int64_t a = max(tok0, pg * bs), z = min(tok0 + n, (pg + 1) * bs);
-                    bytes += (uint32_t)((z - a) * D * 2 * 2);
-                }
             }
-            bad = __any_sync(0xffffffffu, bad);
+            uint32_t bytes = (uint32_t)n * D * 4;
+            if (__any_sync(0xffffffffu, bad)) {
+                uint32_t skip = 0;
+                for (int pc = lane; pc < npieces; pc += 32) {
+                    const int64_t blk = row ? row[pg0 + pc] : it.b;
+                    if (blk < 0 || blk >= p.num_blocks) {
+                        const int pg = pg0 + pc;
+                        skip += (uint32_t)(min((int64_t)tok0 + n, (int64_t)(pg + 1) * bs) -
+                                           max((int64_t)tok0, (int64_t)pg * bs)) * D * 4;
+                    }
+                }
 #pragma unroll
-            for (int o = 16; o; o >>= 1)
-                bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
-            if (lane == 0) {
-                stage_bad[s] = bad ? 1 : 0;
-                stage_n[s] = (int)n;
-                if (bad)
+                for (int o = 16; o; o >>= 1)
+                    skip += __shfl_xor_sync(0xffffffffu, skip, o);
+                bytes -= skip;
+                if (lane == 0)
                     atomicOr(p.status, DEV_BAD_BLOCK);
+            }
+            if (lane == 0) {
+                stage_bad[s] = bytes != (uint32_t)n * D * 4;
+                stage_n[s] = n;
                 mbar_arrive_expect_tx(&full[s], bytes);
             }
             __syncwarp();
+            // Pass 2: issue the copies (K and V rows of each piece).
             for (int pc = lane; pc < npieces; pc += 32) {
-                const int64_t pg = pg0 + pc;
-                const int64_t blk = p.block_table ? p.block_table[(int64_t)it.b * p.max_blocks + pg] : it.b;
-                if (p.block_table && (blk < 0 || blk >= p.num_blocks))
+                const int64_t blk = pc == lane ? blk0 : (row ? row[pg0 + pc] : it.b);
+                if (row && (blk < 0 || blk >= p.num_blocks))
                     continue;
-                const int64_t a = max(tok0, pg * bs), z = min(tok0 + n, (pg + 1) * bs);
-                const int64_t src = ((blk * p.Hkv + it.kvh) * bs + (a - pg * bs)) * D;
-                const int64_t dst = (int64_t)s * C::TILE_ELEMS + (a - tok0) * D;
-                const uint32_t nb = (uint32_t)((z - a) * D * 2);
+                const int pg = pg0 + pc;
+                const int a = max(tok0, pg * bs);
+                const int z = (int)min((int64_t)tok0 + n, (int64_t)(pg + 1) * bs);
+                const int64_t src = ((blk * p.Hkv + it.kvh) * (int64_t)bs + (a - pg * bs)) * D;
+                const int dst = s * C::TILE_ELEMS + (a - tok0) * D;
+                const uint32_t nb = (uint32_t)(z - a) * D * 2;
                 bulk_copy_g2s(kring + dst, p.k + src, nb, &full[s], pol);
                 bulk_copy_g2s(vring + dst, p.v + src, nb, &full[s], pol);
             }
         }
         // Never leave copies in flight: wait for the last issued phase of each slot.
         if (lane == 0) {
-            for (int64_t kk = max((int64_t)0, k - C::STAGES); kk < k; ++kk) {
-                const int s = (int)(kk % C::STAGES);
+            for (int kk = max(0, k - C::STAGES); kk < k; ++kk) {
+                const int s = kk % C::STAGES;
                 const uint32_t ph = (uint32_t)((kk / C::STAGES) & 1);
                 const uint64_t t0 = global_timer_ns();
                 while (!mbar_try_wait(&full[s], ph) && global_timer_ns() - t0 < WAIT_LIMIT_NS) {
@@ -290,7 +308,7 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
     it.init(start, prefix, B, units, p.hch);
     cur = it;
     int64_t piece_first = start;
-    int64_t k = 0;
+    int k = 0;
 
     for (int64_t i = start; i < end; ++i, ++k) {
         if (i > start)
@@ -318,7 +336,7 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
             }
         }
 
-        const int s = (int)(k % C::STAGES);
+        const int s = k % C::STAGES;
         const uint32_t ph = (uint32_t)((k / C::STAGES) & 1);
         const bool ready = bounded_wait(&full[s], ph, abort_flag, p.status);
         if (!ready) {

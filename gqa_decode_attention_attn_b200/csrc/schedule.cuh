@@ -45,9 +45,21 @@ struct Params {
     int B, Hq, Hkv, G, block_size, max_blocks, num_blocks;
     int hch;                      // head chunks per KV head
     int64_t capacity;             // tokens a request can hold
+    uint32_t bs_magic;            // token -> page division by block_size (see page_of)
+    int bs_shift;
     float qscale;                 // scale * log2(e): scores are kept in log2 units
     unsigned long long *timeline; // optional [grid][4]: start ns, end ns, SM id, tiles
 };
+
+// floor(t / block_size) for 0 <= t < 2^31 without a divide: with l = ceil(log2 bs)
+// and m = floor(2^32 (2^l - bs) / bs) + 1 (computed on the host),
+// floor(t / bs) = (umulhi(m, t) + t) >> l (division by an invariant integer,
+// Granlund & Montgomery 1994).
+__device__ __forceinline__ int page_of(const Params &p, int t)
+{
+    const uint32_t u = (uint32_t)t;
+    return (int)((__umulhi(p.bs_magic, u) + u) >> p.bs_shift);
+}
 
 // Walks the global tile order one tile at a time.  prefix[b] = sum of n_b'
 // (b' < b) lives in shared memory; units = Hkv * hch segments per request.  Only
