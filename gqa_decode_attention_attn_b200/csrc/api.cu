@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "decode_simt.cuh"
+#include "decode_tc.cuh"
 #include "gqa_decode.h"
 #include "merge_states.cuh"
 
@@ -83,7 +84,7 @@ struct DeviceGeom {
 std::mutex g_mu;
 DeviceGeom g_dev[MAX_DEVICES];
 struct FnGeom {
-    KernelFn fn;
+    const void *fn;
     int device;
     int ctas_per_sm;
 };
@@ -96,7 +97,7 @@ int current_device(int &dev)
 }
 
 // Persistent grid for a kernel on a device: SMs x resident CTAs per SM.
-int persistent_ctas(const Variant &v, int dev, int &ctas)
+int persistent_ctas_fn(const void *fn, int threads, size_t smem_max, int dev, int &ctas)
 {
     std::lock_guard<std::mutex> lock(g_mu);
     if (dev < 0 || dev >= MAX_DEVICES)
@@ -109,7 +110,7 @@ int persistent_ctas(const Variant &v, int dev, int &ctas)
         g_dev[dev].ready = true;
     }
     for (int i = 0; i < g_nfn; ++i) {
-        if (g_fn[i].fn == v.fn && g_fn[i].device == dev) {
+        if (g_fn[i].fn == fn && g_fn[i].device == dev) {
             ctas = g_dev[dev].sms * g_fn[i].ctas_per_sm;
             return GQA_OK;
         }
@@ -120,18 +121,90 @@ int persistent_ctas(const Variant &v, int dev, int &ctas)
     if (prev != dev && cudaSetDevice(dev) != cudaSuccess)
         return GQA_ERR_CUDA;
     int per_sm = 0;
-    cudaError_t e = cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)v.smem_max);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem_max);
     if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.fn, v.threads, v.smem_max);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem_max);
     if (prev != dev)
         cudaSetDevice(prev);
     if (e != cudaSuccess || per_sm < 1)
         return GQA_ERR_CUDA;
     if (g_nfn < 256)
-        g_fn[g_nfn++] = FnGeom{v.fn, dev, per_sm};
+        g_fn[g_nfn++] = FnGeom{fn, dev, per_sm};
     ctas = g_dev[dev].sms * per_sm;
     return GQA_OK;
+}
+
+int persistent_ctas(const Variant &v, int dev, int &ctas)
+{
+    return persistent_ctas_fn(reinterpret_cast<const void *>(v.fn), v.threads, v.smem_max, dev,
+                              ctas);
+}
+
+int tc_ctas(int dev, int &ctas)
+{
+    return persistent_ctas_fn(reinterpret_cast<const void *>(gqa_decode_tc_kernel), TcCfg::THREADS,
+                              TcCfg::smem_bytes(TcCfg::MAX_BATCH), dev, ctas);
+}
+
+// ---- tensor-core path: applicability and tensor maps -------------------------
+
+// Tokens per TMA box along the cache rows: one box per page, 128 for big pages.
+int tc_box_rows(const int32_t *block_table, int block_size)
+{
+    if (!block_table)
+        return 128;
+    if (block_size >= 128)
+        return block_size % 128 == 0 ? 128 : 0;
+    return (block_size >= 8 && 128 % block_size == 0) ? block_size : 0;
+}
+
+bool tc_applicable(bool states, int B, int Hq, int Hkv, int D, int block_size,
+                   const int32_t *block_table, int num_blocks)
+{
+    if (states || D != TcCfg::D || Hq / Hkv < 8 || B > TcCfg::MAX_BATCH)
+        return false;
+    if (tc_box_rows(block_table, block_size) == 0)
+        return false;
+    const int64_t blocks = block_table ? num_blocks : B;
+    const int64_t rows = blocks * Hkv * (int64_t)block_size;
+    return rows > 0 && rows < (int64_t(1) << 31);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 2-D view of a cache as [rows, 128] bf16; boxes of 64 columns x box_rows rows,
+// 128-byte swizzle (the layout the tensor cores read), zero fill out of range.
+bool encode_kv_map(CUtensorMap *map, const void *base, int64_t rows, int box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)TcCfg::D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)TcCfg::D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 struct WorkspaceLayout {
@@ -191,16 +264,17 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || (out && !aligned16(out)))
         return GQA_ERR_MISALIGNED;
     const int G = Hq / Hkv;
+    const bool use_tc = tc_applicable(states, B, Hq, Hkv, D, block_size, block_table, num_blocks);
     Variant v;
-    if (!pick_variant(D, G, states, v))
+    if (!use_tc && !pick_variant(D, G, states, v))
         return GQA_ERR_UNSUPPORTED;
     int dev = 0;
     if ((rc = current_device(dev)))
         return rc;
     int ctas = 0;
-    if ((rc = persistent_ctas(v, dev, ctas)))
+    if ((rc = use_tc ? tc_ctas(dev, ctas) : persistent_ctas(v, dev, ctas)))
         return rc;
-    const WorkspaceLayout w = layout_for(ctas, v.slot_floats);
+    const WorkspaceLayout w = layout_for(ctas, use_tc ? TcCfg::SLOT_FLOATS : v.slot_floats);
     if (workspace_bytes < w.total)
         return GQA_ERR_WORKSPACE_TOO_SMALL;
 
@@ -227,7 +301,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     p.block_size = block_size;
     p.max_blocks = block_table ? max_blocks : 1;
     p.num_blocks = block_table ? num_blocks : B;
-    p.hch = (G + head_chunk(G) - 1) / head_chunk(G);
+    p.hch = use_tc ? (G + TcCfg::NP - 1) / TcCfg::NP : (G + head_chunk(G) - 1) / head_chunk(G);
     p.capacity = block_table ? (int64_t)max_blocks * block_size : (int64_t)block_size;
     p.qscale = scale * LOG2E;
     p.timeline = nullptr;
@@ -241,7 +315,17 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         p.bs_shift = l;
     }
 
-    v.fn<<<ctas, v.threads, v.smem(B), static_cast<cudaStream_t>(stream)>>>(p);
+    if (use_tc) {
+        const int box_rows = tc_box_rows(block_table, block_size);
+        const int64_t rows = (block_table ? (int64_t)num_blocks : (int64_t)B) * Hkv * block_size;
+        CUtensorMap tmk, tmv;
+        if (!encode_kv_map(&tmk, k_cache, rows, box_rows) || !encode_kv_map(&tmv, v_cache, rows, box_rows))
+            return GQA_ERR_CUDA;
+        gqa_decode_tc_kernel<<<ctas, TcCfg::THREADS, TcCfg::smem_bytes(B),
+                               static_cast<cudaStream_t>(stream)>>>(p, tmk, tmv, box_rows);
+    } else {
+        v.fn<<<ctas, v.threads, v.smem(B), static_cast<cudaStream_t>(stream)>>>(p);
+    }
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
@@ -268,6 +352,13 @@ int gqa_decode_workspace_size(int B, int Hq, int Hkv, int D, int device, size_t 
         if ((rc = persistent_ctas(v, device, ctas)))
             return rc;
         const size_t t = layout_for(ctas, v.slot_floats).total;
+        best = t > best ? t : best;
+    }
+    if (D == TcCfg::D && Hq / Hkv >= 8) {
+        int ctas = 0;
+        if ((rc = tc_ctas(device, ctas)))
+            return rc;
+        const size_t t = layout_for(ctas, TcCfg::SLOT_FLOATS).total;
         best = t > best ? t : best;
     }
     *bytes = best;

@@ -65,24 +65,6 @@ struct SimtCfg {
     static_assert(2 * STAGES <= 24, "flag area");
 };
 
-// Writes one finished output element (and, in states mode, m and l).
-template <bool STATES>
-__device__ __forceinline__ void write_result(const Params &p, int64_t row, int d, int D, float a,
-                                             float ms, float ls, bool poisoned)
-{
-    if (STATES) {
-        p.st_acc[row * D + d] = poisoned ? __int_as_float(0x7fc00000) : a;
-        if (d == 0) {
-            p.st_m[row] = ms == -INFINITY ? -INFINITY : ms * 0.69314718055994531f;
-            p.st_l[row] = poisoned ? __int_as_float(0x7fc00000) : ls;
-        }
-    } else {
-        float o = poisoned ? __int_as_float(0x7fc00000) : (ls > 0.f ? a / ls : 0.f);
-        __nv_bfloat16 h = __float2bfloat16_rn(o);
-        p.out[row * D + d] = *reinterpret_cast<uint16_t *>(&h);
-    }
-}
-
 // Transposed butterfly: NV partial sums per lane, reduced across the LPT lanes of
 // a token.  While a lane still holds two or more values, each level hands half of
 // them to the partner and keeps the other half (one shuffle per kept value);

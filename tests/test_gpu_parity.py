@@ -62,6 +62,13 @@ SMALL = [
     (2, 4, 1, 128, [70, 70], 1),                        # one-token pages
     (2, 4, 2, 128, [101, 55], 3),                       # pages not a power of two
     (2, 4, 2, 128, [1000, 999], 100),
+    # tensor-core path (D = 128, G >= 8): pages of 8..256 tokens, ragged tiles
+    (3, 16, 2, 128, [129, 1, 300], 8),
+    (2, 24, 2, 128, [511, 130], 32),                    # G = 12: padded head chunk
+    (2, 32, 1, 128, [1000, 127], 128),                  # G = 32: two head chunks
+    (1, 16, 1, 128, [700], 256),
+    (2, 8, 1, 128, [5000, 3000], None),                 # contiguous, capacity 5005
+    (4, 64, 4, 128, [2048, 2047, 1, 130], 16),
 ]
 
 
