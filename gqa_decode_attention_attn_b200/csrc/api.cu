@@ -112,6 +112,8 @@ int persistent_ctas_fn(const void *fn, int threads, size_t smem_max, int dev, in
     for (int i = 0; i < g_nfn; ++i) {
         if (g_fn[i].fn == fn && g_fn[i].device == dev) {
             ctas = g_dev[dev].sms * g_fn[i].ctas_per_sm;
+            if (ctas > 512)
+                ctas = 512;
             return GQA_OK;
         }
     }
@@ -132,6 +134,8 @@ int persistent_ctas_fn(const void *fn, int threads, size_t smem_max, int dev, in
     if (g_nfn < 256)
         g_fn[g_nfn++] = FnGeom{fn, dev, per_sm};
     ctas = g_dev[dev].sms * per_sm;
+    if (ctas > 512)  // merge scratch is sized for at most 512 persistent CTAs
+        ctas = 512;
     return GQA_OK;
 }
 
@@ -208,7 +212,7 @@ bool encode_kv_map(CUtensorMap *map, const void *base, int64_t rows, int box_row
 }
 
 struct WorkspaceLayout {
-    size_t counters_off, slots_off, total;
+    size_t counters_off, gcounters_off, slots_off, total;
 };
 
 // Fixed layout: [status | ticket counters for the largest shape | partial-state
@@ -216,12 +220,14 @@ struct WorkspaceLayout {
 // touches is either still zero from allocation or was reset by the call that last
 // used it; slots of one call can never alias counters of another.
 constexpr size_t COUNTERS_BYTES = sizeof(int) * (size_t)GQA_MAX_BATCH * GQA_MAX_QHEADS;
+constexpr size_t GCOUNTERS_BYTES = sizeof(int) * 2 * 512;  // one per slot of <= 512 CTAs
 
 WorkspaceLayout layout_for(int ctas, int slot_floats)
 {
     WorkspaceLayout w;
     w.counters_off = STATUS_BYTES;
-    w.slots_off = w.counters_off + COUNTERS_BYTES;
+    w.gcounters_off = w.counters_off + COUNTERS_BYTES;
+    w.slots_off = w.gcounters_off + GCOUNTERS_BYTES;
     w.total = align_up(w.slots_off + sizeof(float) * 2 * (size_t)ctas * slot_floats, 256);
     return w;
 }
@@ -293,6 +299,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     p.st_l = l;
     p.status = reinterpret_cast<unsigned *>(ws);
     p.counters = reinterpret_cast<int *>(ws + w.counters_off);
+    p.gcounters = reinterpret_cast<int *>(ws + w.gcounters_off);
     p.slots = reinterpret_cast<float *>(ws + w.slots_off);
     p.B = B;
     p.Hq = Hq;
@@ -412,7 +419,7 @@ int gqa_status(void *workspace, void *stream, unsigned *device_error)
     if (cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
         return GQA_ERR_CUDA;
     // After a device error some tickets may be left mid-count: clear them too.
-    if (v && cudaMemset(workspace, 0, STATUS_BYTES + COUNTERS_BYTES) != cudaSuccess)
+    if (v && cudaMemset(workspace, 0, STATUS_BYTES + COUNTERS_BYTES + GCOUNTERS_BYTES) != cudaSuccess)
         return GQA_ERR_CUDA;
     *device_error = v;
     return GQA_OK;
@@ -569,10 +576,13 @@ extern "C" int gqa_decode_noalloc(const void *q, const void *k_cache, const void
         return rc;
     if (need > NOALLOC_SCRATCH_BYTES)
         return GQA_ERR_SCRATCH_LIMIT;
-    // The status word and the ticket counters this call can touch must start at
-    // zero; a previous call that hit a device error may have left them set.
+    // The status word and the ticket counters this call can touch (per segment and
+    // per CTA group) must start at zero; a previous call that hit a device error
+    // may have left them set.
     const size_t clear = STATUS_BYTES + sizeof(int) * (size_t)B * Hq;
-    if (cudaMemsetAsync(scratch, 0, clear, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (cudaMemsetAsync(scratch, 0, clear, static_cast<cudaStream_t>(stream)) != cudaSuccess ||
+        cudaMemsetAsync(static_cast<unsigned char *>(scratch) + STATUS_BYTES + COUNTERS_BYTES, 0,
+                        GCOUNTERS_BYTES, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return GQA_ERR_CUDA;
     return gqa_decode(q, k_cache, v_cache, block_table, seq_lens, out, B, Hq, Hkv, D, block_size,
                       scale, max_blocks_per_seq, num_blocks, scratch, NOALLOC_SCRATCH_BYTES, stream);

@@ -36,14 +36,17 @@ namespace gqa {
 
 template <int D, int GC>
 struct SimtCfg {
-    static constexpr int NC = 8;                       // consumer warps
+    // 7 consumer warps + 1 producer = 256 threads: the register allocator grants
+    // up to 255 registers per thread only to CTAs of at most 256 threads, and each
+    // warp needs ~200 to keep 8 steps (16 tokens at D = 128) in flight per tile.
+    static constexpr int NC = 7;                       // consumer warps
     static constexpr int THREADS = (NC + 1) * 32;
-    static constexpr int T = 32768 / (4 * D);          // tokens per tile: 32 KB of K+V
-    static constexpr int STAGES = 4;
+    static constexpr int STEPS = 8;                    // warp steps per tile
     static constexpr int LPT = D / 8;                  // lanes per token (16 B each)
     static constexpr int TPW = 32 / LPT;               // tokens per warp step
-    static constexpr int TOKW = T / NC;                // tokens per warp per tile
-    static constexpr int STEPS = TOKW / TPW;           // warp steps per tile
+    static constexpr int TOKW = STEPS * TPW;           // tokens per warp per tile
+    static constexpr int T = NC * TOKW;                // tokens per tile: 56 KB of K+V
+    static constexpr int STAGES = (D == 256 && GC == 8) ? 2 : 3;  // shared-memory budget
     static constexpr int NV = STEPS * GC;              // partial dots per lane
     static constexpr int NF = NV >= LPT ? NV / LPT : 1;  // whole scores per lane
     static constexpr int REP = NV >= LPT ? 1 : LPT / NV; // lanes sharing one score
@@ -57,12 +60,15 @@ struct SimtCfg {
     static constexpr size_t FLAG_OFF = BAR_OFF + 2 * STAGES * sizeof(uint64_t);
     static constexpr size_t SCRATCH_OFF = FLAG_OFF + 32 * sizeof(int);
     static constexpr size_t PSCR_OFF = SCRATCH_OFF + (size_t)NC * SCRATCH_PER_WARP * sizeof(float);
-    static constexpr size_t PREFIX_OFF = PSCR_OFF + (size_t)NC * PSCR_PER_WARP * sizeof(float);
-    static constexpr int SLOT_FLOATS = GC * (D + 2);   // one partial state
+    static constexpr size_t MSCR_OFF = PSCR_OFF + (size_t)NC * PSCR_PER_WARP * sizeof(float);
+    static constexpr size_t PREFIX_OFF =
+        MSCR_OFF + (size_t)merge_scratch_floats(GC, NC * 32, 512) * sizeof(float);
+    static constexpr int SLOT_FLOATS = slot_floats(GC, D);  // one partial state
     static size_t smem_bytes(int B) { return PREFIX_OFF + (size_t)(B + 1) * sizeof(int); }
     static_assert(STEPS >= 1 && TOKW % TPW == 0, "tile must split evenly over warps");
     static_assert(32 % GC == 0 && GC <= 8, "head chunk must divide the warp");
     static_assert(2 * STAGES <= 24, "flag area");
+    static_assert(PREFIX_OFF + (4096 + 1) * sizeof(int) <= 232448, "shared memory at the largest batch");
 };
 
 // Transposed butterfly: NV partial sums per lane, reduced across the LPT lanes of
@@ -106,8 +112,10 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
     volatile int *abort_flag = stage_bad + 24;
     int *last_flag = stage_bad + 25;
     int *poison_flag = stage_bad + 26;
+    int *merge_flags = stage_bad + 28;                              // [4]
     float *scratch = reinterpret_cast<float *>(smem + C::SCRATCH_OFF);
     float *pscr = reinterpret_cast<float *>(smem + C::PSCR_OFF);
+    float *mscr = reinterpret_cast<float *>(smem + C::MSCR_OFF);
     int *prefix = reinterpret_cast<int *>(smem + C::PREFIX_OFF);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -514,73 +522,10 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
         named_barrier_sync(1, C::NC * 32);
 
         if (!complete) {
-            if (ctid == 0) {
+            if (ctid == 0)
                 *poison_flag = 0;
-                __threadfence();
-                const int ntiles = (int)(i + 1 - piece_first);
-                const int old = atomicAdd(&p.counters[vseg], ntiles);
-                *last_flag = (old + ntiles == cur.nb) ? 1 : 0;
-            }
-            named_barrier_sync(1, C::NC * 32);
-            if (*reinterpret_cast<volatile int *>(last_flag)) {
-                __threadfence();
-                const int64_t seg1 = cur.seg0 + cur.nb;
-                const int64_t c0 = tile_owner(cur.seg0, W, P), c1 = tile_owner(seg1 - 1, W, P);
-                // Pass 1: common maximum per head (thread g < GC), via shared memory.
-                float *mstar = scratch;  // the warp states are no longer needed
-                if (ctid < GC) {
-                    float ms = -INFINITY;
-                    RunWalker rw(c0, W, P);
-                    for (int64_t cc = c0; cc <= c1; ++cc) {
-                        const int64_t s0 = rw.start();
-                        rw.next();
-                        if (s0 == rw.start())
-                            continue;
-                        const float *sl = p.slots + (2 * cc + (s0 < cur.seg0 ? 1 : 0)) * (int64_t)C::SLOT_FLOATS;
-                        ms = fmaxf(ms, __ldcg(sl + GC * D + ctid));
-                    }
-                    mstar[ctid] = ms;
-                }
-                named_barrier_sync(1, C::NC * 32);
-                // Pass 2: weighted sums, pieces in CTA order.
-                constexpr int EPT = (GC * D + C::NC * 32 - 1) / (C::NC * 32);
-                float a[EPT], ls[EPT];
-#pragma unroll
-                for (int x = 0; x < EPT; ++x) {
-                    a[x] = 0.f;
-                    ls[x] = 0.f;
-                }
-                RunWalker rw(c0, W, P);
-                for (int64_t cc = c0; cc <= c1; ++cc) {
-                    const int64_t s0 = rw.start();
-                    rw.next();
-                    if (s0 == rw.start())
-                        continue;
-                    const float *sl = p.slots + (2 * cc + (s0 < cur.seg0 ? 1 : 0)) * (int64_t)C::SLOT_FLOATS;
-#pragma unroll
-                    for (int x = 0; x < EPT; ++x) {
-                        const int e = ctid + x * C::NC * 32;
-                        if (e >= GC * D)
-                            continue;
-                        const int g = e / D, d = e - (e / D) * D;
-                        const float mw = __ldcg(sl + GC * D + g);
-                        const float wt = mw == -INFINITY ? 0.f : fast_exp2(mw - mstar[g]);
-                        a[x] = fmaf(wt, __ldcg(sl + g * D + d), a[x]);
-                        ls[x] = fmaf(wt, __ldcg(sl + GC * D + GC + g), ls[x]);
-                    }
-                }
-#pragma unroll
-                for (int x = 0; x < EPT; ++x) {
-                    const int e = ctid + x * C::NC * 32;
-                    if (e >= GC * D)
-                        continue;
-                    const int g = e / D, d = e - (e / D) * D;
-                    if (g < rows)
-                        write_result<STATES>(p, row0 + g, d, D, a[x], mstar[g], ls[x], ls[x] != ls[x]);
-                }
-                if (ctid == 0)
-                    p.counters[vseg] = 0;
-            }
+            finish_partial<GC, D, C::NC * 32, STATES>(p, c, cur.seg0, cur.nb, piece_first, i + 1, vseg,
+                                                      W, P, rows, row0, mscr, merge_flags, ctid, 1);
         } else if (ctid == 0) {
             *poison_flag = 0;
         }

@@ -4,15 +4,19 @@
 //
 // Same LeanTile schedule as the CUDA-core kernel (schedule.cuh): each CTA walks a
 // contiguous run of 128-token tiles of (request, KV head, 16-head chunk) segments.
-// Roles (one CTA per SM, 6 warps):
-//   warp 0     TMA: each tile's K and V rows arrive as 128-byte-swizzled boxes
-//              (one per page, two 64-column halves) into a 3-stage ring.
+// Roles (one CTA per SM, 7 warps):
+//   warps 0, 6 TMA: each tile's K rows (warp 0) and V rows (warp 6) arrive as
+//              128-byte-swizzled boxes (one per page, two 64-column halves) into
+//              separate 3-slot rings: a K slot frees as soon as BMM1 has read it,
+//              a V slot only after BMM2, so K loads run further ahead.
 //   warp 1     MMA (one thread): BMM1  S^T[128 x 16] = K[128 x 128] . Q^T, with K
 //              and Q K-major; BMM2  O^T[128 x 16] = V^T . P^T, with V read
 //              MN-major straight from the swizzled TMA boxes and P from shared
-//              memory.  P is passed as two bf16 terms (hi + lo, so that P itself
-//              carries ~16 significant bits) and BMM2 accumulates both.
-//              Accumulators live in tensor memory, two buffers each.
+//              memory.  P is passed as two bf16 terms, hi and lo, so that P itself
+//              carries ~16 significant bits: they are the two halves of one
+//              N = 32 operand, since an MMA of N <= 128 costs the tensor pipe the
+//              same ~90 cycles whatever N is.  Accumulators live in tensor
+//              memory, two buffers each.
 //   warps 2-5  softmax + correction (thread = TMEM lane): read S rows, take the
 //              tile maximum per head across the 128 tokens, update the running
 //              maximum lazily (only when it grows by more than 2^8), write
@@ -31,30 +35,36 @@
 namespace gqa {
 
 struct TcCfg {
+    // (merge scratch lives in the P buffers: checked below)
     static constexpr int D = 128, T = 128, NP = 16;  // head dim, tile tokens, heads per MMA
-    static constexpr int STAGES = 3;
-    static constexpr int THREADS = 192;
+    static constexpr int STAGES = 3;                   // slots per ring (K ring, V ring)
+    static constexpr int THREADS = 224;
     static constexpr int BOX_BYTES = T * 128;          // one 64-column half of a tile: 16 KB
     static constexpr int TILE_BYTES = 2 * BOX_BYTES;   // K or V tile
-    static constexpr int STAGE_BYTES = 2 * TILE_BYTES; // K + V
+    static constexpr int V_RING_OFF = STAGES * TILE_BYTES;
     static constexpr int QBUF_BYTES = 2 * NP * 128;    // two halves, NP rows of 128 B
-    static constexpr int P_LBO = (NP / 8) * 128;       // P: stride between 8-token groups
+    static constexpr int NO = 2 * NP;                  // BMM2 columns: P_hi heads, P_lo heads
+    static constexpr int P_LBO = (NO / 8) * 128;       // P: stride between 8-token groups
     static constexpr int PBUF_BYTES = (T / 8) * P_LBO;
-    static constexpr int TMEM_COLS = 4 * NP;           // S x2, O x2
+    static constexpr int S_COL = 0, O_COL = 2 * NP;    // TMEM columns: S x2, O x2 (NO wide)
+    static constexpr int TMEM_COLS = 128;              // >= 2 * NP + 2 * NO, power of two
     static constexpr float LAZY = 8.f;                 // rescale only when max grows > 2^8
-    static constexpr size_t Q_OFF = (size_t)STAGES * STAGE_BYTES;
+    static constexpr size_t Q_OFF = (size_t)2 * STAGES * TILE_BYTES;
     static constexpr size_t P_OFF = Q_OFF + 2 * QBUF_BYTES;
-    static constexpr size_t BAR_OFF = P_OFF + 4 * PBUF_BYTES;  // [buffer][hi, lo]
-    static constexpr int NBAR = 2 * STAGES + 13;
+    static constexpr size_t BAR_OFF = P_OFF + 2 * PBUF_BYTES;
+    static constexpr int NBAR = 4 * STAGES + 13;
     static constexpr size_t MISC_OFF = BAR_OFF + NBAR * 8;
     // floats: tile maxima [2][4][NP], piece sums [4][NP], merge maxima [NP]
     static constexpr size_t RED_OFF = MISC_OFF + 64 * 4;
     static constexpr size_t PREFIX_OFF = RED_OFF + 13 * NP * 4 + 64;
-    static constexpr int SLOT_FLOATS = NP * (D + 2);
+    static constexpr int SLOT_FLOATS = slot_floats(NP, D);
     static constexpr int MAX_BATCH = 1024;
     // +1024: the dynamic shared-memory base is re-aligned to 1024 bytes in-kernel.
     static size_t smem_bytes(int B) { return PREFIX_OFF + (size_t)(B + 1) * sizeof(int) + 1024; }
 };
+static_assert(merge_scratch_floats(TcCfg::NP, 128, 512) * 4 <= 2 * TcCfg::PBUF_BYTES,
+              "merge scratch must fit in the P buffers");
+static_assert(TcCfg::O_COL + 2 * TcCfg::NO <= TcCfg::TMEM_COLS, "tensor memory columns");
 
 // Max or sum of NV per-lane values across the 32 lanes of a warp, transposed so
 // that lane l ends with the result for index l / (32 / NV) (NV <= 32).
@@ -94,8 +104,8 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     unsigned char *qbuf = smem + C::Q_OFF;
     unsigned char *pbuf = smem + C::P_OFF;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
-    uint64_t *kv_full = bars, *kv_empty = bars + S;
-    uint64_t *s_full = bars + 2 * S, *s_free = s_full + 2, *p_full = s_free + 2;
+    uint64_t *k_full = bars, *k_empty = bars + S, *v_full = bars + 2 * S, *v_empty = bars + 3 * S;
+    uint64_t *s_full = bars + 4 * S, *s_free = s_full + 2, *p_full = s_free + 2;
     uint64_t *o_full = p_full + 2, *o_free = o_full + 2, *q_full = o_free + 2, *drain = q_full + 2;
     int *misc = reinterpret_cast<int *>(smem + C::MISC_OFF);
     int *stage_n = misc, *stage_bad = misc + 8;
@@ -111,8 +121,10 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
             stage_bad[s] = 0;
         }
         for (int b = 0; b < 2; ++b) {
@@ -179,8 +191,12 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             write_result<false>(p, (int64_t)b * p.Hq + e / D, e % D, D, 0.f, -INFINITY, 0.f, bad);
     }
 
-    if (start < end && warp == 0) {
+    if (start < end && (warp == 0 || warp == 6)) {
         // ---------------------------------------------------------------- TMA
+        const bool is_k = warp == 0;
+        const CUtensorMap *map = is_k ? &tmk : &tmv;
+        unsigned char *base = ring + (is_k ? 0 : C::V_RING_OFF);
+        uint64_t *full = is_k ? k_full : v_full, *emptyb = is_k ? k_empty : v_empty;
         const uint64_t pol = l2_evict_first_policy();
         TileIter it;
         it.init(start, prefix, B, units, p.hch);
@@ -190,7 +206,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 it.next(prefix, B, p.Hkv, p.hch);
             const int s = k % S;
             const uint32_t ph = (uint32_t)((k / S) & 1);
-            if (k >= S && !bounded_wait(&kv_empty[s], ph ^ 1u, abort_flag, p.status))
+            if (k >= S && !bounded_wait(&emptyb[s], ph ^ 1u, abort_flag, p.status))
                 break;
             if (it.b != cur_b) {
                 cur_b = it.b;
@@ -216,26 +232,29 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             }
             const unsigned badmask = __ballot_sync(0xffffffffu, bad);
             if (lane == 0) {
-                stage_n[s] = n;
-                stage_bad[s] = badmask != 0;
-                if (badmask)
-                    atomicOr(p.status, DEV_BAD_BLOCK);
+                // Tile metadata travels with the V slot: a V slot is recycled only
+                // after every softmax thread has posted this tile's P, while a K
+                // slot may be refilled before a slow softmax thread looks at it.
+                if (!is_k) {
+                    stage_n[s] = n;
+                    stage_bad[s] = badmask != 0;
+                    if (badmask)
+                        atomicOr(p.status, DEV_BAD_BLOCK);
+                }
                 const uint32_t boxes = (uint32_t)(nbox - __popc(badmask));
-                mbar_arrive_expect_tx(&kv_full[s], boxes * 4u * (uint32_t)box_rows * 128u);
+                mbar_arrive_expect_tx(&full[s], boxes * 2u * (uint32_t)box_rows * 128u);
             }
             __syncwarp();
             if (lane < nbox && !bad) {
-                unsigned char *kd = ring + (size_t)s * C::STAGE_BYTES + (size_t)lane * box_rows * 128;
-                tma_load_2d(kd, &tmk, 0, row, &kv_full[s], pol);
-                tma_load_2d(kd + C::BOX_BYTES, &tmk, 64, row, &kv_full[s], pol);
-                tma_load_2d(kd + C::TILE_BYTES, &tmv, 0, row, &kv_full[s], pol);
-                tma_load_2d(kd + C::TILE_BYTES + C::BOX_BYTES, &tmv, 64, row, &kv_full[s], pol);
+                unsigned char *d = base + (size_t)s * C::TILE_BYTES + (size_t)lane * box_rows * 128;
+                tma_load_2d(d, map, 0, row, &full[s], pol);
+                tma_load_2d(d + C::BOX_BYTES, map, 64, row, &full[s], pol);
             }
         }
         if (lane == 0) {
             for (int kk = max(0, k - S); kk < k; ++kk) {
                 const uint64_t t0 = global_timer_ns();
-                while (!mbar_try_wait(&kv_full[kk % S], (uint32_t)((kk / S) & 1)) &&
+                while (!mbar_try_wait(&full[kk % S], (uint32_t)((kk / S) & 1)) &&
                        global_timer_ns() - t0 < WAIT_LIMIT_NS) {
                 }
             }
@@ -244,7 +263,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         // ---------------------------------------------------------------- MMA
         if (lane == 0) {
             const uint32_t idesc1 = umma_idesc_bf16(128, NP, 0, 0);
-            const uint32_t idesc2 = umma_idesc_bf16(128, NP, 1, 1);
+            const uint32_t idesc2 = umma_idesc_bf16(128, C::NO, 1, 1);
             const uint32_t ring_a = smem_addr(ring), q_a = smem_addr(qbuf), p_a = smem_addr(pbuf);
             const int ntiles = (int)(end - start);
             TileIter it1;
@@ -260,46 +279,45 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                     ++piece1;
                 }
                 const int s = k % S, b = k & 1, qb = (piece1 - 1) & 1;
-                ok = ok && bounded_wait(&kv_full[s], (uint32_t)((k / S) & 1), abort_flag, p.status);
+                ok = ok && bounded_wait(&k_full[s], (uint32_t)((k / S) & 1), abort_flag, p.status);
                 if (k >= 2)
                     ok = ok && bounded_wait(&s_free[b], (uint32_t)(((k - 2) >> 1) & 1), abort_flag, p.status);
                 ok = ok && bounded_wait(&q_full[qb], (uint32_t)(((piece1 - 1) >> 1) & 1), abort_flag, p.status);
                 if (!ok)
                     return;
                 tc_fence_after_sync();
-                const uint32_t ka = ring_a + (uint32_t)(s * C::STAGE_BYTES);
+                const uint32_t ka = ring_a + (uint32_t)(s * C::TILE_BYTES);
                 const uint32_t qa = q_a + (uint32_t)(qb * C::QBUF_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (uint32_t)((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32);
                     const uint32_t qoff = (uint32_t)((kk >> 2) * NP * 128 + (kk & 3) * 32);
-                    umma_bf16(tbase + (uint32_t)(b * NP), umma_smem_desc(ka + off, 16, 1024, SMEM_LAYOUT_SW128),
+                    umma_bf16(tbase + (uint32_t)(C::S_COL + b * NP), umma_smem_desc(ka + off, 16, 1024, SMEM_LAYOUT_SW128),
                               umma_smem_desc(qa + qoff, 16, 1024, SMEM_LAYOUT_SW128), idesc1, kk > 0);
                 }
                 umma_commit(&s_full[b]);
+                umma_commit(&k_empty[s]);
             };
             auto mma2 = [&](int k) {
                 const int s = k % S, b = k & 1;
                 ok = ok && bounded_wait(&p_full[b], (uint32_t)((k >> 1) & 1), abort_flag, p.status);
+                ok = ok && bounded_wait(&v_full[s], (uint32_t)((k / S) & 1), abort_flag, p.status);
                 if (k >= 2)
                     ok = ok && bounded_wait(&o_free[b], (uint32_t)(((k - 2) >> 1) & 1), abort_flag, p.status);
                 if (!ok)
                     return;
                 tc_fence_after_sync();
-                const uint32_t va = ring_a + (uint32_t)(s * C::STAGE_BYTES + C::TILE_BYTES);
+                const uint32_t va = ring_a + (uint32_t)(C::V_RING_OFF + s * C::TILE_BYTES);
+                const uint32_t pa = p_a + (uint32_t)(b * C::PBUF_BYTES);
 #pragma unroll
-                for (int part = 0; part < 2; ++part) {
-                    const uint32_t pa = p_a + (uint32_t)((2 * b + part) * C::PBUF_BYTES);
-#pragma unroll
-                    for (int kk = 0; kk < T / 16; ++kk) {
-                        umma_bf16(tbase + (uint32_t)(2 * NP + b * NP),
-                                  umma_smem_desc(va + (uint32_t)(kk * 2048), C::BOX_BYTES, 1024, SMEM_LAYOUT_SW128),
-                                  umma_smem_desc(pa + (uint32_t)(2 * kk * C::P_LBO), C::P_LBO, 128, SMEM_LAYOUT_NONE),
-                                  idesc2, (part | kk) > 0);
-                    }
+                for (int kk = 0; kk < T / 16; ++kk) {
+                    umma_bf16(tbase + (uint32_t)(C::O_COL + b * C::NO),
+                              umma_smem_desc(va + (uint32_t)(kk * 2048), C::BOX_BYTES, 1024, SMEM_LAYOUT_SW128),
+                              umma_smem_desc(pa + (uint32_t)(2 * kk * C::P_LBO), C::P_LBO, 128, SMEM_LAYOUT_NONE),
+                              idesc2, kk > 0);
                 }
                 umma_commit(&o_full[b]);
-                umma_commit(&kv_empty[s]);
+                umma_commit(&v_empty[s]);
             };
             mma1(0);
             for (int k = 0; k < ntiles && ok; ++k) {
@@ -333,9 +351,14 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             const int bc = kc & 1;
             float o[NP];
             if (ok && bounded_wait(&o_full[bc], (uint32_t)((kc >> 1) & 1), abort_flag, p.status)) {
+                float olo[NP];
                 tc_fence_after_sync();
-                tmem_load16(tlane + (uint32_t)(2 * NP + bc * NP), o);
+                tmem_load16(tlane + (uint32_t)(C::O_COL + bc * C::NO), o);
+                tmem_load16(tlane + (uint32_t)(C::O_COL + bc * C::NO + NP), olo);
                 tc_fence_before_sync();
+#pragma unroll
+                for (int g = 0; g < NP; ++g)
+                    o[g] += olo[g];
             } else {
                 ok = false;
                 poisoned = true;
@@ -395,61 +418,12 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             }
             named_barrier_sync(1, 128);
             if (!complete) {
-                if (stid == 0) {
+                if (stid == 0)
                     *poison_flag = 0;
-                    __threadfence();
-                    const int ntiles = (int)(last_excl - piece_first);
-                    const int old = atomicAdd(&p.counters[vseg], ntiles);
-                    *last_flag = (old + ntiles == cur.nb) ? 1 : 0;
-                }
-                named_barrier_sync(1, 128);
-                if (*reinterpret_cast<volatile int *>(last_flag)) {
-                    __threadfence();
-                    const int64_t seg1 = cur.seg0 + cur.nb;
-                    const int64_t c0 = tile_owner(cur.seg0, W, P), c1 = tile_owner(seg1 - 1, W, P);
-                    float *mstar = red + 12 * NP;
-                    if (stid < NP) {
-                        float ms = -INFINITY;
-                        RunWalker rw(c0, W, P);
-                        for (int64_t cc = c0; cc <= c1; ++cc) {
-                            const int64_t s0 = rw.start();
-                            rw.next();
-                            if (s0 == rw.start())
-                                continue;
-                            const float *sl = p.slots + (2 * cc + (s0 < cur.seg0 ? 1 : 0)) * (int64_t)C::SLOT_FLOATS;
-                            ms = fmaxf(ms, __ldcg(sl + NP * D + stid));
-                        }
-                        mstar[stid] = ms;
-                    }
-                    named_barrier_sync(1, 128);
-                    float a[NP], ls[NP];
-#pragma unroll
-                    for (int g = 0; g < NP; ++g) {
-                        a[g] = 0.f;
-                        ls[g] = 0.f;
-                    }
-                    RunWalker rw(c0, W, P);
-                    for (int64_t cc = c0; cc <= c1; ++cc) {
-                        const int64_t s0 = rw.start();
-                        rw.next();
-                        if (s0 == rw.start())
-                            continue;
-                        const float *sl = p.slots + (2 * cc + (s0 < cur.seg0 ? 1 : 0)) * (int64_t)C::SLOT_FLOATS;
-#pragma unroll
-                        for (int g = 0; g < NP; ++g) {
-                            const float mw = __ldcg(sl + NP * D + g);
-                            const float wt = mw == -INFINITY ? 0.f : fast_exp2(mw - mstar[g]);
-                            a[g] = fmaf(wt, __ldcg(sl + g * D + ti), a[g]);
-                            ls[g] = fmaf(wt, __ldcg(sl + NP * D + NP + g), ls[g]);
-                        }
-                    }
-#pragma unroll
-                    for (int g = 0; g < NP; ++g)
-                        if (g < rows)
-                            write_result<false>(p, row0 + g, ti, D, a[g], mstar[g], ls[g], ls[g] != ls[g]);
-                    if (stid == 0)
-                        p.counters[vseg] = 0;
-                }
+                // The P buffers are idle between pieces: merge scratch.
+                finish_partial<NP, D, 128, false>(p, c, cur.seg0, cur.nb, piece_first, last_excl, vseg,
+                                                  W, P, rows, row0, reinterpret_cast<float *>(pbuf),
+                                                  misc + 20, stid, 1);
             } else if (stid == 0) {
                 *poison_flag = 0;
             }
@@ -502,12 +476,12 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             const int s = k % S, b = k & 1;
             float sc[NP];
             int n = 0;
-            if (ok && bounded_wait(&kv_full[s], (uint32_t)((k / S) & 1), abort_flag, p.status) &&
+            if (ok && bounded_wait(&v_full[s], (uint32_t)((k / S) & 1), abort_flag, p.status) &&
                 bounded_wait(&s_full[b], (uint32_t)((k >> 1) & 1), abort_flag, p.status)) {
                 n = stage_n[s];
                 poisoned |= stage_bad[s] != 0;
                 tc_fence_after_sync();
-                tmem_load16(tlane + (uint32_t)(b * NP), sc);
+                tmem_load16(tlane + (uint32_t)(C::S_COL + b * NP), sc);
                 tc_fence_before_sync();
             } else {
                 ok = false;
@@ -537,9 +511,10 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 pr[g] = (valid && m_new != -INFINITY) ? fast_exp2(sc[g] - m_new) : 0.f;
                 l_t[g] = fmaf(l_t[g], alpha[g], pr[g]);
             }
-            // P = hi + lo, both bf16, in the no-swizzle MN-major layout: token ti's
-            // 8-head groups are 16-byte rows of 8x8 core matrices.
-            unsigned char *pd = pbuf + 2 * b * C::PBUF_BYTES + (ti >> 3) * C::P_LBO + (ti & 7) * 16;
+            // P = hi + lo, both bf16, as one N = 32 operand (hi heads, then lo
+            // heads) in the no-swizzle MN-major layout: token ti's 8-head groups
+            // are 16-byte rows of 8x8 core matrices.
+            unsigned char *pd = pbuf + b * C::PBUF_BYTES + (ti >> 3) * C::P_LBO + (ti & 7) * 16;
 #pragma unroll
             for (int ng = 0; ng < NP / 8; ++ng) {
                 uint32_t whi[4], wlo[4];
@@ -553,13 +528,13 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                     wlo[j] = *reinterpret_cast<uint32_t *>(&lo);
                 }
                 *reinterpret_cast<uint4 *>(pd + ng * 128) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
-                *reinterpret_cast<uint4 *>(pd + C::PBUF_BYTES + ng * 128) =
+                *reinterpret_cast<uint4 *>(pd + (NP / 8 + ng) * 128) =
                     make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
             }
             // Rows past the valid tokens may hold anything (stale tiles, poison):
             // zero this token's V row so that 0-weight rows add exact zeros.
             if (!valid) {
-                unsigned char *vr = ring + (size_t)s * C::STAGE_BYTES + C::TILE_BYTES + ti * 128;
+                unsigned char *vr = ring + C::V_RING_OFF + (size_t)s * C::TILE_BYTES + ti * 128;
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
 #pragma unroll

@@ -43,6 +43,7 @@ struct Params {
     float *st_l;                  // [B, Hq]
     unsigned *status;             // device status word
     int *counters;                // one ticket per segment
+    int *gcounters;               // one ticket per CTA-group merge (index: leader slot)
     float *slots;                 // 2 partial states per CTA
     int B, Hq, Hkv, G, block_size, max_blocks, num_blocks;
     int hch;                      // head chunks per KV head
@@ -201,6 +202,254 @@ __device__ __forceinline__ void write_result(const Params &p, int64_t row, int d
         float o = poisoned ? __int_as_float(0x7fc00000) : (ls > 0.f ? a / ls : 0.f);
         __nv_bfloat16 h = __float2bfloat16_rn(o);
         p.out[row * D + d] = *reinterpret_cast<uint16_t *>(&h);
+    }
+}
+
+
+// Slot of one partial state: acc [NH][D], then m [NH] and l [NH] (log2 units),
+// padded to a 16-byte multiple so float4 loads stay aligned.
+__host__ __device__ constexpr int slot_floats(int NH, int D) { return NH * D + ((2 * NH + 3) / 4) * 4; }
+
+// ---------------------------------------------------------------------------
+// Exact merge of partial pieces (LeanAttention decode tiles digest, section
+// "Exact softmax that merges piece by piece"): every piece keeps its own maximum,
+// normaliser and weighted values; rescaling all of them to the common maximum and
+// adding is exact in any order.  Pieces are combined in CTA order, so the result
+// does not depend on which CTA arrived last.
+//
+// Two levels, so that no single CTA reads every piece of a long segment: the
+// owners of a segment are grouped by MERGE_GROUP consecutive CTAs; the last
+// arriver of each group merges the group's pieces into the slot of the group's
+// first owner, then takes the segment ticket; the last group merger combines the
+// group results (one group: it writes the output directly).
+constexpr int MERGE_GROUP = 8;
+
+__host__ __device__ constexpr int merge_chunk() { return 32; }
+__host__ __device__ constexpr int merge_scratch_floats(int NP, int NT, int P)
+{
+    return 2 * NP + 2 * merge_chunk() * NP + NT + P + 8;
+}
+
+// Merges the n slots listed in `list` (shared memory).  dst_slot == nullptr: the
+// result goes to output rows row0 .. row0 + rows - 1; otherwise into dst_slot (a
+// partial state again, log2 units).  NT threads t, named barrier bar_id; scr has
+// merge_scratch_floats() floats.
+template <int NP, int D, int NT, bool STATES>
+__device__ __forceinline__ void merge_slots(const Params &p, const int *list, int n,
+                                            float *dst_slot, int rows, int64_t row0, float *scr,
+                                            int t, int bar_id)
+{
+    constexpr int SF = slot_floats(NP, D);
+    constexpr int OC = merge_chunk();
+    float *mstar = scr;                  // [NP]
+    float *lsum = mstar + NP;            // [NP]
+    float *wch = lsum + NP;              // [OC][NP] weights of a chunk of pieces
+    float *lch = wch + OC * NP;          // [OC][NP] their weighted normalisers
+    float *red = lch + OC * NP;          // [NT]
+    {
+        const int g = t % NP;
+        float mx = -INFINITY;
+        for (int o = t / NP; o < n; o += NT / NP)
+            mx = fmaxf(mx, __ldcg(p.slots + (int64_t)list[o] * SF + NP * D + g));
+        red[t] = mx;
+        named_barrier_sync(bar_id, NT);
+        if (t < NP) {
+            float m = -INFINITY;
+            for (int x = t; x < NT - NT % NP; x += NP)
+                m = fmaxf(m, red[x]);
+            mstar[t] = m;
+            lsum[t] = 0.f;
+        }
+        named_barrier_sync(bar_id, NT);
+    }
+    constexpr int NF4 = NP * D / 4;                  // float4 outputs
+    constexpr int R = (NF4 + NT - 1) / NT;
+    constexpr int U = R >= 4 ? 4 : 8 / R;            // pieces whose loads are in flight together
+    float4 acc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+        acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int base = 0; base < n; base += OC) {
+        const int nc = min(OC, n - base);
+        for (int x = t; x < nc * NP; x += NT) {
+            const int o = x / NP, g = x % NP;
+            const float *sl = p.slots + (int64_t)list[base + o] * SF;
+            const float mw = __ldcg(sl + NP * D + g);
+            const float w = mw == -INFINITY ? 0.f : fast_exp2(mw - mstar[g]);
+            wch[o * NP + g] = w;
+            lch[o * NP + g] = w * __ldcg(sl + NP * D + NP + g);
+        }
+        named_barrier_sync(bar_id, NT);
+        if (t < NP) {
+            float ls = lsum[t];
+            for (int o = 0; o < nc; ++o)
+                ls += lch[o * NP + t];
+            lsum[t] = ls;
+        }
+        for (int o0 = 0; o0 < nc; o0 += U) {
+            float4 v[U][R];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const bool have = o0 + u < nc;
+                const float4 *sl = reinterpret_cast<const float4 *>(
+                    p.slots + (int64_t)(have ? list[base + o0 + u] : list[base]) * SF);
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const int f = t + r * NT;
+                    v[u][r] = (have && f < NF4) ? __ldcg(sl + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const int f = t + r * NT;
+                    const float w = (o0 + u < nc && f < NF4) ? wch[(o0 + u) * NP + (4 * f) / D] : 0.f;
+                    acc[r].x = fmaf(w, v[u][r].x, acc[r].x);
+                    acc[r].y = fmaf(w, v[u][r].y, acc[r].y);
+                    acc[r].z = fmaf(w, v[u][r].z, acc[r].z);
+                    acc[r].w = fmaf(w, v[u][r].w, acc[r].w);
+                }
+            }
+        }
+        named_barrier_sync(bar_id, NT);
+    }
+    if (dst_slot) {
+        // Every source slot has been read (barrier above): dst may be one of them.
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int f = t + r * NT;
+            if (f < NF4)
+                reinterpret_cast<float4 *>(dst_slot)[f] = acc[r];
+        }
+        if (t < NP) {
+            dst_slot[NP * D + t] = mstar[t];
+            dst_slot[NP * D + NP + t] = lsum[t];
+        }
+        return;
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int f = t + r * NT;
+        if (f >= NF4)
+            continue;
+        const int g = (4 * f) / D, d = (4 * f) % D;
+        if (g >= rows)
+            continue;
+        const float ls = lsum[g], ms = mstar[g];
+        const bool bad = ls != ls;
+        write_result<STATES>(p, row0 + g, d, D, acc[r].x, ms, ls, bad);
+        write_result<STATES>(p, row0 + g, d + 1, D, acc[r].y, ms, ls, bad);
+        write_result<STATES>(p, row0 + g, d + 2, D, acc[r].z, ms, ls, bad);
+        write_result<STATES>(p, row0 + g, d + 3, D, acc[r].w, ms, ls, bad);
+    }
+}
+
+// Slot of CTA cc's piece of the segment starting at tile seg0, or -1 if cc owns
+// no tile (its run is empty).
+__device__ __forceinline__ int piece_slot(int64_t cc, int64_t seg0, int64_t W, int64_t P)
+{
+    const int64_t s0 = run_start(cc, W, P), s1 = run_start(cc + 1, W, P);
+    return s0 == s1 ? -1 : (int)(2 * cc + (s0 < seg0 ? 1 : 0));
+}
+
+// Called by all NT threads after this CTA wrote its partial piece of a segment
+// (tiles [piece_first, piece_end) of [seg0, seg0 + nb)) to its slot.  Takes the
+// group ticket and, for the last arriver of the group, merges the group and
+// takes the segment ticket; the last group merger writes the output.
+// counters: per-segment ticket (index vseg); gcounters: per-group tickets (index =
+// slot of the group's first owner).  Both are left at zero by whoever finishes.
+template <int NP, int D, int NT, bool STATES>
+__device__ __forceinline__ void finish_partial(const Params &p, int64_t c, int64_t seg0, int nb,
+                                               int64_t piece_first, int64_t piece_end,
+                                               int64_t vseg, int64_t W, int64_t P, int rows,
+                                               int64_t row0, float *scr, int *flag, int t,
+                                               int bar_id)
+{
+    // Slot list after the float scratch of merge_slots.
+    int *list = reinterpret_cast<int *>(scr + 2 * NP + 2 * merge_chunk() * NP + NT);
+    const int64_t seg1 = seg0 + nb;
+    // Every thread's slot writes are ordered before the ticket (release).
+    __threadfence();
+    named_barrier_sync(bar_id, NT);
+    const int64_t c0 = tile_owner(seg0, W, P), c1 = tile_owner(seg1 - 1, W, P);
+    const int64_t g = c / MERGE_GROUP;
+    const int64_t ga = max(c0, g * MERGE_GROUP), gb = min(c1, g * MERGE_GROUP + MERGE_GROUP - 1);
+    const bool one_group = c0 / MERGE_GROUP == c1 / MERGE_GROUP;
+    if (t == 0) {
+        // Group ticket (tiles of this segment owned by the group's CTAs).
+        const int64_t gt0 = max(seg0, run_start(ga, W, P)), gt1 = min(seg1, run_start(gb + 1, W, P));
+        int lead = -1;
+        for (int64_t cc = ga; cc <= gb && lead < 0; ++cc)
+            lead = piece_slot(cc, seg0, W, P);
+        __threadfence();
+        const int mine = (int)(piece_end - piece_first);
+        const int old = atomicAdd(&p.gcounters[lead], mine);
+        flag[0] = (old + mine == (int)(gt1 - gt0)) ? 1 : 0;
+        flag[1] = lead;
+        flag[2] = (int)(gt1 - gt0);
+    }
+    named_barrier_sync(bar_id, NT);
+    if (!*reinterpret_cast<volatile int *>(flag))
+        return;
+    __threadfence();
+    const int lead = flag[1], gtiles = flag[2];
+    // Group merge: the group's owners in CTA order.
+    {
+        const int no = (int)(gb - ga + 1);
+        for (int o = t; o < no; o += NT)
+            list[o] = piece_slot(ga + o, seg0, W, P);
+        named_barrier_sync(bar_id, NT);
+        if (t == 0) {
+            int m = 0;
+            for (int o = 0; o < no; ++o)
+                if (list[o] >= 0)
+                    list[m++] = list[o];
+            flag[3] = m;
+        }
+        named_barrier_sync(bar_id, NT);
+        const int m = flag[3];
+        float *dst = one_group ? nullptr : p.slots + (int64_t)lead * slot_floats(NP, D);
+        merge_slots<NP, D, NT, STATES>(p, list, m, dst, rows, row0, scr, t, bar_id);
+        if (t == 0)
+            p.gcounters[lead] = 0;
+    }
+    if (one_group)
+        return;
+    // Segment ticket, counted in tiles; the last group merger combines the groups.
+    __threadfence();
+    named_barrier_sync(bar_id, NT);
+    if (t == 0) {
+        __threadfence();
+        const int old = atomicAdd(&p.counters[vseg], gtiles);
+        flag[0] = (old + gtiles == nb) ? 1 : 0;
+    }
+    named_barrier_sync(bar_id, NT);
+    if (!*reinterpret_cast<volatile int *>(flag))
+        return;
+    __threadfence();
+    {
+        const int64_t g0 = c0 / MERGE_GROUP, g1 = c1 / MERGE_GROUP;
+        const int ng = (int)(g1 - g0 + 1);
+        for (int o = t; o < ng; o += NT) {
+            const int64_t gg = g0 + o;
+            const int64_t a = max(c0, gg * MERGE_GROUP), z = min(c1, gg * MERGE_GROUP + MERGE_GROUP - 1);
+            int s = -1;
+            for (int64_t cc = a; cc <= z && s < 0; ++cc)
+                s = piece_slot(cc, seg0, W, P);
+            list[o] = s;
+        }
+        named_barrier_sync(bar_id, NT);
+        if (t == 0) {
+            int m = 0;
+            for (int o = 0; o < ng; ++o)
+                if (list[o] >= 0)
+                    list[m++] = list[o];
+            flag[3] = m;
+            p.counters[vseg] = 0;
+        }
+        named_barrier_sync(bar_id, NT);
+        merge_slots<NP, D, NT, STATES>(p, list, flag[3], nullptr, rows, row0, scr, t, bar_id);
     }
 }
 

@@ -69,6 +69,10 @@ SMALL = [
     (1, 16, 1, 128, [700], 256),
     (2, 8, 1, 128, [5000, 3000], None),                 # contiguous, capacity 5005
     (4, 64, 4, 128, [2048, 2047, 1, 130], 16),
+    # one long segment spread over every CTA: group merges plus a segment merge
+    (1, 4, 1, 128, [100000], None),
+    (1, 16, 1, 128, [200000], 64),
+    (1, 2, 1, 64, [150000], 16),
 ]
 
 
