@@ -38,8 +38,21 @@ SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 KERNEL_SOURCES = ["gqa_decode_attention_attn_b200/csrc/decode_simt.cuh",
+                  "gqa_decode_attention_attn_b200/csrc/decode_tc.cuh",
                   "gqa_decode_attention_attn_b200/csrc/schedule.cuh",
+                  "gqa_decode_attention_attn_b200/csrc/tc.cuh",
                   "gqa_decode_attention_attn_b200/csrc/ptx.cuh"]
+
+
+def kernel_for(p) -> str:
+    """Which decode kernel the library runs for this problem (mirrors the library's
+    dispatch: tensor cores for D = 128 with at least 8 query heads per KV head and
+    pages that tile into 128-token boxes, CUDA cores otherwise)."""
+    bs = p.block_size
+    boxes = (not p.paged) or (bs % 128 == 0 if bs >= 128 else (bs >= 8 and 128 % bs == 0))
+    if p.D == 128 and p.G >= 8 and p.B <= 1024 and boxes:
+        return "gqa_decode_tc_kernel"
+    return "gqa_decode_simt_kernel"
 
 
 def parse():
@@ -340,7 +353,7 @@ def main():
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
-                         "kernel": "gqa_decode_simt_kernel",
+                         "kernel": kernel_for(p),
                          "algorithmic_bytes_per_launch": bytes_step},
             "gpu_launches": args.steps,
             "timed_region_ms": region_ms,

@@ -299,6 +299,8 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
     cur = it;
     int64_t piece_first = start;
     int k = 0;
+    PendingPiece pending[2];  // a run has at most a first and a last partial piece
+    int npending = 0;
 
     for (int64_t i = start; i < end; ++i, ++k) {
         if (i > start)
@@ -524,11 +526,17 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
         if (!complete) {
             if (ctid == 0)
                 *poison_flag = 0;
-            finish_partial<GC, D, C::NC * 32, STATES>(p, c, cur.seg0, cur.nb, piece_first, i + 1, vseg,
-                                                      W, P, rows, row0, mscr, merge_flags, ctid, 1);
+            pending[npending++] = PendingPiece{cur.seg0, piece_first, i + 1, vseg, row0, cur.nb, rows};
         } else if (ctid == 0) {
             *poison_flag = 0;
         }
+        named_barrier_sync(1, C::NC * 32);
+    }
+
+    for (int x = 0; x < npending; ++x) {
+        const PendingPiece &pp = pending[x];
+        finish_partial<GC, D, C::NC * 32, STATES>(p, c, pp.seg0, pp.nb, pp.first, pp.end, pp.vseg, W,
+                                                  P, pp.rows, pp.row0, mscr, merge_flags, ctid, 1);
         named_barrier_sync(1, C::NC * 32);
     }
 

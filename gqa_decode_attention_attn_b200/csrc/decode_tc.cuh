@@ -339,6 +339,8 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         const uint32_t tlane = tbase + ((uint32_t)(q4 * 32) << 16);
         const float qscale = p.qscale;
         float m_ref[NP], l_t[NP], acc[NP], alpha_prev[NP];
+        PendingPiece pending[2];  // a run has at most a first and a last partial piece
+        int npending = 0;
         bool poisoned = false, pend = false;
         TileIter it, cur;
         it.init(start, prefix, B, units, p.hch);
@@ -420,10 +422,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             if (!complete) {
                 if (stid == 0)
                     *poison_flag = 0;
-                // The P buffers are idle between pieces: merge scratch.
-                finish_partial<NP, D, 128, false>(p, c, cur.seg0, cur.nb, piece_first, last_excl, vseg,
-                                                  W, P, rows, row0, reinterpret_cast<float *>(pbuf),
-                                                  misc + 20, stid, 1);
+                pending[npending++] = PendingPiece{cur.seg0, piece_first, last_excl, vseg, row0, cur.nb, rows};
             } else if (stid == 0) {
                 *poison_flag = 0;
             }
@@ -553,6 +552,14 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         if (pend)
             correction(k - 1);
         epilogue(end);
+        // Tickets and merges after streaming; the P buffers are idle: merge scratch.
+        for (int x = 0; x < npending; ++x) {
+            const PendingPiece &pp = pending[x];
+            finish_partial<NP, D, 128, false>(p, c, pp.seg0, pp.nb, pp.first, pp.end, pp.vseg, W, P,
+                                              pp.rows, pp.row0, reinterpret_cast<float *>(pbuf),
+                                              misc + 20, stid, 1);
+            named_barrier_sync(1, 128);
+        }
     }
 
     // Timeline record and tensor-memory release.

@@ -224,119 +224,96 @@ __host__ __device__ constexpr int slot_floats(int NH, int D) { return NH * D + (
 // group results (one group: it writes the output directly).
 constexpr int MERGE_GROUP = 8;
 
-__host__ __device__ constexpr int merge_chunk() { return 32; }
 __host__ __device__ constexpr int merge_scratch_floats(int NP, int NT, int P)
 {
-    return 2 * NP + 2 * merge_chunk() * NP + NT + P + 8;
+    return P + 8;  // the slot list (ints)
 }
 
-// Merges the n slots listed in `list` (shared memory).  dst_slot == nullptr: the
-// result goes to output rows row0 .. row0 + rows - 1; otherwise into dst_slot (a
-// partial state again, log2 units).  NT threads t, named barrier bar_id; scr has
-// merge_scratch_floats() floats.
+// Merges the n slots listed in `list` (shared memory), in list order.  Every
+// thread owns R float4 outputs and merges them online, four pieces per round
+// trip to L2: load (m, l, acc) of the pieces, raise the running maximum, rescale
+// and add.  No barriers: threads never exchange data.  dst_slot == nullptr: the
+// result goes to output rows row0 .. row0 + rows - 1; otherwise it is written to
+// dst_slot as a partial state again (log2 units); dst_slot may be one of the
+// sources, so every thread finishes reading (barrier bar_id) before any writes.
 template <int NP, int D, int NT, bool STATES>
 __device__ __forceinline__ void merge_slots(const Params &p, const int *list, int n,
-                                            float *dst_slot, int rows, int64_t row0, float *scr,
-                                            int t, int bar_id)
+                                            float *dst_slot, int rows, int64_t row0, int t,
+                                            int bar_id)
 {
     constexpr int SF = slot_floats(NP, D);
-    constexpr int OC = merge_chunk();
-    float *mstar = scr;                  // [NP]
-    float *lsum = mstar + NP;            // [NP]
-    float *wch = lsum + NP;              // [OC][NP] weights of a chunk of pieces
-    float *lch = wch + OC * NP;          // [OC][NP] their weighted normalisers
-    float *red = lch + OC * NP;          // [NT]
-    {
-        const int g = t % NP;
-        float mx = -INFINITY;
-        for (int o = t / NP; o < n; o += NT / NP)
-            mx = fmaxf(mx, __ldcg(p.slots + (int64_t)list[o] * SF + NP * D + g));
-        red[t] = mx;
-        named_barrier_sync(bar_id, NT);
-        if (t < NP) {
-            float m = -INFINITY;
-            for (int x = t; x < NT - NT % NP; x += NP)
-                m = fmaxf(m, red[x]);
-            mstar[t] = m;
-            lsum[t] = 0.f;
-        }
-        named_barrier_sync(bar_id, NT);
-    }
     constexpr int NF4 = NP * D / 4;                  // float4 outputs
     constexpr int R = (NF4 + NT - 1) / NT;
-    constexpr int U = R >= 4 ? 4 : 8 / R;            // pieces whose loads are in flight together
+    constexpr int U = R >= 4 ? 4 : 8 / R;            // pieces per round trip
     float4 acc[R];
+    float mrun[R], lrun[R];
 #pragma unroll
-    for (int r = 0; r < R; ++r)
+    for (int r = 0; r < R; ++r) {
         acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int base = 0; base < n; base += OC) {
-        const int nc = min(OC, n - base);
-        for (int x = t; x < nc * NP; x += NT) {
-            const int o = x / NP, g = x % NP;
-            const float *sl = p.slots + (int64_t)list[base + o] * SF;
-            const float mw = __ldcg(sl + NP * D + g);
-            const float w = mw == -INFINITY ? 0.f : fast_exp2(mw - mstar[g]);
-            wch[o * NP + g] = w;
-            lch[o * NP + g] = w * __ldcg(sl + NP * D + NP + g);
-        }
-        named_barrier_sync(bar_id, NT);
-        if (t < NP) {
-            float ls = lsum[t];
-            for (int o = 0; o < nc; ++o)
-                ls += lch[o * NP + t];
-            lsum[t] = ls;
-        }
-        for (int o0 = 0; o0 < nc; o0 += U) {
-            float4 v[U][R];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const bool have = o0 + u < nc;
-                const float4 *sl = reinterpret_cast<const float4 *>(
-                    p.slots + (int64_t)(have ? list[base + o0 + u] : list[base]) * SF);
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const int f = t + r * NT;
-                    v[u][r] = (have && f < NF4) ? __ldcg(sl + f) : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const int f = t + r * NT;
-                    const float w = (o0 + u < nc && f < NF4) ? wch[(o0 + u) * NP + (4 * f) / D] : 0.f;
-                    acc[r].x = fmaf(w, v[u][r].x, acc[r].x);
-                    acc[r].y = fmaf(w, v[u][r].y, acc[r].y);
-                    acc[r].z = fmaf(w, v[u][r].z, acc[r].z);
-                    acc[r].w = fmaf(w, v[u][r].w, acc[r].w);
-                }
-            }
-        }
-        named_barrier_sync(bar_id, NT);
+        mrun[r] = -INFINITY;
+        lrun[r] = 0.f;
     }
-    if (dst_slot) {
-        // Every source slot has been read (barrier above): dst may be one of them.
+    for (int o0 = 0; o0 < n; o0 += U) {
+        float4 v[U][R];
+        float mv[U][R], lv[U][R];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const bool have = o0 + u < n;
+            const float *sl = p.slots + (int64_t)(have ? list[o0 + u] : list[0]) * SF;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const int f = t + r * NT;
+                const bool ok = have && f < NF4;
+                const int g = ok ? (4 * f) / D : 0;
+                v[u][r] = ok ? __ldcg(reinterpret_cast<const float4 *>(sl) + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+                mv[u][r] = ok ? __ldcg(sl + NP * D + g) : -INFINITY;
+                lv[u][r] = ok ? __ldcg(sl + NP * D + NP + g) : 0.f;
+            }
+        }
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            const int f = t + r * NT;
-            if (f < NF4)
-                reinterpret_cast<float4 *>(dst_slot)[f] = acc[r];
+            float mnew = mrun[r];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                mnew = fmaxf(mnew, mv[u][r]);
+            if (mnew == -INFINITY)
+                continue;  // nothing non-empty yet
+            const float sc = fast_exp2(mrun[r] - mnew);  // exp2(-inf) = 0
+            float4 a = make_float4(acc[r].x * sc, acc[r].y * sc, acc[r].z * sc, acc[r].w * sc);
+            float l = lrun[r] * sc;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const float w = mv[u][r] == -INFINITY ? 0.f : fast_exp2(mv[u][r] - mnew);
+                a.x = fmaf(w, v[u][r].x, a.x);
+                a.y = fmaf(w, v[u][r].y, a.y);
+                a.z = fmaf(w, v[u][r].z, a.z);
+                a.w = fmaf(w, v[u][r].w, a.w);
+                l = fmaf(w, lv[u][r], l);
+            }
+            acc[r] = a;
+            lrun[r] = l;
+            mrun[r] = mnew;
         }
-        if (t < NP) {
-            dst_slot[NP * D + t] = mstar[t];
-            dst_slot[NP * D + NP + t] = lsum[t];
-        }
-        return;
     }
+    if (dst_slot)
+        named_barrier_sync(bar_id, NT);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
         const int f = t + r * NT;
         if (f >= NF4)
             continue;
         const int g = (4 * f) / D, d = (4 * f) % D;
+        if (dst_slot) {
+            reinterpret_cast<float4 *>(dst_slot)[f] = acc[r];
+            if (d == 0) {
+                dst_slot[NP * D + g] = mrun[r];
+                dst_slot[NP * D + NP + g] = lrun[r];
+            }
+            continue;
+        }
         if (g >= rows)
             continue;
-        const float ls = lsum[g], ms = mstar[g];
+        const float ls = lrun[r], ms = mrun[r];
         const bool bad = ls != ls;
         write_result<STATES>(p, row0 + g, d, D, acc[r].x, ms, ls, bad);
         write_result<STATES>(p, row0 + g, d + 1, D, acc[r].y, ms, ls, bad);
@@ -344,6 +321,26 @@ __device__ __forceinline__ void merge_slots(const Params &p, const int *list, in
         write_result<STATES>(p, row0 + g, d + 3, D, acc[r].w, ms, ls, bad);
     }
 }
+
+// Ticket: atomic add with acquire-release semantics at GPU scope.  Called by one
+// thread after a CTA barrier, it publishes every write the CTA made before the
+// barrier (release) and, for the last arriver, makes every other CTA's published
+// writes visible to this CTA after the next barrier (acquire).
+__device__ __forceinline__ int ticket_add(int *counter, int v)
+{
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(counter), "r"(v) : "memory");
+    return old;
+}
+
+// A partial piece whose slot is written and whose ticket is still to be taken.
+// Tickets (and the merges they may trigger) wait until the CTA has streamed all
+// its tiles: the segment cannot complete before its other owners reach the end
+// of their runs anyway, and a merge in mid-run would stall this CTA's pipeline.
+struct PendingPiece {
+    int64_t seg0, first, end, vseg, row0;
+    int nb, rows;
+};
 
 // Slot of CTA cc's piece of the segment starting at tile seg0, or -1 if cc owns
 // no tile (its run is empty).
@@ -366,12 +363,9 @@ __device__ __forceinline__ void finish_partial(const Params &p, int64_t c, int64
                                                int64_t row0, float *scr, int *flag, int t,
                                                int bar_id)
 {
-    // Slot list after the float scratch of merge_slots.
-    int *list = reinterpret_cast<int *>(scr + 2 * NP + 2 * merge_chunk() * NP + NT);
+    int *list = reinterpret_cast<int *>(scr);  // slot list: <= P ints
     const int64_t seg1 = seg0 + nb;
-    // Every thread's slot writes are ordered before the ticket (release).
-    __threadfence();
-    named_barrier_sync(bar_id, NT);
+    named_barrier_sync(bar_id, NT);  // this CTA's slot writes precede the ticket
     const int64_t c0 = tile_owner(seg0, W, P), c1 = tile_owner(seg1 - 1, W, P);
     const int64_t g = c / MERGE_GROUP;
     const int64_t ga = max(c0, g * MERGE_GROUP), gb = min(c1, g * MERGE_GROUP + MERGE_GROUP - 1);
@@ -382,9 +376,8 @@ __device__ __forceinline__ void finish_partial(const Params &p, int64_t c, int64
         int lead = -1;
         for (int64_t cc = ga; cc <= gb && lead < 0; ++cc)
             lead = piece_slot(cc, seg0, W, P);
-        __threadfence();
         const int mine = (int)(piece_end - piece_first);
-        const int old = atomicAdd(&p.gcounters[lead], mine);
+        const int old = ticket_add(&p.gcounters[lead], mine);
         flag[0] = (old + mine == (int)(gt1 - gt0)) ? 1 : 0;
         flag[1] = lead;
         flag[2] = (int)(gt1 - gt0);
@@ -392,7 +385,6 @@ __device__ __forceinline__ void finish_partial(const Params &p, int64_t c, int64
     named_barrier_sync(bar_id, NT);
     if (!*reinterpret_cast<volatile int *>(flag))
         return;
-    __threadfence();
     const int lead = flag[1], gtiles = flag[2];
     // Group merge: the group's owners in CTA order.
     {
@@ -410,24 +402,21 @@ __device__ __forceinline__ void finish_partial(const Params &p, int64_t c, int64
         named_barrier_sync(bar_id, NT);
         const int m = flag[3];
         float *dst = one_group ? nullptr : p.slots + (int64_t)lead * slot_floats(NP, D);
-        merge_slots<NP, D, NT, STATES>(p, list, m, dst, rows, row0, scr, t, bar_id);
+        merge_slots<NP, D, NT, STATES>(p, list, m, dst, rows, row0, t, bar_id);
         if (t == 0)
             p.gcounters[lead] = 0;
     }
     if (one_group)
         return;
     // Segment ticket, counted in tiles; the last group merger combines the groups.
-    __threadfence();
-    named_barrier_sync(bar_id, NT);
+    named_barrier_sync(bar_id, NT);  // the group result precedes the ticket
     if (t == 0) {
-        __threadfence();
-        const int old = atomicAdd(&p.counters[vseg], gtiles);
+        const int old = ticket_add(&p.counters[vseg], gtiles);
         flag[0] = (old + gtiles == nb) ? 1 : 0;
     }
     named_barrier_sync(bar_id, NT);
     if (!*reinterpret_cast<volatile int *>(flag))
         return;
-    __threadfence();
     {
         const int64_t g0 = c0 / MERGE_GROUP, g1 = c1 / MERGE_GROUP;
         const int ng = (int)(g1 - g0 + 1);
@@ -449,7 +438,7 @@ __device__ __forceinline__ void finish_partial(const Params &p, int64_t c, int64
             p.counters[vseg] = 0;
         }
         named_barrier_sync(bar_id, NT);
-        merge_slots<NP, D, NT, STATES>(p, list, flag[3], nullptr, rows, row0, scr, t, bar_id);
+        merge_slots<NP, D, NT, STATES>(p, list, flag[3], nullptr, rows, row0, t, bar_id);
     }
 }
 
