@@ -39,6 +39,7 @@ FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 KERNEL_SOURCES = ["gqa_decode_attention_attn_b200/csrc/decode_simt.cuh",
                   "gqa_decode_attention_attn_b200/csrc/decode_tc.cuh",
+                  "gqa_decode_attention_attn_b200/csrc/gather_merge.cuh",
                   "gqa_decode_attention_attn_b200/csrc/schedule.cuh",
                   "gqa_decode_attention_attn_b200/csrc/tc.cuh",
                   "gqa_decode_attention_attn_b200/csrc/ptx.cuh"]
@@ -46,12 +47,13 @@ KERNEL_SOURCES = ["gqa_decode_attention_attn_b200/csrc/decode_simt.cuh",
 
 def kernel_for(p) -> str:
     """Which decode kernel the library runs for this problem (mirrors the library's
-    dispatch: tensor cores for D = 128 with at least 8 query heads per KV head and
+    dispatch: tensor cores for D = 128 with at least 4 query heads per KV head and
     pages that tile into 128-token boxes, CUDA cores otherwise)."""
     bs = p.block_size
     boxes = (not p.paged) or (bs % 128 == 0 if bs >= 128 else (bs >= 8 and 128 % bs == 0))
-    if p.D == 128 and p.G >= 8 and p.B <= 1024 and boxes:
-        return "gqa_decode_tc_kernel"
+    if p.D == 128 and p.G >= 4 and p.B <= 1024 and boxes:
+        nv = 4 if p.G <= 4 else (8 if p.G <= 8 else 16)
+        return f"gqa_decode_tc_kernel<{nv}>"
     return "gqa_decode_simt_kernel"
 
 

@@ -19,6 +19,9 @@ constexpr int MAX_DEVICES = 64;
 constexpr size_t STATUS_BYTES = 256;
 constexpr float LOG2E = 1.4426950408889634f;
 
+// Smallest group (query heads per KV head) that runs on the tensor-core kernel.
+constexpr int TC_MIN_G = 4;
+
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Query heads per chunk for the CUDA-core kernel: the next power of two >= G,
@@ -145,9 +148,21 @@ int persistent_ctas(const Variant &v, int dev, int &ctas)
                               ctas);
 }
 
-int tc_ctas(int dev, int &ctas)
+// Tensor-core kernel for G query heads per KV head: the softmax carries 4, 8 or
+// 16 heads (the smallest that holds G, capped at the MMA width 16).
+using TcKernelFn = void (*)(Params, CUtensorMap, CUtensorMap, int);
+TcKernelFn tc_kernel_for(int G)
 {
-    return persistent_ctas_fn(reinterpret_cast<const void *>(gqa_decode_tc_kernel), TcCfg::THREADS,
+    if (G <= 4)
+        return gqa_decode_tc_kernel<4>;
+    if (G <= 8)
+        return gqa_decode_tc_kernel<8>;
+    return gqa_decode_tc_kernel<16>;
+}
+
+int tc_ctas(int G, int dev, int &ctas)
+{
+    return persistent_ctas_fn(reinterpret_cast<const void *>(tc_kernel_for(G)), TcCfg::THREADS,
                               TcCfg::smem_bytes(TcCfg::MAX_BATCH), dev, ctas);
 }
 
@@ -166,7 +181,7 @@ int tc_box_rows(const int32_t *block_table, int block_size)
 bool tc_applicable(bool states, int B, int Hq, int Hkv, int D, int block_size,
                    const int32_t *block_table, int num_blocks)
 {
-    if (states || D != TcCfg::D || Hq / Hkv < 8 || B > TcCfg::MAX_BATCH)
+    if (states || D != TcCfg::D || Hq / Hkv < TC_MIN_G || B > TcCfg::MAX_BATCH)
         return false;
     if (tc_box_rows(block_table, block_size) == 0)
         return false;
@@ -278,7 +293,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     if ((rc = current_device(dev)))
         return rc;
     int ctas = 0;
-    if ((rc = use_tc ? tc_ctas(dev, ctas) : persistent_ctas(v, dev, ctas)))
+    if ((rc = use_tc ? tc_ctas(G, dev, ctas) : persistent_ctas(v, dev, ctas)))
         return rc;
     const WorkspaceLayout w = layout_for(ctas, use_tc ? TcCfg::SLOT_FLOATS : v.slot_floats);
     if (workspace_bytes < w.total)
@@ -328,8 +343,21 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         CUtensorMap tmk, tmv;
         if (!encode_kv_map(&tmk, k_cache, rows, box_rows) || !encode_kv_map(&tmv, v_cache, rows, box_rows))
             return GQA_ERR_CUDA;
-        gqa_decode_tc_kernel<<<ctas, TcCfg::THREADS, TcCfg::smem_bytes(B),
-                               static_cast<cudaStream_t>(stream)>>>(p, tmk, tmv, box_rows);
+        // Cooperative launch: the owners of a split segment wait for one another's
+        // pieces, so every CTA of the grid must be resident (the launch fails
+        // rather than run otherwise).
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)ctas);
+        cfg.blockDim = dim3(TcCfg::THREADS);
+        cfg.dynamicSmemBytes = TcCfg::smem_bytes(B);
+        cfg.stream = static_cast<cudaStream_t>(stream);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, tc_kernel_for(G), p, tmk, tmv, box_rows) != cudaSuccess)
+            return GQA_ERR_CUDA;
     } else {
         v.fn<<<ctas, v.threads, v.smem(B), static_cast<cudaStream_t>(stream)>>>(p);
     }
@@ -361,9 +389,9 @@ int gqa_decode_workspace_size(int B, int Hq, int Hkv, int D, int device, size_t 
         const size_t t = layout_for(ctas, v.slot_floats).total;
         best = t > best ? t : best;
     }
-    if (D == TcCfg::D && Hq / Hkv >= 8) {
+    if (D == TcCfg::D && Hq / Hkv >= TC_MIN_G) {
         int ctas = 0;
-        if ((rc = tc_ctas(device, ctas)))
+        if ((rc = tc_ctas(Hq / Hkv, device, ctas)))
             return rc;
         const size_t t = layout_for(ctas, TcCfg::SLOT_FLOATS).total;
         best = t > best ? t : best;

@@ -535,8 +535,11 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
 
     for (int x = 0; x < npending; ++x) {
         const PendingPiece &pp = pending[x];
-        finish_partial<GC, D, C::NC * 32, STATES>(p, c, pp.seg0, pp.nb, pp.first, pp.end, pp.vseg, W,
-                                                  P, pp.rows, pp.row0, mscr, merge_flags, ctid, 1);
+        finish_partial<GC, D, C::NC * 32, STATES>(
+            p, c, pp.seg0, pp.nb, pp.first, pp.end, pp.vseg, W, P, mscr, merge_flags, ctid, 1,
+            [&](const int *list, int n, float *dst) {
+                merge_slots<GC, D, C::NC * 32, STATES>(p, list, n, dst, pp.rows, pp.row0, ctid, 1);
+            });
         named_barrier_sync(1, C::NC * 32);
     }
 

@@ -1,34 +1,40 @@
 // decode_tc.cuh -- persistent stream-K decode attention on the 5th-generation
-// tensor cores (tcgen05), for groups of G >= 8 query heads per KV head where
-// q.K^T is a real dense contraction (M = 128 tokens, N = 16 heads, K = D = 128).
+// tensor cores (tcgen05), for groups of G >= 4 query heads per KV head (D = 128).
+// The MMAs run M = 128 tokens by N = 16 heads; the softmax threads carry only
+// the NV <= 16 heads that exist.
 //
 // Same LeanTile schedule as the CUDA-core kernel (schedule.cuh): each CTA walks a
 // contiguous run of 128-token tiles of (request, KV head, 16-head chunk) segments.
-// Roles (one CTA per SM, 7 warps):
+// Roles (one CTA per SM, 8 warps):
 //   warps 0, 6 TMA: each tile's K rows (warp 0) and V rows (warp 6) arrive as
 //              128-byte-swizzled boxes (one per page, two 64-column halves) into
 //              separate 3-slot rings: a K slot frees as soon as BMM1 has read it,
-//              a V slot only after BMM2, so K loads run further ahead.
-//   warp 1     MMA (one thread): BMM1  S^T[128 x 16] = K[128 x 128] . Q^T, with K
-//              and Q K-major; BMM2  O^T[128 x 16] = V^T . P^T, with V read
-//              MN-major straight from the swizzled TMA boxes and P from shared
-//              memory.  P is passed as two bf16 terms, hi and lo, so that P itself
-//              carries ~16 significant bits: they are the two halves of one
-//              N = 32 operand, since an MMA of N <= 128 costs the tensor pipe the
-//              same ~90 cycles whatever N is.  Accumulators live in tensor
-//              memory, two buffers each.
-//   warps 2-5  softmax + correction (thread = TMEM lane): read S rows, take the
-//              tile maximum per head across the 128 tokens, update the running
-//              maximum lazily (only when it grows by more than 2^8), write
-//              P = exp2(s - m) as bf16, and fold each tile's O into fp32 registers
-//              rescaled by the running-maximum changes.
-// Piece epilogue, partial-state slots and last-arriver merge as in the CUDA-core
-// kernel.  (Attention co-design for long-context inference, sections "FlashAttention
-// and GEMM shapes" and "Effect of group size G": decode GEMM-M equals G; LeanAttention
-// decode tiles digest, sections "Exact softmax that merges piece by piece" and
-// "Hardware-sized work units".)
+//              a V slot only after BMM2.
+//   warp 1     BMM1 (one thread): S^T[128 x 16] = K[128 x 128] . Q^T, K and Q
+//              K-major, into one of two TMEM S buffers.
+//   warp 7     BMM2 (one thread): O^T[128 x 32] += V^T . [P_hi | P_lo]^T, V read
+//              MN-major straight from the swizzled TMA boxes, P from shared
+//              memory as two bf16 terms (hi and lo) so that P carries ~16
+//              significant bits; the two terms are the halves of one N = 32
+//              operand, since an MMA of N <= 128 costs the same ~90 cycles.  O
+//              accumulates in TMEM across tiles while the softmax reference
+//              maximum stays put (two O buffers: one open, one being read back).
+//              Two issuing threads let a late K tile never hold back the BMM2 that
+//              frees a V slot.
+//   warps 2-5  softmax (thread = TMEM lane = token row): read S, and while no
+//              score exceeds the reference maximum by more than 2^8 (one
+//              barrier-OR per tile decides) write P = 2^(s - m) directly; otherwise
+//              take the tile maximum, move the reference, rescale, and have BMM2
+//              close the open O buffer, which is folded into fp32 registers.
+// Pieces: whole segments are written at once; split segments are merged by all
+// of their owners together after streaming (gather_merge.cuh; the launch is
+// cooperative, so every CTA is resident).  (Attention co-design for long-context
+// inference, sections "FlashAttention and GEMM shapes" and "Effect of group size
+// G": decode GEMM-M equals G; LeanAttention decode tiles digest, sections "Exact
+// softmax that merges piece by piece" and "Hardware-sized work units".)
 #pragma once
 
+#include "gather_merge.cuh"
 #include "schedule.cuh"
 #include "tc.cuh"
 
@@ -38,7 +44,7 @@ struct TcCfg {
     // (merge scratch lives in the P buffers: checked below)
     static constexpr int D = 128, T = 128, NP = 16;  // head dim, tile tokens, heads per MMA
     static constexpr int STAGES = 3;                   // slots per ring (K ring, V ring)
-    static constexpr int THREADS = 224;
+    static constexpr int THREADS = 256;
     static constexpr int BOX_BYTES = T * 128;          // one 64-column half of a tile: 16 KB
     static constexpr int TILE_BYTES = 2 * BOX_BYTES;   // K or V tile
     static constexpr int V_RING_OFF = STAGES * TILE_BYTES;
@@ -52,7 +58,7 @@ struct TcCfg {
     static constexpr size_t Q_OFF = (size_t)2 * STAGES * TILE_BYTES;
     static constexpr size_t P_OFF = Q_OFF + 2 * QBUF_BYTES;
     static constexpr size_t BAR_OFF = P_OFF + 2 * PBUF_BYTES;
-    static constexpr int NBAR = 4 * STAGES + 13;
+    static constexpr int NBAR = 4 * STAGES + 16;
     static constexpr size_t MISC_OFF = BAR_OFF + NBAR * 8;
     // floats: tile maxima [2][4][NP], piece sums [4][NP], merge maxima [NP]
     static constexpr size_t RED_OFF = MISC_OFF + 64 * 4;
@@ -62,8 +68,12 @@ struct TcCfg {
     // +1024: the dynamic shared-memory base is re-aligned to 1024 bytes in-kernel.
     static size_t smem_bytes(int B) { return PREFIX_OFF + (size_t)(B + 1) * sizeof(int) + 1024; }
 };
-static_assert(merge_scratch_floats(TcCfg::NP, 128, 512) * 4 <= 2 * TcCfg::PBUF_BYTES,
-              "merge scratch must fit in the P buffers");
+// Segment merge: the owner list (<= 512 ints) in the P buffers; the gathered
+// slices, at most E + no + 3 no (E / D + 2) + 2 NP floats (E <= NP x D outputs,
+// no <= 512 owners), in the rings.
+static_assert(512 * 4 <= 2 * TcCfg::PBUF_BYTES, "owner list must fit in the P buffers");
+static_assert((16 * 128 + 512 + 3 * 512 * (16 + 2) + 32) * 4 <= 2 * TcCfg::STAGES * TcCfg::TILE_BYTES,
+              "gathered slices must fit in the rings");
 static_assert(TcCfg::O_COL + 2 * TcCfg::NO <= TcCfg::TMEM_COLS, "tensor memory columns");
 
 // Max or sum of NV per-lane values across the 32 lanes of a warp, transposed so
@@ -92,12 +102,19 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[NV], int lane)
     return v[0];
 }
 
+// NV: query heads the softmax threads carry (4, 8 or 16 = the MMA width NP);
+// the MMAs always run NP = 16 columns, and columns NV..NP-1 of S and O are
+// never read (zero Q rows in, P left as is: an O column depends on its P column only).
+template <int NV>
 __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     gqa_decode_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv, int box_rows)
 {
     using C = TcCfg;
     constexpr int S = C::STAGES, NP = C::NP, D = C::D, T = C::T;
+    constexpr int SLOT = slot_floats(NV, D);
+    constexpr int LPH = 32 / NV;  // lanes per head after a transposed warp reduction
+    static_assert(NV == 4 || NV == 8 || NV == 16, "softmax head count");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     unsigned char *ring = smem;
@@ -106,12 +123,14 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
     uint64_t *k_full = bars, *k_empty = bars + S, *v_full = bars + 2 * S, *v_empty = bars + 3 * S;
     uint64_t *s_full = bars + 4 * S, *s_free = s_full + 2, *p_full = s_free + 2;
-    uint64_t *o_full = p_full + 2, *o_free = o_full + 2, *q_full = o_free + 2, *drain = q_full + 2;
+    uint64_t *o_full = p_full + 2, *o_free = o_full + 2, *q_full = o_free + 2, *p_free = q_full + 2;
+    uint64_t *drain = p_free + 2;  // two: one per MMA-issuing thread
     int *misc = reinterpret_cast<int *>(smem + C::MISC_OFF);
     int *stage_n = misc, *stage_bad = misc + 8;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 16);
     volatile int *abort_flag = misc + 17;
     int *last_flag = misc + 18, *poison_flag = misc + 19;
+    volatile int *ctl = misc + 28;  // per P buffer: the softmax moved its reference max
     float *red = reinterpret_cast<float *>(smem + C::RED_OFF);
     int *prefix = reinterpret_cast<int *>(smem + C::PREFIX_OFF);
 
@@ -134,8 +153,10 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             mbar_init(&o_full[b], 1);
             mbar_init(&o_free[b], 128);
             mbar_init(&q_full[b], 128);
+            mbar_init(&p_free[b], 1);
         }
-        mbar_init(drain, 1);
+        mbar_init(&drain[0], 1);
+        mbar_init(&drain[1], 1);
         *abort_flag = 0;
         *last_flag = 0;
         *poison_flag = 0;
@@ -259,76 +280,110 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 }
             }
         }
-    } else if (start < end && warp == 1) {
+    } else if (start < end && (warp == 1 || warp == 7)) {
         // ---------------------------------------------------------------- MMA
+        // Two issuing threads: warp 1 issues every BMM1, warp 7 every BMM2, each in
+        // tile order and each waiting (asleep) only for its own operands, so a late
+        // K tile never holds back the BMM2 that frees a V slot.  tcgen05.commit
+        // tracks the MMAs of the committing thread alone.
         if (lane == 0) {
-            const uint32_t idesc1 = umma_idesc_bf16(128, NP, 0, 0);
-            const uint32_t idesc2 = umma_idesc_bf16(128, C::NO, 1, 1);
             const uint32_t ring_a = smem_addr(ring), q_a = smem_addr(qbuf), p_a = smem_addr(pbuf);
             const int ntiles = (int)(end - start);
-            TileIter it1;
-            it1.init(start, prefix, B, units, p.hch);
-            int64_t seg1 = -1;
-            int piece1 = 0;
             bool ok = true;
-            auto mma1 = [&](int k) {
-                if (k > 0)
-                    it1.next(prefix, B, p.Hkv, p.hch);
-                if (it1.seg0 != seg1) {
-                    seg1 = it1.seg0;
-                    ++piece1;
-                }
-                const int s = k % S, b = k & 1, qb = (piece1 - 1) & 1;
-                ok = ok && bounded_wait(&k_full[s], (uint32_t)((k / S) & 1), abort_flag, p.status);
-                if (k >= 2)
-                    ok = ok && bounded_wait(&s_free[b], (uint32_t)(((k - 2) >> 1) & 1), abort_flag, p.status);
-                ok = ok && bounded_wait(&q_full[qb], (uint32_t)(((piece1 - 1) >> 1) & 1), abort_flag, p.status);
-                if (!ok)
-                    return;
-                tc_fence_after_sync();
-                const uint32_t ka = ring_a + (uint32_t)(s * C::TILE_BYTES);
-                const uint32_t qa = q_a + (uint32_t)(qb * C::QBUF_BYTES);
+            if (warp == 1) {
+                const uint32_t idesc1 = umma_idesc_bf16(128, NP, 0, 0);
+                TileIter it1;
+                it1.init(start, prefix, B, units, p.hch);
+                int64_t seg1 = -1;
+                int piece1 = 0;
+                for (int k = 0; k < ntiles && ok; ++k) {
+                    if (k > 0)
+                        it1.next(prefix, B, p.Hkv, p.hch);
+                    if (it1.seg0 != seg1) {
+                        seg1 = it1.seg0;
+                        ++piece1;
+                    }
+                    const int s = k % S, b = k & 1, qb = (piece1 - 1) & 1;
+                    ok = bounded_wait(&k_full[s], (uint32_t)((k / S) & 1), abort_flag, p.status) &&
+                         (k < 2 || bounded_wait(&s_free[b], (uint32_t)(((k - 2) >> 1) & 1), abort_flag, p.status)) &&
+                         bounded_wait(&q_full[qb], (uint32_t)(((piece1 - 1) >> 1) & 1), abort_flag, p.status);
+                    if (!ok)
+                        break;
+                    tc_fence_after_sync();
+                    const uint32_t ka = ring_a + (uint32_t)(s * C::TILE_BYTES);
+                    const uint32_t qa = q_a + (uint32_t)(qb * C::QBUF_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (uint32_t)((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32);
-                    const uint32_t qoff = (uint32_t)((kk >> 2) * NP * 128 + (kk & 3) * 32);
-                    umma_bf16(tbase + (uint32_t)(C::S_COL + b * NP), umma_smem_desc(ka + off, 16, 1024, SMEM_LAYOUT_SW128),
-                              umma_smem_desc(qa + qoff, 16, 1024, SMEM_LAYOUT_SW128), idesc1, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (uint32_t)((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32);
+                        const uint32_t qoff = (uint32_t)((kk >> 2) * NP * 128 + (kk & 3) * 32);
+                        umma_bf16(tbase + (uint32_t)(C::S_COL + b * NP),
+                                  umma_smem_desc(ka + off, 16, 1024, SMEM_LAYOUT_SW128),
+                                  umma_smem_desc(qa + qoff, 16, 1024, SMEM_LAYOUT_SW128), idesc1, kk > 0);
+                    }
+                    umma_commit(&s_full[b]);
+                    umma_commit(&k_empty[s]);
                 }
-                umma_commit(&s_full[b]);
-                umma_commit(&k_empty[s]);
-            };
-            auto mma2 = [&](int k) {
-                const int s = k % S, b = k & 1;
-                ok = ok && bounded_wait(&p_full[b], (uint32_t)((k >> 1) & 1), abort_flag, p.status);
-                ok = ok && bounded_wait(&v_full[s], (uint32_t)((k / S) & 1), abort_flag, p.status);
-                if (k >= 2)
-                    ok = ok && bounded_wait(&o_free[b], (uint32_t)(((k - 2) >> 1) & 1), abort_flag, p.status);
-                if (!ok)
-                    return;
-                tc_fence_after_sync();
-                const uint32_t va = ring_a + (uint32_t)(C::V_RING_OFF + s * C::TILE_BYTES);
-                const uint32_t pa = p_a + (uint32_t)(b * C::PBUF_BYTES);
+            } else {
+                // O accumulates in one TMEM buffer across tiles while the softmax
+                // reference maximum stays put.  A buffer is closed (committed to
+                // o_full) when the softmax moves the reference (ctl flag of the tile)
+                // or when a piece ends; the next tile opens the other buffer afresh.
+                // Closes are counted by `u`: use u lives in buffer u & 1.
+                const uint32_t idesc2 = umma_idesc_bf16(128, C::NO, 1, 1);
+                TileIter itp;
+                itp.init(start, prefix, B, units, p.hch);
+                int64_t segp = itp.seg0;
+                int u = 0;
+                bool fresh = true;
+                for (int k = 0; k < ntiles && ok; ++k) {
+                    const int s = k % S, b = k & 1;
+                    if (!bounded_wait(&p_full[b], (uint32_t)((k >> 1) & 1), abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    if (ctl[b] && !fresh) {
+                        umma_commit(&o_full[u & 1]);
+                        ++u;
+                        fresh = true;
+                    }
+                    ok = (!fresh || u < 2 ||
+                          bounded_wait(&o_free[u & 1], (uint32_t)(((u - 2) >> 1) & 1), abort_flag, p.status)) &&
+                         bounded_wait(&v_full[s], (uint32_t)((k / S) & 1), abort_flag, p.status);
+                    if (!ok)
+                        break;
+                    // Does the piece end with tile k?  (itp runs one tile ahead.)
+                    bool piece_ends = true;
+                    if (k + 1 < ntiles) {
+                        itp.next(prefix, B, p.Hkv, p.hch);
+                        piece_ends = itp.seg0 != segp;
+                        segp = itp.seg0;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t va = ring_a + (uint32_t)(C::V_RING_OFF + s * C::TILE_BYTES);
+                    const uint32_t pa = p_a + (uint32_t)(b * C::PBUF_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < T / 16; ++kk) {
-                    umma_bf16(tbase + (uint32_t)(C::O_COL + b * C::NO),
-                              umma_smem_desc(va + (uint32_t)(kk * 2048), C::BOX_BYTES, 1024, SMEM_LAYOUT_SW128),
-                              umma_smem_desc(pa + (uint32_t)(2 * kk * C::P_LBO), C::P_LBO, 128, SMEM_LAYOUT_NONE),
-                              idesc2, kk > 0);
+                    for (int kk = 0; kk < T / 16; ++kk) {
+                        umma_bf16(tbase + (uint32_t)(C::O_COL + (u & 1) * C::NO),
+                                  umma_smem_desc(va + (uint32_t)(kk * 2048), C::BOX_BYTES, 1024, SMEM_LAYOUT_SW128),
+                                  umma_smem_desc(pa + (uint32_t)(2 * kk * C::P_LBO), C::P_LBO, 128, SMEM_LAYOUT_NONE),
+                                  idesc2, kk > 0 || !fresh);
+                    }
+                    fresh = false;
+                    umma_commit(&v_empty[s]);
+                    umma_commit(&p_free[b]);
+                    if (piece_ends) {
+                        umma_commit(&o_full[u & 1]);
+                        ++u;
+                        fresh = true;
+                    }
                 }
-                umma_commit(&o_full[b]);
-                umma_commit(&v_empty[s]);
-            };
-            mma1(0);
-            for (int k = 0; k < ntiles && ok; ++k) {
-                if (k + 1 < ntiles)
-                    mma1(k + 1);
-                mma2(k);
             }
+            (void)ok;
             // Nothing of ours may still be running on the tensor cores at exit.
-            umma_commit(drain);
+            uint64_t *dr = &drain[warp == 1 ? 0 : 1];
+            umma_commit(dr);
             const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < WAIT_LIMIT_NS) {
+            while (!mbar_try_wait(dr, 0) && global_timer_ns() - t0 < WAIT_LIMIT_NS) {
             }
         }
     } else if (start < end) {
@@ -338,84 +393,93 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         const int stid = tid - 64;               // 0..127 among the softmax threads
         const uint32_t tlane = tbase + ((uint32_t)(q4 * 32) << 16);
         const float qscale = p.qscale;
-        float m_ref[NP], l_t[NP], acc[NP], alpha_prev[NP];
+        // acc holds the closed O buffers, relative to the current reference m_ref
+        // (the open TMEM buffer shares that reference).
+        float m_ref[NV], l_t[NV], acc[NV];
         PendingPiece pending[2];  // a run has at most a first and a last partial piece
         int npending = 0;
-        bool poisoned = false, pend = false;
+        bool poisoned = false;
         TileIter it, cur;
         it.init(start, prefix, B, units, p.hch);
         cur = it;
         int64_t piece_first = start;
-        int piece = 0;
+        int piece = 0, u = 0;
         bool ok = true;
 
-        auto correction = [&](int kc) {
-            const int bc = kc & 1;
-            float o[NP];
-            if (ok && bounded_wait(&o_full[bc], (uint32_t)((kc >> 1) & 1), abort_flag, p.status)) {
-                float olo[NP];
+        // Fold closed O buffer use u (scaled by w[g]) into acc and hand it back.
+        auto fold = [&](const float (&w)[NV]) {
+            const int bc = u & 1;
+            float o[NV];
+            if (ok && bounded_wait(&o_full[bc], (uint32_t)((u >> 1) & 1), abort_flag, p.status)) {
+                float olo[NV];
                 tc_fence_after_sync();
-                tmem_load16(tlane + (uint32_t)(C::O_COL + bc * C::NO), o);
-                tmem_load16(tlane + (uint32_t)(C::O_COL + bc * C::NO + NP), olo);
+                tmem_load<NV>(tlane + (uint32_t)(C::O_COL + bc * C::NO), o);
+                tmem_load<NV>(tlane + (uint32_t)(C::O_COL + bc * C::NO + NP), olo);
                 tc_fence_before_sync();
 #pragma unroll
-                for (int g = 0; g < NP; ++g)
+                for (int g = 0; g < NV; ++g)
                     o[g] += olo[g];
             } else {
                 ok = false;
                 poisoned = true;
 #pragma unroll
-                for (int g = 0; g < NP; ++g)
+                for (int g = 0; g < NV; ++g)
                     o[g] = 0.f;
             }
             mbar_arrive(&o_free[bc]);
+            ++u;
 #pragma unroll
-            for (int g = 0; g < NP; ++g)
-                acc[g] = fmaf(acc[g], alpha_prev[g], o[g]);
+            for (int g = 0; g < NV; ++g)
+                acc[g] = fmaf(o[g], w[g], acc[g]);
         };
 
         auto epilogue = [&](int64_t last_excl) {
-            // Normaliser per head: sum of every token thread's partial.
-            float lv[NP];
+            float one[NV];
 #pragma unroll
-            for (int g = 0; g < NP; ++g)
+            for (int g = 0; g < NV; ++g)
+                one[g] = 1.f;
+            fold(one);
+            // Normaliser per head: sum of every token thread's partial.
+            float lv[NV];
+#pragma unroll
+            for (int g = 0; g < NV; ++g)
                 lv[g] = l_t[g];
-            const float mine = warp_transpose_reduce<NP, false>(lv, lane);
+            const float mine = warp_transpose_reduce<NV, false>(lv, lane);
             float *lred = red + 8 * NP;
-            if ((lane & 1) == 0)
-                lred[q4 * NP + (lane >> 1)] = mine;
+            if (lane % LPH == 0)
+                lred[q4 * NV + lane / LPH] = mine;
             if (poisoned)
                 atomicOr(poison_flag, 1);
             named_barrier_sync(1, 128);
-            float lsum[NP];
+            float lsum[NV];
 #pragma unroll
-            for (int g = 0; g < NP; ++g)
-                lsum[g] = lred[g] + lred[NP + g] + lred[2 * NP + g] + lred[3 * NP + g];
+            for (int g = 0; g < NV; ++g)
+                lsum[g] = lred[g] + lred[NV + g] + lred[2 * NV + g] + lred[3 * NV + g];
             const bool pois = *reinterpret_cast<volatile int *>(poison_flag) != 0;
             const bool complete = piece_first == cur.seg0 && last_excl == cur.seg0 + cur.nb;
-            const int rows = min(NP, G - cur.hc * NP);
+            const int rows = min(NV, G - cur.hc * NP);
             const int64_t row0 = (int64_t)cur.b * p.Hq + (int64_t)cur.kvh * G + (int64_t)cur.hc * NP;
             const int64_t vseg = ((int64_t)cur.b * p.Hkv + cur.kvh) * p.hch + cur.hc;
-            float *slot = p.slots + (2 * c + (piece_first == start ? 0 : 1)) * (int64_t)C::SLOT_FLOATS;
+            float *slot = p.slots + (2 * c + (piece_first == start ? 0 : 1)) * (int64_t)SLOT;
             if (complete) {
 #pragma unroll
-                for (int g = 0; g < NP; ++g)
+                for (int g = 0; g < NV; ++g)
                     if (g < rows)
                         write_result<false>(p, row0 + g, ti, D, acc[g], m_ref[g], lsum[g], pois);
             } else {
 #pragma unroll
-                for (int g = 0; g < NP; ++g)
+                for (int g = 0; g < NV; ++g)
                     slot[g * D + ti] = acc[g];
-                if (ti < NP) {
+                if (ti < NV) {
                     float mv = m_ref[0], lvv = lsum[0];
 #pragma unroll
-                    for (int g = 1; g < NP; ++g)
+                    for (int g = 1; g < NV; ++g)
                         if (g == ti) {
                             mv = m_ref[g];
                             lvv = lsum[g];
                         }
-                    slot[NP * D + ti] = mv;
-                    slot[NP * D + NP + ti] = pois ? __int_as_float(0x7fc00000) : lvv;
+                    slot[NV * D + ti] = mv;
+                    slot[NV * D + NV + ti] = pois ? __int_as_float(0x7fc00000) : lvv;
                 }
             }
             named_barrier_sync(1, 128);
@@ -429,11 +493,23 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             named_barrier_sync(1, 128);
         };
 
+        // A buffer closed by a moved reference is folded one tile later: its close
+        // is committed with the tile's BMM2, which the MMA warp issues only after
+        // the next tile's BMM1, and that may wait for the next piece's Q.
+        float alpha_pend[NV];
+        bool fold_pend = false;
+        auto flush_fold = [&]() {
+            if (fold_pend)
+                fold(alpha_pend);
+            fold_pend = false;
+        };
+
         int k = 0;
         for (int64_t i = start; i < end; ++i, ++k) {
             if (i > start)
                 it.next(prefix, B, p.Hkv, p.hch);
-            if (i == start || it.seg0 != cur.seg0) {
+            const bool first_tile = i == start || it.seg0 != cur.seg0;
+            if (first_tile) {
                 // Q of the new (request, KV head, head chunk) goes out first: the MMA
                 // warp issues this tile's BMM1 before the previous tile's BMM2, and
                 // closing the previous piece below waits on that BMM2.  Layout: the
@@ -455,80 +531,110 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 fence_proxy_async_smem();
                 mbar_arrive(&q_full[(piece - 1) & 1]);
                 if (i > start) {
-                    if (pend)
-                        correction(k - 1);
-                    pend = false;
+                    flush_fold();
                     epilogue(i);
                 }
                 cur = it;
                 piece_first = i;
                 poisoned = false;
 #pragma unroll
-                for (int g = 0; g < NP; ++g) {
+                for (int g = 0; g < NV; ++g) {
                     m_ref[g] = -INFINITY;
                     l_t[g] = 0.f;
                     acc[g] = 0.f;
-                    alpha_prev[g] = 1.f;
                 }
             }
 
             const int s = k % S, b = k & 1;
-            float sc[NP];
+            float sc[NV];
             int n = 0;
             if (ok && bounded_wait(&v_full[s], (uint32_t)((k / S) & 1), abort_flag, p.status) &&
                 bounded_wait(&s_full[b], (uint32_t)((k >> 1) & 1), abort_flag, p.status)) {
                 n = stage_n[s];
                 poisoned |= stage_bad[s] != 0;
                 tc_fence_after_sync();
-                tmem_load16(tlane + (uint32_t)(C::S_COL + b * NP), sc);
+                tmem_load<NV>(tlane + (uint32_t)(C::S_COL + b * NP), sc);
                 tc_fence_before_sync();
             } else {
                 ok = false;
                 poisoned = true;
             }
             mbar_arrive(&s_free[b]);
+            flush_fold();  // before this tile may rescale acc again
             const bool valid = ti < n;
-            float mx[NP];
+            // x = scaled score relative to the reference.  While no score of the tile
+            // exceeds its reference by more than 2^LAZY, P = 2^x <= 2^LAZY is used as
+            // is and nothing is rescaled: one barrier-OR decides that for the CTA.
+            float x[NV];
+            float xmax = -INFINITY;
 #pragma unroll
-            for (int g = 0; g < NP; ++g) {
-                sc[g] = valid ? sc[g] * qscale : -INFINITY;
-                mx[g] = sc[g];
+            for (int g = 0; g < NV; ++g) {
+                x[g] = valid ? fmaf(sc[g], qscale, -m_ref[g]) : -INFINITY;
+                xmax = fmaxf(xmax, x[g]);
             }
-            // Tile maximum per head over the 128 tokens: warp, then the 4 warps.
-            const float wmax = warp_transpose_reduce<NP, true>(mx, lane);
-            float *tred = red + (k & 1) * 4 * NP;
-            if ((lane & 1) == 0)
-                tred[q4 * NP + (lane >> 1)] = wmax;
-            named_barrier_sync(1, 128);
-            float alpha[NP], pr[NP];
+            const bool moved = named_barrier_or(1, 128, !(xmax <= C::LAZY));
+            float alpha[NV];
+            if (moved) {
+                // Tile maximum per head over the 128 tokens: warp, then the 4 warps.
+                float mx[NV];
 #pragma unroll
-            for (int g = 0; g < NP; ++g) {
-                const float tm = fmaxf(fmaxf(tred[g], tred[NP + g]), fmaxf(tred[2 * NP + g], tred[3 * NP + g]));
-                const float m_new = tm > m_ref[g] + C::LAZY ? tm : m_ref[g];
-                alpha[g] = m_new == m_ref[g] ? 1.f : fast_exp2(m_ref[g] - m_new);
-                m_ref[g] = m_new;
-                pr[g] = (valid && m_new != -INFINITY) ? fast_exp2(sc[g] - m_new) : 0.f;
-                l_t[g] = fmaf(l_t[g], alpha[g], pr[g]);
+                for (int g = 0; g < NV; ++g)
+                    mx[g] = valid ? sc[g] * qscale : -INFINITY;
+                const float wmax = warp_transpose_reduce<NV, true>(mx, lane);
+                float *tred = red + (k & 1) * 4 * NP;
+                if (lane % LPH == 0)
+                    tred[q4 * NV + lane / LPH] = wmax;
+                named_barrier_sync(1, 128);
+#pragma unroll
+                for (int g = 0; g < NV; ++g) {
+                    const float tm = fmaxf(fmaxf(tred[g], tred[NV + g]), fmaxf(tred[2 * NV + g], tred[3 * NV + g]));
+                    const float m_new = tm > m_ref[g] + C::LAZY ? tm : m_ref[g];
+                    alpha[g] = m_new == m_ref[g] ? 1.f : fast_exp2(m_ref[g] - m_new);
+                    m_ref[g] = m_new;
+                    x[g] = (valid && m_new != -INFINITY) ? fmaf(sc[g], qscale, -m_new) : -INFINITY;
+                    l_t[g] *= alpha[g];
+                    acc[g] *= alpha[g];
+                }
             }
-            // P = hi + lo, both bf16, as one N = 32 operand (hi heads, then lo
-            // heads) in the no-swizzle MN-major layout: token ti's 8-head groups
-            // are 16-byte rows of 8x8 core matrices.
+            // This P buffer was last read by BMM2 two tiles ago.
+            if (k >= 2 && ok && !bounded_wait(&p_free[b], (uint32_t)(((k - 2) >> 1) & 1), abort_flag, p.status)) {
+                ok = false;
+                poisoned = true;
+            }
+            float pr[NV];
+#pragma unroll
+            for (int g = 0; g < NV; ++g) {
+                pr[g] = fast_exp2(x[g]);
+                l_t[g] += pr[g];
+            }
+            // P = hi + lo, both bf16, as one N = 32 operand (hi heads in columns
+            // 0..NP-1, lo heads in NP..2NP-1) in the no-swizzle MN-major layout:
+            // token ti's 8-head groups are 16-byte rows of 8x8 core matrices.
             unsigned char *pd = pbuf + b * C::PBUF_BYTES + (ti >> 3) * C::P_LBO + (ti & 7) * 16;
+            {
+                constexpr int NW = NV / 2;  // bf16 pairs per term
+                uint32_t whi[NW], wlo[NW];
 #pragma unroll
-            for (int ng = 0; ng < NP / 8; ++ng) {
-                uint32_t whi[4], wlo[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float a = pr[ng * 8 + 2 * j], bb = pr[ng * 8 + 2 * j + 1];
+                for (int j = 0; j < NW; ++j) {
+                    const float a = pr[2 * j], bb = pr[2 * j + 1];
                     __nv_bfloat162 hi = __floats2bfloat162_rn(a, bb);
                     const float2 hf = __bfloat1622float2(hi);
                     __nv_bfloat162 lo = __floats2bfloat162_rn(a - hf.x, bb - hf.y);
                     whi[j] = *reinterpret_cast<uint32_t *>(&hi);
                     wlo[j] = *reinterpret_cast<uint32_t *>(&lo);
                 }
-                *reinterpret_cast<uint4 *>(pd + ng * 128) = make_uint4(whi[0], whi[1], whi[2], whi[3]);
-                *reinterpret_cast<uint4 *>(pd + (NP / 8 + ng) * 128) =
-                    make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
+                if constexpr (NV == 4) {
+                    *reinterpret_cast<uint2 *>(pd) = make_uint2(whi[0], whi[1]);
+                    *reinterpret_cast<uint2 *>(pd + (NP / 8) * 128) = make_uint2(wlo[0], wlo[1]);
+                } else {
+#pragma unroll
+                    for (int ng = 0; ng < NV / 8; ++ng) {
+                        *reinterpret_cast<uint4 *>(pd + ng * 128) =
+                            make_uint4(whi[4 * ng], whi[4 * ng + 1], whi[4 * ng + 2], whi[4 * ng + 3]);
+                        *reinterpret_cast<uint4 *>(pd + (NP / 8 + ng) * 128) =
+                            make_uint4(wlo[4 * ng], wlo[4 * ng + 1], wlo[4 * ng + 2], wlo[4 * ng + 3]);
+                    }
+                }
             }
             // Rows past the valid tokens may hold anything (stale tiles, poison):
             // zero this token's V row so that 0-weight rows add exact zeros.
@@ -540,25 +646,33 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                     for (int cc = 0; cc < 8; ++cc)
                         *reinterpret_cast<uint4 *>(vr + h * C::BOX_BYTES + cc * 16) = make_uint4(0, 0, 0, 0);
             }
+            // A moved reference closes the open O buffer (unless this tile opens a
+            // piece, whose buffer is fresh anyway).
+            const bool close = moved && !first_tile;
+            if (stid == 0)
+                ctl[b] = close ? 1 : 0;
             fence_proxy_async_smem();
             mbar_arrive(&p_full[b]);
-            if (pend)
-                correction(k - 1);
+            if (close) {
 #pragma unroll
-            for (int g = 0; g < NP; ++g)
-                alpha_prev[g] = alpha[g];
-            pend = true;
+                for (int g = 0; g < NV; ++g)
+                    alpha_pend[g] = alpha[g];
+                fold_pend = true;
+            }
         }
-        if (pend)
-            correction(k - 1);
+        flush_fold();
         epilogue(end);
-        // Tickets and merges after streaming; the P buffers are idle: merge scratch.
+        // Split segments: publish every partial piece of this run, then merge this
+        // CTA's share of each (all owners are resident: cooperative launch).  Every
+        // tile has been consumed, so the P buffers and the rings are scratch.
+        for (int x = 0; x < npending; ++x)
+            publish_piece(p, pending[x].vseg, stid, 1, 128);
         for (int x = 0; x < npending; ++x) {
             const PendingPiece &pp = pending[x];
-            finish_partial<NP, D, 128, false>(p, c, pp.seg0, pp.nb, pp.first, pp.end, pp.vseg, W, P,
-                                              pp.rows, pp.row0, reinterpret_cast<float *>(pbuf),
-                                              misc + 20, stid, 1);
-            named_barrier_sync(1, 128);
+            merge_segment_gather<NV, D, 128>(p, c, pp.seg0, pp.nb, pp.first, pp.vseg, W, P, pp.rows,
+                                             pp.row0, reinterpret_cast<int *>(pbuf),
+                                             reinterpret_cast<float *>(ring), misc + 20, stid, 1,
+                                             abort_flag);
         }
     }
 

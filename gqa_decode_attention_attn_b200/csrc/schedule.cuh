@@ -139,14 +139,24 @@ struct RunWalker {
     }
 };
 
+// Quotient of non-negative x by positive y, in 32 bits when both fit (the
+// 64-bit division is several times longer, and the merge tail calls these on
+// its critical path).
+__device__ __forceinline__ int64_t div_nonneg(int64_t x, int64_t y)
+{
+    if ((((uint64_t)x | (uint64_t)y) >> 32) == 0)
+        return (int64_t)((uint32_t)x / (uint32_t)y);
+    return x / y;
+}
+
 // First tile of CTA c, and the CTA whose run holds tile i.
 __device__ __forceinline__ int64_t run_start(int64_t c, int64_t W, int64_t P)
 {
-    return c * W / P;
+    return div_nonneg(c * W, P);
 }
 __device__ __forceinline__ int64_t tile_owner(int64_t i, int64_t W, int64_t P)
 {
-    return ((i + 1) * P - 1) / W;
+    return div_nonneg((i + 1) * P - 1, W);
 }
 
 // Requested key range of request b; returns false for an invalid range.
@@ -356,12 +366,13 @@ __device__ __forceinline__ int piece_slot(int64_t cc, int64_t seg0, int64_t W, i
 // takes the segment ticket; the last group merger writes the output.
 // counters: per-segment ticket (index vseg); gcounters: per-group tickets (index =
 // slot of the group's first owner).  Both are left at zero by whoever finishes.
-template <int NP, int D, int NT, bool STATES>
+// merge(list, n, dst_slot) combines the n listed slots (merge_slots bound to
+// this segment's rows).
+template <int NP, int D, int NT, bool STATES, class MergeFn>
 __device__ __forceinline__ void finish_partial(const Params &p, int64_t c, int64_t seg0, int nb,
                                                int64_t piece_first, int64_t piece_end,
-                                               int64_t vseg, int64_t W, int64_t P, int rows,
-                                               int64_t row0, float *scr, int *flag, int t,
-                                               int bar_id)
+                                               int64_t vseg, int64_t W, int64_t P, float *scr,
+                                               int *flag, int t, int bar_id, MergeFn &&merge)
 {
     int *list = reinterpret_cast<int *>(scr);  // slot list: <= P ints
     const int64_t seg1 = seg0 + nb;
@@ -402,7 +413,7 @@ __device__ __forceinline__ void finish_partial(const Params &p, int64_t c, int64
         named_barrier_sync(bar_id, NT);
         const int m = flag[3];
         float *dst = one_group ? nullptr : p.slots + (int64_t)lead * slot_floats(NP, D);
-        merge_slots<NP, D, NT, STATES>(p, list, m, dst, rows, row0, t, bar_id);
+        merge(list, m, dst);
         if (t == 0)
             p.gcounters[lead] = 0;
     }
@@ -438,7 +449,7 @@ __device__ __forceinline__ void finish_partial(const Params &p, int64_t c, int64
             p.counters[vseg] = 0;
         }
         named_barrier_sync(bar_id, NT);
-        merge_slots<NP, D, NT, STATES>(p, list, flag[3], nullptr, rows, row0, t, bar_id);
+        merge(list, flag[3], static_cast<float *>(nullptr));
     }
 }
 

@@ -85,7 +85,13 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
 
 // 16 consecutive 32-bit columns of this thread's TMEM lane (32x32b shape), and
 // the wait for them, in one statement so no use can be scheduled before the wait.
-__device__ __forceinline__ void tmem_load16(uint32_t taddr, float (&v)[16])
+// N consecutive 32-bit columns of this warp's 32 TMEM lanes (one lane per
+// thread), N = 4, 8 or 16, waiting for the load to complete.
+template <int N>
+__device__ __forceinline__ void tmem_load(uint32_t taddr, float (&v)[N]);
+
+template <>
+__device__ __forceinline__ void tmem_load<16>(uint32_t taddr, float (&v)[16])
 {
     uint32_t r[16];
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
@@ -98,6 +104,35 @@ __device__ __forceinline__ void tmem_load16(uint32_t taddr, float (&v)[16])
                  : "memory");
 #pragma unroll
     for (int i = 0; i < 16; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
+template <>
+__device__ __forceinline__ void tmem_load<8>(uint32_t taddr, float (&v)[8])
+{
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
+template <>
+__device__ __forceinline__ void tmem_load<4>(uint32_t taddr, float (&v)[4])
+{
+    uint32_t r[4];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr)
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
         v[i] = __uint_as_float(r[i]);
 }
 

@@ -86,6 +86,32 @@ def test_small_shapes(case):
     parity(out, ref(p), str(case))
 
 
+# Key outliers move the softmax reference maximum in the middle of a run, also in
+# the last tile of a piece: every rescaling path of both kernels, with many
+# segments and pieces per CTA.
+OUTLIER = [
+    # B, Hq, Hkv, D, lens, block_size, outlier scale
+    (16, 32, 8, 128, [3000] * 16, None, 8.0),
+    (8, 64, 4, 128, [4000, 100, 3000, 7, 5000, 1200, 999, 2500], 16, 8.0),
+    (8, 64, 4, 128, [4000, 100, 3000, 7, 5000, 1200, 999, 2500], 16, 24.0),
+    (2, 32, 2, 128, [60000, 30000], 64, 16.0),
+    (6, 8, 1, 128, [2000, 1, 4097, 640, 130, 9000], 32, 16.0),
+    (1, 16, 1, 128, [100000], None, 24.0),
+    (4, 16, 4, 64, [5000, 3000, 1, 700], 16, 16.0),
+]
+
+
+@pytest.mark.parametrize("case", OUTLIER,
+                         ids=lambda c: f"B{c[0]}_Hq{c[1]}_Hkv{c[2]}_D{c[3]}_bs{c[5]}_x{c[6]:g}")
+def test_key_outliers_rescale(case):
+    B, Hq, Hkv, D, lens, bs, xs = case
+    p = make_problem("outliers", B, Hq, Hkv, D, lens, seed=300 + sum(lens) + int(xs), block_size=bs,
+                     key_outlier_frac=0.02, key_outlier_scale=xs)
+    out = run(p)
+    torch.cuda.synchronize()
+    parity(out, ref(p), str(case), bf16_scaled=True)
+
+
 def test_empty_batch_and_all_empty_requests():
     p = make_problem("empty", 3, 4, 1, 128, [0, 0, 0], seed=5, block_size=16)
     out = run(p)
