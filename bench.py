@@ -66,6 +66,13 @@ def parse():
     ap.add_argument("--workload", default="llama3_8b", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--schedule", choices=["auto", "streamk", "fixed"], default="auto",
+                    help="auto: gqa_decode_auto (the library's runtime schedule selection); "
+                         "streamk: gqa_decode; fixed: the fixed-split comparator "
+                         "(gqa_decode_fixed_split) with --splits chunks per segment")
+    ap.add_argument("--splits", type=int, default=0,
+                    help="chunks per segment for --schedule fixed (0: enough chunks for "
+                         "one CTA per SM, FlashDecoding's usual choice)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target duration of the CPU-baseline sample")
     return ap.parse_args()
@@ -288,9 +295,29 @@ def main():
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    splits = 0
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    lens_host = p.seq_lens.to(torch.int32).contiguous()
+    if args.schedule == "fixed":
+        segs = p.B * p.Hkv * -(-p.G // 16)
+        splits = args.splits if args.splits > 0 else max(1, -(-sms // segs))
+        schedule = f"fixed-split x{splits}"
+    elif args.schedule == "auto":
+        chosen, _ = gq.select_schedule(lens_host, p.Hq, p.Hkv, p.D, sms, max_splits=1)
+        schedule = "auto: one CTA per (request, KV head)" if chosen else "auto: stream-K"
+    else:
+        schedule = "stream-K"
+
     def step():
-        gq.gqa_decode(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens, out=out,
-                      scale=p.scale, workspace=ws, stream=stream)
+        if splits:
+            gq.gqa_decode_fixed_split(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,
+                                      splits, out=out, scale=p.scale, workspace=ws, stream=stream)
+        elif args.schedule == "auto":
+            gq.gqa_decode_auto(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens, lens_host,
+                               out=out, scale=p.scale, workspace=ws, stream=stream)
+        else:
+            gq.gqa_decode(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens, out=out,
+                          scale=p.scale, workspace=ws, stream=stream)
 
     for _ in range(max(3, args.warmup)):
         flush.fill_(1)
@@ -351,16 +378,18 @@ def main():
             "pct_of_spec_8tbs": 100.0 * achieved / SPEC_HBM_GBS,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 q/K/V; no trained weights)",
-            "config": workload_config(p),
+            "config": dict(workload_config(p), schedule=schedule),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
                          "kernel": kernel_for(p),
                          "algorithmic_bytes_per_launch": bytes_step},
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * (2 if splits > 1 else 1),
             "timed_region_ms": region_ms,
             "clocks": clocks,
         }
+    if splits:  # comparator runs report the kernel numbers only
+        args.no_e2e = args.no_cpu_baseline = True
     if rank == 0 and not args.no_e2e:
         line["e2e"] = measure_e2e(gq, p, dev, args, stream)
     if rank == 0 and not args.no_cpu_baseline and world == 1:

@@ -32,7 +32,8 @@ DEV_TIMEOUT = 4
 
 EXPORTED = ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states", "gqa_merge_states",
             "gqa_status", "gqa_decode_host_buffer_bytes", "gqa_decode_host", "gqa_error_string",
-            "gqa_decode_noalloc")
+            "gqa_decode_noalloc", "gqa_decode_fixed_split_workspace_size",
+            "gqa_decode_fixed_split", "gqa_select_schedule", "gqa_decode_auto")
 GQA_ERR_SCRATCH_LIMIT = 6
 
 _lib = None
@@ -62,10 +63,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_decode_host_buffer_bytes.argtypes = [I, I, I, I, I, I, I, I]
     lib.gqa_decode_host_buffer_bytes.restype = SZ
     lib.gqa_decode_host.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, SZ, P, SZ, P]
+    lib.gqa_decode_fixed_split_workspace_size.argtypes = [I, I, I, I, I, I, ctypes.POINTER(SZ)]
+    lib.gqa_decode_fixed_split.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, SZ, P]
+    lib.gqa_select_schedule.argtypes = [I, I, I, I, P, I, I, ctypes.POINTER(I), P]
+    lib.gqa_decode_auto.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, SZ, P]
     lib.gqa_error_string.argtypes = [I]
     lib.gqa_error_string.restype = ctypes.c_char_p
     for name in ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states",
-                 "gqa_merge_states", "gqa_status", "gqa_decode_host"):
+                 "gqa_merge_states", "gqa_status", "gqa_decode_host",
+                 "gqa_decode_fixed_split_workspace_size", "gqa_decode_fixed_split",
+                 "gqa_select_schedule", "gqa_decode_auto"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -176,6 +183,91 @@ def gqa_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                             _ptr(buf), buf.numel(), _stream_ptr(stream))
     _check("gqa_decode", rc)
     return out
+
+
+def fixed_split_workspace_size(B: int, Hq: int, Hkv: int, D: int, num_splits: int,
+                               device: int | None = None) -> int:
+    lib = load_library()
+    dev = torch.cuda.current_device() if device is None else device
+    n = ctypes.c_size_t()
+    _check("gqa_decode_fixed_split_workspace_size",
+           lib.gqa_decode_fixed_split_workspace_size(B, Hq, Hkv, D, num_splits, dev,
+                                                     ctypes.byref(n)))
+    return n.value
+
+
+def gqa_decode_fixed_split(q, k_cache, v_cache, block_table, seq_lens, num_splits: int,
+                           out=None, scale=None, workspace: Optional[Workspace] = None,
+                           stream=None) -> torch.Tensor:
+    """The fixed-split comparator (see include/gqa_decode.h): same result as gqa_decode."""
+    lib = load_library()
+    B, Hq, Hkv, D, bs, mb, nb = _shape(q, k_cache, block_table)
+    dev = q.device
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _require(t, n, torch.bfloat16, dev)
+    _require(seq_lens, "seq_lens", torch.int32, dev)
+    if block_table is not None:
+        _require(block_table, "block_table", torch.int32, dev)
+    if out is None:
+        out = torch.empty_like(q)
+    _require(out, "out", torch.bfloat16, dev)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    ws = default_workspace(dev) if workspace is None else workspace
+    buf = ws.get(fixed_split_workspace_size(B, Hq, Hkv, D, num_splits, dev.index))
+    with torch.cuda.device(dev):
+        rc = lib.gqa_decode_fixed_split(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                        _ptr(seq_lens), _ptr(out), B, Hq, Hkv, D, bs, scale, mb,
+                                        nb, int(num_splits), _ptr(buf), buf.numel(),
+                                        _stream_ptr(stream))
+    _check("gqa_decode_fixed_split", rc)
+    return out
+
+
+def gqa_decode_auto(q, k_cache, v_cache, block_table, seq_lens, seq_lens_host=None, out=None,
+                    scale=None, workspace: Optional[Workspace] = None, stream=None) -> torch.Tensor:
+    """gqa_decode with the runtime schedule selection; seq_lens_host: int32 CPU tensor
+    (a copy of seq_lens; taken from the device, with a sync, when omitted)."""
+    lib = load_library()
+    B, Hq, Hkv, D, bs, mb, nb = _shape(q, k_cache, block_table)
+    dev = q.device
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _require(t, n, torch.bfloat16, dev)
+    _require(seq_lens, "seq_lens", torch.int32, dev)
+    if block_table is not None:
+        _require(block_table, "block_table", torch.int32, dev)
+    host = seq_lens.cpu() if seq_lens_host is None else seq_lens_host
+    if host.device.type != "cpu" or host.dtype != torch.int32 or not host.is_contiguous() \
+            or host.numel() != B:
+        raise ValueError("seq_lens_host must be a contiguous int32 CPU tensor of length B")
+    if out is None:
+        out = torch.empty_like(q)
+    _require(out, "out", torch.bfloat16, dev)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    ws = default_workspace(dev) if workspace is None else workspace
+    buf = ws.get(workspace_size(B, Hq, Hkv, D, dev.index))
+    with torch.cuda.device(dev):
+        rc = lib.gqa_decode_auto(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                 _ptr(seq_lens), ctypes.c_void_p(host.data_ptr()), _ptr(out), B, Hq,
+                                 Hkv, D, bs, scale, mb, nb, _ptr(buf), buf.numel(),
+                                 _stream_ptr(stream))
+    _check("gqa_decode_auto", rc)
+    return out
+
+
+def select_schedule(seq_lens, Hq: int, Hkv: int, D: int, num_sms: int, max_splits: int = 64):
+    """Host-side schedule choice: (num_splits, est_us) with num_splits = 0 for the
+    stream-K gqa_decode, n > 0 for gqa_decode_fixed_split with n chunks; est_us =
+    (stream-K estimate, best fixed-split estimate or -1).  max_splits = 1 gives the
+    choice gqa_decode_auto makes."""
+    lib = load_library()
+    lens = (seq_lens.detach().to("cpu", torch.int32).contiguous() if torch.is_tensor(seq_lens)
+            else torch.tensor(list(seq_lens), dtype=torch.int32))
+    ns = ctypes.c_int()
+    est = (ctypes.c_float * 2)()
+    _check("gqa_select_schedule",
+           lib.gqa_select_schedule(lens.numel(), Hq, Hkv, D, ctypes.c_void_p(lens.data_ptr()),
+                                   int(num_sms), int(max_splits), ctypes.byref(ns), est))
+    return ns.value, (est[0], est[1])
 
 
 def gqa_decode_states(q, k_cache, v_cache, block_table, kv_begin, kv_end, scale=None,

@@ -6,6 +6,9 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <queue>
+#include <vector>
+#include <algorithm>
 
 #include "decode_simt.cuh"
 #include "decode_tc.cuh"
@@ -21,6 +24,19 @@ constexpr float LOG2E = 1.4426950408889634f;
 
 // Smallest group (query heads per KV head) that runs on the tensor-core kernel.
 constexpr int TC_MIN_G = 4;
+
+// Schedule selector cost model (gqa_select_schedule, gqa_decode_auto), fitted to
+// this library's tensor-core kernel on B200: a CTA streams K+V at
+// min(SCHED_SM_GBS, SCHED_HBM_GBS / active CTAs) -- one SM alone is limited by
+// its own copies in flight, many share the HBM -- after a start-up of
+// SCHED_CTA_US (prologue and the first tile's trip from HBM); a split segment
+// adds the merge tail SCHED_MERGE_US to stream-K and a second launch plus merge
+// SCHED_SPLIT_MERGE_US to fixed split.
+constexpr double SCHED_SM_GBS = 79.0;
+constexpr double SCHED_HBM_GBS = 6300.0;
+constexpr double SCHED_CTA_US = 3.0;
+constexpr double SCHED_MERGE_US = 3.0;
+constexpr double SCHED_SPLIT_MERGE_US = 5.0;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -160,6 +176,16 @@ TcKernelFn tc_kernel_for(int G)
     return gqa_decode_tc_kernel<16>;
 }
 
+using MergeFn = void (*)(Params);
+MergeFn tc_merge_for(int G)
+{
+    if (G <= 4)
+        return merge_split_kernel<4>;
+    if (G <= 8)
+        return merge_split_kernel<8>;
+    return merge_split_kernel<16>;
+}
+
 int tc_ctas(int G, int dev, int &ctas)
 {
     return persistent_ctas_fn(reinterpret_cast<const void *>(tc_kernel_for(G)), TcCfg::THREADS,
@@ -265,11 +291,14 @@ int check_shape(int B, int Hq, int Hkv, int D, int block_size, const int32_t *bl
     return GQA_OK;
 }
 
+// nsplit = 0: the stream-K schedule; nsplit > 0: the fixed-split comparator
+// (tensor-core shapes only), a grid of one CTA per (segment, chunk) followed by
+// merge_split_kernel.
 int run_decode(bool states, const void *q, const void *k_cache, const void *v_cache,
                const int32_t *block_table, const int32_t *seq_lens, const int32_t *kv_begin,
                const int32_t *kv_end, void *out, float *acc, float *m, float *l, int B, int Hq,
                int Hkv, int D, int block_size, float scale, int max_blocks, int num_blocks,
-               void *workspace, size_t workspace_bytes, void *stream)
+               void *workspace, size_t workspace_bytes, void *stream, int nsplit = 0)
 {
     int rc = check_shape(B, Hq, Hkv, D, block_size, block_table, max_blocks, num_blocks, scale);
     if (rc)
@@ -295,7 +324,16 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     int ctas = 0;
     if ((rc = use_tc ? tc_ctas(G, dev, ctas) : persistent_ctas(v, dev, ctas)))
         return rc;
-    const WorkspaceLayout w = layout_for(ctas, use_tc ? TcCfg::SLOT_FLOATS : v.slot_floats);
+    if (nsplit > 0 && !use_tc)
+        return GQA_ERR_UNSUPPORTED;
+    const int hch_tc = (G + TcCfg::NP - 1) / TcCfg::NP;
+    const int64_t items = nsplit > 0 ? (int64_t)B * Hkv * hch_tc * nsplit : 0;
+    if (items > (int64_t)1 << 30)
+        return GQA_ERR_INVALID_ARG;
+    // One chunk per segment (nsplit = 1) always finishes its segment: no slots.
+    const WorkspaceLayout w = nsplit > 1    ? layout_for((int)((items + 1) / 2), TcCfg::SLOT_FLOATS)
+                              : nsplit == 1 ? layout_for(0, TcCfg::SLOT_FLOATS)
+                                            : layout_for(ctas, use_tc ? TcCfg::SLOT_FLOATS : v.slot_floats);
     if (workspace_bytes < w.total)
         return GQA_ERR_WORKSPACE_TOO_SMALL;
 
@@ -323,7 +361,8 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     p.block_size = block_size;
     p.max_blocks = block_table ? max_blocks : 1;
     p.num_blocks = block_table ? num_blocks : B;
-    p.hch = use_tc ? (G + TcCfg::NP - 1) / TcCfg::NP : (G + head_chunk(G) - 1) / head_chunk(G);
+    p.hch = use_tc ? hch_tc : (G + head_chunk(G) - 1) / head_chunk(G);
+    p.nsplit = nsplit > 0 ? nsplit : 0;
     p.capacity = block_table ? (int64_t)max_blocks * block_size : (int64_t)block_size;
     p.qscale = scale * LOG2E;
     p.timeline = nullptr;
@@ -343,6 +382,18 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         CUtensorMap tmk, tmv;
         if (!encode_kv_map(&tmk, k_cache, rows, box_rows) || !encode_kv_map(&tmv, v_cache, rows, box_rows))
             return GQA_ERR_CUDA;
+        if (nsplit > 0) {
+            // Fixed split: as many CTAs as chunks, in waves; no CTA waits for another.
+            const cudaStream_t st = static_cast<cudaStream_t>(stream);
+            tc_kernel_for(G)<<<(unsigned)items, TcCfg::THREADS, TcCfg::smem_bytes(B), st>>>(p, tmk, tmv,
+                                                                                        box_rows);
+            if (B > 0 && nsplit > 1) {
+                const int nv = G <= 4 ? 4 : (G <= 8 ? 8 : 16);
+                const int64_t threads = (int64_t)B * Hkv * hch_tc * nv * TcCfg::D;
+                tc_merge_for(G)<<<(unsigned)((threads + 127) / 128), 128, 0, st>>>(p);
+            }
+            return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+        }
         // Cooperative launch: the owners of a split segment wait for one another's
         // pieces, so every CTA of the grid must be resident (the launch fails
         // rather than run otherwise).
@@ -368,6 +419,100 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
 }  // namespace gqa
 
 using namespace gqa;
+
+// The schedule selector (gqa_select_schedule, gqa_decode_auto): fixed split
+// with 1, 2, 4, ..., max_splits chunks against stream-K.
+int select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int num_sms,
+                    int max_splits, int *num_splits, float *est_us)
+{
+    if (!num_splits || num_sms <= 0 || (B > 0 && !seq_lens))
+        return GQA_ERR_INVALID_ARG;
+    int rc = check_shape(B, Hq, Hkv, D, 1, nullptr, 0, 0, 1.0f);
+    if (rc)
+        return rc;
+    for (int b = 0; b < B; ++b)
+        if (seq_lens[b] < 0)
+            return GQA_ERR_INVALID_ARG;
+    const int G = Hq / Hkv;
+    const bool tc = D == TcCfg::D && G >= TC_MIN_G && B <= TcCfg::MAX_BATCH;
+    const int64_t units = (int64_t)Hkv * (tc ? (G + TcCfg::NP - 1) / TcCfg::NP
+                                             : (G + head_chunk(G) - 1) / head_chunk(G));
+    // Microseconds per 128-token K+V tile for a CTA while `active` CTAs stream.
+    const double tile_bytes = 4.0 * TcCfg::T * D;
+    auto tile_us = [&](int64_t active) {
+        const double gbs = std::min(SCHED_SM_GBS, SCHED_HBM_GBS / (double)std::max<int64_t>(active, 1));
+        return tile_bytes / (gbs * 1e3);
+    };
+    std::vector<int64_t> nb(B);
+    int64_t W = 0;
+    for (int b = 0; b < B; ++b) {
+        nb[b] = ((int64_t)seq_lens[b] + TcCfg::T - 1) / TcCfg::T;
+        W += units * nb[b];
+    }
+    const int64_t P = num_sms;
+    if (W == 0) {  // nothing to stream: any schedule is a no-op
+        *num_splits = 0;
+        if (est_us) {
+            est_us[0] = 0.0f;
+            est_us[1] = tc ? 0.0f : -1.0f;
+        }
+        return GQA_OK;
+    }
+    // Does any segment straddle two stream-K runs?  (tile_owner of its first and
+    // last tile differ.)
+    bool sk_split = false;
+    int64_t seg0 = 0;
+    for (int b = 0; b < B && !sk_split; ++b)
+        for (int64_t u = 0; u < units && !sk_split; ++u, seg0 += nb[b])
+            if (nb[b] > 0 && ((seg0 + 1) * P - 1) / W != ((seg0 + nb[b]) * P - 1) / W)
+                sk_split = true;
+    const int64_t sk_active = std::min(P, W);
+    const double sk = (W + sk_active - 1) / sk_active * tile_us(sk_active) + SCHED_CTA_US +
+                      (sk_split ? SCHED_MERGE_US : 0.0);
+    // Fixed split: chunks are handed to SMs in index order as SMs free up.
+    double best = -1.0;
+    int best_s = 1;
+    if (tc) {
+        for (int sp = 1; sp <= max_splits; sp *= 2) {
+            if ((int64_t)B * units * sp > ((int64_t)1 << 21))
+                break;  // keep the host-side estimate cheap
+            int64_t items = 0;
+            for (int b = 0; b < B; ++b)
+                items += units * std::min<int64_t>(nb[b], sp);
+            const double tu = tile_us(std::min(P, items));
+            std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
+            for (int64_t i = 0; i < P; ++i)
+                free_at.push(0.0);
+            double makespan = 0.0;
+            bool any_split = false;
+            for (int b = 0; b < B; ++b)
+                for (int64_t u = 0; u < units; ++u) {
+                    int nonempty = 0;
+                    for (int i = 0; i < sp; ++i) {
+                        const int64_t len = (int64_t)(i + 1) * nb[b] / sp - (int64_t)i * nb[b] / sp;
+                        const double t0 = free_at.top();
+                        free_at.pop();
+                        const double t1 = t0 + (len > 0 ? SCHED_CTA_US + len * tu : 0.0);
+                        free_at.push(t1);
+                        makespan = std::max(makespan, t1);
+                        nonempty += len > 0;
+                    }
+                    any_split |= nonempty > 1;
+                }
+            const double t = makespan + (any_split ? SCHED_SPLIT_MERGE_US : 0.0);
+            if (best < 0.0 || t < best) {
+                best = t;
+                best_s = sp;
+            }
+        }
+    }
+    *num_splits = (tc && best < sk) ? best_s : 0;
+    if (est_us) {
+        est_us[0] = (float)sk;
+        est_us[1] = tc ? (float)best : -1.0f;
+    }
+    return GQA_OK;
+}
 
 extern "C" {
 
@@ -408,6 +553,64 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
     return run_decode(false, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, out,
                       nullptr, nullptr, nullptr, B, Hq, Hkv, D, block_size, scale,
                       max_blocks_per_seq, num_blocks, workspace, workspace_bytes, stream);
+}
+
+int gqa_decode_fixed_split_workspace_size(int B, int Hq, int Hkv, int D, int num_splits, int device,
+                                          size_t *bytes)
+{
+    if (!bytes || num_splits <= 0)
+        return GQA_ERR_INVALID_ARG;
+    int rc = check_shape(B, Hq, Hkv, D, 1, nullptr, 0, 0, 1.0f);
+    if (rc)
+        return rc;
+    (void)device;
+    const int G = Hq / Hkv;
+    const int64_t items = (int64_t)B * Hkv * ((G + TcCfg::NP - 1) / TcCfg::NP) * num_splits;
+    if (items > (int64_t)1 << 30)
+        return GQA_ERR_INVALID_ARG;
+    *bytes = layout_for(num_splits > 1 ? (int)((items + 1) / 2) : 0, TcCfg::SLOT_FLOATS).total;
+    return GQA_OK;
+}
+
+int gqa_decode_fixed_split(const void *q, const void *k_cache, const void *v_cache,
+                           const int32_t *block_table, const int32_t *seq_lens, void *out, int B,
+                           int Hq, int Hkv, int D, int block_size, float scale,
+                           int max_blocks_per_seq, int num_blocks, int num_splits,
+                           void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (num_splits <= 0)
+        return GQA_ERR_INVALID_ARG;
+    return run_decode(false, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, out,
+                      nullptr, nullptr, nullptr, B, Hq, Hkv, D, block_size, scale,
+                      max_blocks_per_seq, num_blocks, workspace, workspace_bytes, stream,
+                      num_splits);
+}
+
+int gqa_select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int num_sms,
+                        int max_splits, int *num_splits, float *est_us)
+{
+    if (max_splits < 1 || max_splits > 64)
+        return GQA_ERR_INVALID_ARG;
+    return select_schedule(B, Hq, Hkv, D, seq_lens, num_sms, max_splits, num_splits, est_us);
+}
+
+int gqa_decode_auto(const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_table, const int32_t *seq_lens,
+                    const int32_t *seq_lens_host, void *out, int B, int Hq, int Hkv, int D,
+                    int block_size, float scale, int max_blocks_per_seq, int num_blocks,
+                    void *workspace, size_t workspace_bytes, void *stream)
+{
+    int dev = 0, sms = 0, rc;
+    if ((rc = current_device(dev)))
+        return rc;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    int ns = 0;
+    if ((rc = select_schedule(B, Hq, Hkv, D, seq_lens_host, sms, 1, &ns, nullptr)))
+        return rc;
+    return run_decode(false, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, out,
+                      nullptr, nullptr, nullptr, B, Hq, Hkv, D, block_size, scale,
+                      max_blocks_per_seq, num_blocks, workspace, workspace_bytes, stream, ns);
 }
 
 int gqa_decode_states(const void *q, const void *k_cache, const void *v_cache,
@@ -514,11 +717,11 @@ int gqa_decode_host(const void *q, const void *k_cache, const void *v_cache,
                                s) == cudaSuccess;
     if (!ok)
         return GQA_ERR_CUDA;
-    rc = gqa_decode(dbuf + h.q, dbuf + h.k, dbuf + h.v,
-                    paged ? reinterpret_cast<const int32_t *>(dbuf + h.bt) : nullptr,
-                    reinterpret_cast<const int32_t *>(dbuf + h.lens), dbuf + h.out, B, Hq, Hkv, D,
-                    block_size, scale, max_blocks_per_seq, num_blocks, workspace, workspace_bytes,
-                    stream);
+    rc = gqa_decode_auto(dbuf + h.q, dbuf + h.k, dbuf + h.v,
+                         paged ? reinterpret_cast<const int32_t *>(dbuf + h.bt) : nullptr,
+                         reinterpret_cast<const int32_t *>(dbuf + h.lens), seq_lens, dbuf + h.out,
+                         B, Hq, Hkv, D, block_size, scale, max_blocks_per_seq, num_blocks,
+                         workspace, workspace_bytes, stream);
     if (rc)
         return rc;
     if (cudaMemcpyAsync(out, dbuf + h.out, qbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)

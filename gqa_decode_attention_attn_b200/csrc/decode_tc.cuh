@@ -69,10 +69,10 @@ struct TcCfg {
     static size_t smem_bytes(int B) { return PREFIX_OFF + (size_t)(B + 1) * sizeof(int) + 1024; }
 };
 // Segment merge: the owner list (<= 512 ints) in the P buffers; the gathered
-// slices, at most E + no + 3 no (E / D + 2) + 2 NP floats (E <= NP x D outputs,
-// no <= 512 owners), in the rings.
+// slices, at most E + 4 no + 3 no (E / D + 2) + 2 NP floats (E <= NP x D outputs,
+// no <= 512 owners, slices rounded to 4 elements), in the rings.
 static_assert(512 * 4 <= 2 * TcCfg::PBUF_BYTES, "owner list must fit in the P buffers");
-static_assert((16 * 128 + 512 + 3 * 512 * (16 + 2) + 32) * 4 <= 2 * TcCfg::STAGES * TcCfg::TILE_BYTES,
+static_assert((16 * 128 + 4 * 512 + 3 * 512 * (16 + 2) + 32) * 4 <= 2 * TcCfg::STAGES * TcCfg::TILE_BYTES,
               "gathered slices must fit in the rings");
 static_assert(TcCfg::O_COL + 2 * TcCfg::NO <= TcCfg::TMEM_COLS, "tensor memory columns");
 
@@ -200,7 +200,21 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     const int64_t units = (int64_t)p.Hkv * p.hch;
     const int64_t W = units * prefix[B];
     const int64_t P = gridDim.x, c = blockIdx.x;
-    const int64_t start = run_start(c, W, P), end = run_start(c + 1, W, P);
+    // Stream-K: CTA c takes tiles [cW/P, (c+1)W/P) of the global order.  Fixed
+    // split (the FlashDecoding comparator): CTA c takes chunk c % nsplit of
+    // segment c / nsplit, the chunks cutting the segment's tiles evenly.
+    int64_t start, end;
+    if (p.nsplit == 0) {
+        start = run_start(c, W, P);
+        end = run_start(c + 1, W, P);
+    } else {
+        const int64_t j = c / p.nsplit, i = c - j * p.nsplit;
+        const int b = (int)(j / units);
+        const int64_t nbj = prefix[b + 1] - prefix[b];
+        const int64_t seg0 = units * prefix[b] + (j - (int64_t)b * units) * nbj;
+        start = seg0 + i * nbj / p.nsplit;
+        end = seg0 + (i + 1) * nbj / p.nsplit;
+    }
     const int G = p.G;
 
     for (int b = (int)c; b < B; b += (int)P) {
@@ -221,6 +235,18 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         const uint64_t pol = l2_evict_first_policy();
         TileIter it;
         it.init(start, prefix, B, units, p.hch);
+        // Global row of this lane's box of tile `ti` (lane < boxes), or -1 for a
+        // block id outside the pool.
+        auto box_row = [&](const TileIter &ti, int tok0) -> int {
+            const int t = tok0 + lane * box_rows;
+            if (!p.block_table)
+                return (int)(((int64_t)ti.b * p.Hkv + ti.kvh) * p.block_size + t);
+            const int pg = page_of(p, t);
+            const int64_t blk = p.block_table[(int64_t)ti.b * p.max_blocks + pg];
+            if (blk < 0 || blk >= p.num_blocks)
+                return -1;
+            return (int)((blk * p.Hkv + ti.kvh) * p.block_size + (t - pg * p.block_size));
+        };
         int cur_b = -1, len = 0, k = 0;
         for (int64_t i = start; i < end; ++i, ++k) {
             if (i > start)
@@ -241,15 +267,9 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             bool bad = false;
             int row = 0;
             if (lane < nbox) {
-                const int t = tok0 + lane * box_rows;
-                if (p.block_table) {
-                    const int pg = page_of(p, t);
-                    const int64_t blk = p.block_table[(int64_t)it.b * p.max_blocks + pg];
-                    bad = blk < 0 || blk >= p.num_blocks;
-                    row = bad ? 0 : (int)((blk * p.Hkv + it.kvh) * p.block_size + (t - pg * p.block_size));
-                } else {
-                    row = (int)(((int64_t)it.b * p.Hkv + it.kvh) * p.block_size + t);
-                }
+                row = box_row(it, tok0);
+                bad = row < 0;
+                row = bad ? 0 : row;
             }
             const unsigned badmask = __ballot_sync(0xffffffffu, bad);
             if (lane == 0) {
@@ -460,7 +480,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             const int rows = min(NV, G - cur.hc * NP);
             const int64_t row0 = (int64_t)cur.b * p.Hq + (int64_t)cur.kvh * G + (int64_t)cur.hc * NP;
             const int64_t vseg = ((int64_t)cur.b * p.Hkv + cur.kvh) * p.hch + cur.hc;
-            float *slot = p.slots + (2 * c + (piece_first == start ? 0 : 1)) * (int64_t)SLOT;
+            float *slot = p.slots + (p.nsplit ? c : 2 * c + (piece_first == start ? 0 : 1)) * (int64_t)SLOT;
             if (complete) {
 #pragma unroll
                 for (int g = 0; g < NV; ++g)
@@ -665,6 +685,8 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         // Split segments: publish every partial piece of this run, then merge this
         // CTA's share of each (all owners are resident: cooperative launch).  Every
         // tile has been consumed, so the P buffers and the rings are scratch.
+        if (p.nsplit)
+            npending = 0;  // fixed split: merge_split_kernel combines the chunks
         for (int x = 0; x < npending; ++x)
             publish_piece(p, pending[x].vseg, stid, 1, 128);
         for (int x = 0; x < npending; ++x) {
@@ -692,6 +714,70 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         rec[2] = sm;
         rec[3] = (unsigned long long)(end - start);
     }
+}
+
+// Second kernel of the fixed-split comparator: one thread per output element
+// (segment j, head g, column d) merges the segment's chunks (slot c of chunk CTA
+// c) in chunk order; a segment with fewer than two non-empty chunks was written by
+// the decode kernel itself.  (Attention co-design for long-context inference,
+// section "FlashAttention and GEMM shapes": FlashDecoding's split-KV reduction.)
+template <int NV>
+__global__ void __launch_bounds__(128)
+    merge_split_kernel(const Params p)
+{
+    constexpr int D = TcCfg::D, NP = TcCfg::NP, T = TcCfg::T;
+    constexpr int SLOT = slot_floats(NV, D);
+    constexpr int U = 8;  // chunks per batch of independent loads
+    const int64_t units = (int64_t)p.Hkv * p.hch;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t j = gid / (NV * D);
+    if (j >= (int64_t)p.B * units)
+        return;
+    const int e = (int)(gid - j * (NV * D)), g = e / D, d = e - g * D;
+    const int b = (int)(j / units);
+    const int u = (int)(j - (int64_t)b * units), kvh = u / p.hch, hc = u - kvh * p.hch;
+    const int G = p.G;
+    if (g >= min(NV, G - hc * NP))
+        return;
+    int64_t begin, len;
+    request_range<false>(p, b, begin, len);
+    const int64_t nb = (len + T - 1) / T;
+    const int ns = p.nsplit;
+    if ((nb < ns ? nb : (int64_t)ns) < 2)
+        return;  // at most one non-empty chunk: written by the decode kernel
+    const float *base = p.slots + j * ns * SLOT;
+    auto nonempty = [&](int i) { return (int64_t)(i + 1) * nb / ns > (int64_t)i * nb / ns; };
+    float mx = -INFINITY;
+    for (int i0 = 0; i0 < ns; i0 += U) {
+        float mv[U];
+#pragma unroll
+        for (int q = 0; q < U; ++q)
+            mv[q] = (i0 + q < ns && nonempty(i0 + q)) ? __ldcg(base + (i0 + q) * SLOT + NV * D + g)
+                                                       : -INFINITY;
+#pragma unroll
+        for (int q = 0; q < U; ++q)
+            mx = fmaxf(mx, mv[q]);
+    }
+    float a = 0.f, ls = 0.f;
+    for (int i0 = 0; i0 < ns; i0 += U) {
+        float mv[U], lv[U], av[U];
+#pragma unroll
+        for (int q = 0; q < U; ++q) {
+            const bool have = i0 + q < ns && nonempty(i0 + q);
+            const float *sl = base + (i0 + q) * SLOT;
+            mv[q] = have ? __ldcg(sl + NV * D + g) : -INFINITY;
+            lv[q] = have ? __ldcg(sl + NV * D + NV + g) : 0.f;
+            av[q] = have ? __ldcg(sl + g * D + d) : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < U; ++q) {
+            const float w = mv[q] == -INFINITY ? 0.f : fast_exp2(mv[q] - mx);
+            a = fmaf(w, av[q], a);
+            ls = fmaf(w, lv[q], ls);
+        }
+    }
+    const int64_t row = (int64_t)b * p.Hq + (int64_t)kvh * G + (int64_t)hc * NP + g;
+    write_result<false>(p, row, d, D, a, mx, ls, ls != ls);
 }
 
 }  // namespace gqa

@@ -85,8 +85,9 @@ __device__ __forceinline__ void merge_segment_gather(const Params &p, int64_t c,
     named_barrier_sync(bar_id, NT);
     const bool ok = *reinterpret_cast<volatile int *>(flag) != 0;
 
-    const int E = rows * D;
-    const int e0 = (int)((int64_t)k * E / no), e1 = (int)((int64_t)(k + 1) * E / no);
+    // Slices start on 4-element boundaries, so every piece's slice is whole float4s.
+    const int E4 = rows * D / 4;
+    const int e0 = 4 * (int)((int64_t)k * E4 / no), e1 = 4 * (int)((int64_t)(k + 1) * E4 / no);
     const int Ec = e1 - e0;
     if (Ec > 0) {
         const int g0 = e0 / D, NH = (e1 - 1) / D - g0 + 1;
@@ -97,15 +98,44 @@ __device__ __forceinline__ void merge_segment_gather(const Params &p, int64_t c,
         float *hm_s = w_s + no * NH;   // [NH] common maximum
         float *hl_s = hm_s + NH;       // [NH] merged normaliser
         if (ok) {
-            for (int x = t; x < no * Ec; x += NT) {
-                const int i = x / Ec;
-                acc_s[x] = __ldcg(p.slots + (int64_t)list[i] * SF + e0 + (x - i * Ec));
-            }
-            for (int x = t; x < no * NH; x += NT) {
-                const int i = x / NH, g = g0 + (x - i * NH);
-                const float *sl = p.slots + (int64_t)list[i] * SF;
-                m_s[x] = __ldcg(sl + NV * D + g);
-                l_s[x] = __ldcg(sl + NV * D + NV + g);
+            // Per round, up to UA float4 of slices and UH (m, l) pairs per thread are
+            // in flight together before any is stored: one round trip to L2 for
+            // slices of up to UA x NT float4 in all (every shape here).
+            constexpr int UA = 8, UH = 2;
+            const int Ec4 = Ec / 4, na4 = no * Ec4, nh = no * NH;
+            for (int r0 = 0; r0 * NT * UA < na4 || r0 * NT * UH < nh; ++r0) {
+                float4 av[UA];
+                float mv[UH], lv[UH];
+#pragma unroll
+                for (int q = 0; q < UH; ++q) {
+                    const int x = (r0 * UH + q) * NT + t;
+                    const int i = x < nh ? x / NH : 0, g = g0 + (x - i * NH);
+                    const float *sl = p.slots + (int64_t)list[i] * SF;
+                    mv[q] = x < nh ? __ldcg(sl + NV * D + g) : 0.f;
+                    lv[q] = x < nh ? __ldcg(sl + NV * D + NV + g) : 0.f;
+                }
+#pragma unroll
+                for (int q = 0; q < UA; ++q) {
+                    const int x = (r0 * UA + q) * NT + t;
+                    const int i = x < na4 ? x / Ec4 : 0;
+                    av[q] = x < na4 ? __ldcg(reinterpret_cast<const float4 *>(
+                                          p.slots + (int64_t)list[i] * SF + e0) + (x - i * Ec4))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int q = 0; q < UH; ++q) {
+                    const int x = (r0 * UH + q) * NT + t;
+                    if (x < nh) {
+                        m_s[x] = mv[q];
+                        l_s[x] = lv[q];
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < UA; ++q) {
+                    const int x = (r0 * UA + q) * NT + t;
+                    if (x < na4)
+                        reinterpret_cast<float4 *>(acc_s)[x] = av[q];
+                }
             }
         }
         named_barrier_sync(bar_id, NT);
@@ -137,15 +167,25 @@ __device__ __forceinline__ void merge_segment_gather(const Params &p, int64_t c,
             }
         }
         named_barrier_sync(bar_id, NT);
-        for (int x = t; x < Ec; x += NT) {
+        // TPE adjacent threads share an element (few elements, many pieces), each
+        // summing every TPE-th piece; a fixed shuffle tree combines them.
+        const int TPE = Ec <= NT / 4 ? 4 : (Ec <= NT / 2 ? 2 : 1);
+        const int per = NT / TPE, sub = t % TPE;
+        for (int x0 = 0; x0 < Ec; x0 += per) {
+            const int x = x0 + t / TPE;
             const int e = e0 + x, g = e / D, h = g - g0;
+            float a = 0.f;
+            if (ok && x < Ec)
+                for (int i = sub; i < no; i += TPE)
+                    a = fmaf(w_s[i * NH + h], acc_s[i * Ec + x], a);
+            for (int o = 1; o < TPE; o <<= 1)
+                a += __shfl_xor_sync(0xffffffffu, a, o);
+            if (sub != 0 || x >= Ec)
+                continue;
             if (!ok) {
                 write_result<false>(p, row0 + g, e - g * D, D, 0.f, 0.f, 0.f, true);
                 continue;
             }
-            float a = 0.f;
-            for (int i = 0; i < no; ++i)
-                a = fmaf(w_s[i * NH + h], acc_s[i * Ec + x], a);
             const float ls = hl_s[h];
             write_result<false>(p, row0 + g, e - g * D, D, a, hm_s[h], ls, ls != ls);
         }

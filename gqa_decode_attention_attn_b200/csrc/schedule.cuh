@@ -47,6 +47,7 @@ struct Params {
     float *slots;                 // 2 partial states per CTA
     int B, Hq, Hkv, G, block_size, max_blocks, num_blocks;
     int hch;                      // head chunks per KV head
+    int nsplit;                   // 0: stream-K runs; n > 0: fixed split, CTA = (segment, chunk)
     int64_t capacity;             // tokens a request can hold
     uint32_t bs_magic;            // token -> page division by block_size (see page_of)
     int bs_shift;

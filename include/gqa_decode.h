@@ -94,8 +94,14 @@ GQA_API int gqa_decode_workspace_size(int B, int Hq, int Hkv, int D, int device,
  * persistent CTA takes one contiguous run of that global order, so long
  * requests spread over many SMs (LeanAttention decode tiles digest, sections
  * "Exact softmax that merges piece by piece" and "Hardware-sized work units").
- * A (request, KV head) split across CTAs is finished by whichever CTA arrives
- * last, which merges the partial states exactly; no CTA ever waits on another.
+ * A (request, KV head) split across CTAs is merged exactly from the partial
+ * states.  On the tensor-core kernel (D = 128, at least 4 query heads per KV head,
+ * pages of 8..128 tokens dividing 128 or multiples of 128, B <= 1024) the launch
+ * is cooperative: every CTA is resident, and the owners of a split segment wait
+ * (bounded, GQA_DEV_TIMEOUT on expiry) for one another and merge one slice of its
+ * outputs each; the launch fails with GQA_ERR_CUDA rather than run when the grid
+ * cannot be resident.  On the CUDA-core kernel the CTA that arrives last merges,
+ * and no CTA waits.
  *
  *   block_table        NULL for a contiguous cache
  *   max_blocks_per_seq row stride of block_table (ignored when it is NULL)
@@ -107,6 +113,55 @@ GQA_API int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
                int B, int Hq, int Hkv, int D, int block_size, float scale,
                int max_blocks_per_seq, int num_blocks,
                void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Fixed-split comparator (FlashDecoding-style, the prior art the LeanAttention
+ * decode tiles digest measures against in "Evaluation figures and their scope"):
+ * the tiles of every (request, KV head) are cut into num_splits even chunks, one
+ * CTA per chunk (a grid of B * Hkv * ceil(G / 16) * num_splits CTAs run in
+ * waves), and a second kernel merges each segment's chunks exactly.  Same
+ * arguments and result as gqa_decode; tensor-core shapes only (else
+ * GQA_ERR_UNSUPPORTED); workspace from gqa_decode_fixed_split_workspace_size,
+ * zero-filled once.  It exists to measure the stream-K schedule against.
+ */
+GQA_API int gqa_decode_fixed_split_workspace_size(int B, int Hq, int Hkv, int D, int num_splits,
+                                                  int device, size_t *bytes);
+GQA_API int gqa_decode_fixed_split(const void *q, const void *k_cache, const void *v_cache,
+                                   const int32_t *block_table, const int32_t *seq_lens, void *out,
+                                   int B, int Hq, int Hkv, int D, int block_size, float scale,
+                                   int max_blocks_per_seq, int num_blocks, int num_splits,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Runtime schedule selection on the host (LeanAttention decode tiles digest,
+ * section "Runtime selection policy": the choice depends on the batch's context
+ * length distribution, the heads per device, the head dimension and the SM
+ * count).  seq_lens is a HOST array [B].  A cost model of this library on B200
+ * (per-CTA streaming rate, shared HBM bandwidth, start-up and merge costs)
+ * estimates the stream-K schedule and the fixed split with 1, 2, 4, ...,
+ * max_splits (<= 64) chunks, chunks assigned to SMs in order as they free up.
+ * *num_splits = 0 selects gqa_decode (stream-K), n > 0 selects
+ * gqa_decode_fixed_split with n chunks.  est_us (NULL or float[2]) receives the
+ * two estimates: stream-K, best fixed split (-1 when fixed split does not apply).
+ * Contention from other kernels, which the digest also lists, is not modelled.
+ */
+GQA_API int gqa_select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int num_sms,
+                                int max_splits, int *num_splits, float *est_us);
+
+/*
+ * gqa_decode with the runtime selection of the LeanAttention decode tiles digest
+ * ("Runtime selection policy": short contexts or large batches fill the GPU with
+ * one CTA per (request, KV head) and need no reduction; long contexts, few heads
+ * per device and uneven batches want stream-K).  seq_lens_host is a HOST copy of
+ * seq_lens [B]; gqa_select_schedule's cost model, restricted to the two choices
+ * stream-K and one chunk per segment, picks the schedule.  Same arguments,
+ * workspace (gqa_decode_workspace_size) and result as gqa_decode.
+ */
+GQA_API int gqa_decode_auto(const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *block_table, const int32_t *seq_lens,
+                            const int32_t *seq_lens_host, void *out, int B, int Hq, int Hkv, int D,
+                            int block_size, float scale, int max_blocks_per_seq, int num_blocks,
+                            void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Partial softmax states of every query row over the key range
@@ -147,9 +202,10 @@ GQA_API int gqa_status(void *workspace, void *stream, unsigned *device_error);
 /*
  * gqa_decode with HOST buffers: copies q, k_cache, v_cache, block_table and
  * seq_lens from host memory into `device_buffer` (at least
- * gqa_decode_host_buffer_bytes() bytes, device), runs gqa_decode, copies out
- * back to host memory and synchronises the stream.  Pinned host memory gives
- * asynchronous, full-bandwidth copies.  Same shapes and errors as gqa_decode.
+ * gqa_decode_host_buffer_bytes() bytes, device), runs gqa_decode_auto (the
+ * lengths are on the host already), copies out back to host memory and
+ * synchronises the stream.  Pinned host memory gives asynchronous,
+ * full-bandwidth copies.  Same shapes and errors as gqa_decode.
  */
 GQA_API size_t gqa_decode_host_buffer_bytes(int B, int Hq, int Hkv, int D, int block_size,
                                     int max_blocks_per_seq, int num_blocks, int paged);
