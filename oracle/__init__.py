@@ -104,6 +104,9 @@ class Oracle:
         P, I, I64, Dbl = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
         lib.oracle_gqa_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, Dbl, I64, I64, P]
         lib.oracle_gqa_decode.restype = I
+        lib.oracle_gqa_decode_multi.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, Dbl, I64,
+                                                I64, P]
+        lib.oracle_gqa_decode_multi.restype = I
         lib.oracle_gqa_decode_states.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, Dbl,
                                                  I64, I64, P, P, P]
         lib.oracle_gqa_decode_states.restype = I
@@ -142,6 +145,32 @@ class Oracle:
 
         _run_spans(run, _split(r1 - r0, threads))
         return out.reshape(B, Hq, D) if rows is None else out
+
+    def gqa_decode_multi(self, q, k_cache, v_cache, block_table, seq_lens, scale: float,
+                         rows=None, threads: int | None = None) -> np.ndarray:
+        """Several query tokens per request (speculative verification): q [B, Q, Hq, D];
+        query token i of request b attends keys t <= L_b - Q + i.  Returns [B, Q, Hq, D]
+        float64 (or [row_end-row_begin, D] over the flattened [B*Q*Hq] rows)."""
+        lib = self.lib
+        qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+        bt, sl = _i32(block_table), _i32(seq_lens)
+        B, Q, Hq, D = qb.shape
+        _, _, Hkv, D2, bs, max_blocks, num_blocks = _shape(qb.reshape(B, Q * Hq, D), kb, bt)
+        r0, r1 = (0, B * Q * Hq) if rows is None else rows
+        out = np.zeros((r1 - r0, D), dtype=np.float64)
+        threads = host_threads() if threads is None else threads
+
+        def run(span):
+            a, b = span
+            rc = lib.oracle_gqa_decode_multi(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(bt), _ptr(sl), B,
+                                             Q, Hq, Hkv, D, bs, max_blocks, num_blocks,
+                                             float(scale), r0 + a, r0 + b,
+                                             ctypes.c_void_p(out.ctypes.data + a * D * 8))
+            if rc:
+                raise RuntimeError(f"oracle_gqa_decode_multi: {ORACLE_ERRORS.get(rc, rc)}")
+
+        _run_spans(run, _split(r1 - r0, threads))
+        return out.reshape(B, Q, Hq, D) if rows is None else out
 
     def gqa_decode_states(self, q, k_cache, v_cache, block_table, kv_begin, kv_end,
                           scale: float, threads: int | None = None):
@@ -208,6 +237,10 @@ def default() -> Oracle:
 
 def gqa_decode(*args, **kw):
     return default().gqa_decode(*args, **kw)
+
+
+def gqa_decode_multi(*args, **kw):
+    return default().gqa_decode_multi(*args, **kw)
 
 
 def gqa_decode_states(*args, **kw):

@@ -196,6 +196,54 @@ int oracle_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t
 }
 
 /*
+ * Several query tokens per request (the verification pass of speculative
+ * decoding: the large model scores the gamma drafted positions together in one
+ * pass; Inference optimization: KV cache, MQA/GQA, batching..., section 5
+ * "Speculative decoding").  The drafted tokens' keys and values are already in
+ * the cache, so request b holds L_b >= Q tokens and query token i (0 <= i < Q)
+ * sits at position L_b - Q + i.  Reading of the pages: each position sees the
+ * keys up to and including its own, t <= L_b - Q + i (causal inside the Q new
+ * tokens), as in a prefill pass over them.
+ *
+ * q and out are [B, Q, Hq, D]; rows r in [row_begin, row_end) of the flattened
+ * [B, Q, Hq] grid (r = (b * Q + i) * Hq + h).  With Q = 1 this is
+ * oracle_gqa_decode.  L_b < Q is an error (ORACLE_BAD_ARG).
+ */
+int oracle_gqa_decode_multi(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                            const int32_t *block_table, const int32_t *seq_lens,
+                            int B, int Q, int Hq, int Hkv, int D, int block_size,
+                            int max_blocks, int num_blocks, double scale,
+                            int64_t row_begin, int64_t row_end, double *out)
+{
+    int rc = check_shape(B, Hq, Hkv, D, block_size, block_table, max_blocks, num_blocks);
+    if (rc)
+        return rc;
+    if (Q <= 0 || row_begin < 0 || row_end > (int64_t)B * Q * Hq || row_begin > row_end)
+        return ORACLE_BAD_ARG;
+    kv_cache c = {k_cache, v_cache, block_table, Hkv, D, block_size, max_blocks, num_blocks};
+    const int G = Hq / Hkv;
+    int64_t capacity = block_table ? (int64_t)max_blocks * block_size : block_size;
+
+    for (int64_t r = row_begin; r < row_end; ++r) {
+        int h = (int)(r % Hq);
+        int64_t bi = r / Hq;
+        int b = (int)(bi / Q), i = (int)(bi % Q);
+        int kvh = h / G;
+        int64_t L = seq_lens[b];
+        if (L < Q || L > capacity)
+            return ORACLE_BAD_ARG;
+        double m, l;
+        double *o = out + (r - row_begin) * D;
+        rc = attention_state(&c, q + r * D, scale, b, kvh, 0, L - Q + i + 1, o, &m, &l);
+        if (rc)
+            return rc;
+        for (int d = 0; d < D; ++d)
+            o[d] = l > 0.0 ? o[d] / l : 0.0;
+    }
+    return ORACLE_OK;
+}
+
+/*
  * Partial softmax states (acc unnormalised, m, l; natural-log units) for query
  * rows [row_begin, row_end) over the per-request key range
  * [kv_begin[b], kv_end[b]).  acc holds (row_end - row_begin) * D doubles; m and

@@ -304,4 +304,60 @@ def pin_bad_block_rejected(o):
     raise AssertionError("out-of-pool block id was accepted")
 
 
+# --------------------------------------------------------------------------- several query tokens
+
+def _multi_problem(B, Q, Hq, Hkv, D, lens, seed, bs):
+    """A problem with Q query tokens per request: q [B, Q, Hq, D]."""
+    p = make_problem("multi", B, Q * Hq, Hkv, D, lens, seed=seed, block_size=bs)
+    return p, p.q.reshape(B, Q, Hq, D).contiguous()
+
+
+MULTI_CASES = [(2, 3, 4, 2, 8, [9, 5], 4), (1, 4, 2, 1, 6, [4], None), (2, 2, 6, 3, 4, [3, 7], 2)]
+
+
+def pin_multi_brute_force(o):
+    """Speculative verification (Inference optimization ..., section 5): query token
+    i of Q sits at position L - Q + i and sees keys t <= L - Q + i.  Checked against
+    the full score matrix with an explicit causal mask, softmax and matmul in numpy
+    extended precision."""
+    for (B, Q, Hq, Hkv, D, lens, bs) in MULTI_CASES:
+        p, q = _multi_problem(B, Q, Hq, Hkv, D, lens, 31 + D, bs)
+        out = o.gqa_decode_multi(q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, p.scale)
+        G = Hq // Hkv
+        for b in range(B):
+            L = int(p.seq_lens[b])
+            for h in range(Hq):
+                K, V = _kv_rows(p, b, h // G)
+                Kl, Vl = f64(K).astype(np.longdouble), f64(V).astype(np.longdouble)
+                for i in range(Q):
+                    S = (Kl @ f64(q[b, i, h]).astype(np.longdouble)) * np.longdouble(p.scale)
+                    S[np.arange(L) > L - Q + i] = -np.inf
+                    P = np.exp(S - S.max())
+                    ref = (P / P.sum()) @ Vl
+                    assert np.allclose(out[b, i, h], ref.astype(np.float64), rtol=1e-13, atol=1e-15)
+
+
+def pin_multi_query_prefix(o):
+    """Query token i sees exactly what a single-query decode of the request cut to
+    L - Q + i + 1 tokens sees; the last token sees the whole request."""
+    for (B, Q, Hq, Hkv, D, lens, bs) in MULTI_CASES:
+        p, q = _multi_problem(B, Q, Hq, Hkv, D, lens, 57 + D, bs)
+        out = o.gqa_decode_multi(q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, p.scale)
+        for i in range(Q):
+            lens_i = (p.seq_lens - Q + i + 1).to(torch.int32)
+            ref = o.gqa_decode(q[:, i].contiguous(), p.k_cache, p.v_cache, p.block_table, lens_i,
+                               p.scale)
+            assert np.allclose(out[:, i], ref, rtol=1e-13, atol=1e-15)
+
+
+def pin_multi_too_short_rejected(o):
+    """A request shorter than its Q query tokens is an error, not a guess."""
+    p, q = _multi_problem(1, 3, 2, 1, 4, [2], 5, None)
+    try:
+        o.gqa_decode_multi(q, p.k_cache, p.v_cache, None, p.seq_lens, p.scale)
+    except RuntimeError:
+        return
+    raise AssertionError("L < Q accepted")
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

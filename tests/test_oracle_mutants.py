@@ -18,7 +18,8 @@ MUTANTS = {
     "scale_dropped": ("s[i] = scale * dot;", "s[i] = dot;"),
     "exp_sign_flipped": ("double w = exp(s[i] - m);", "double w = exp(m - s[i]);"),
     "max_pass_dropped": ("if (s[i] > m)\n            m = s[i];", "m = 0.0;"),
-    "head_map_modulo": ("int kvh = h / G;", "int kvh = h % Hkv;"),
+    "head_map_modulo": ("int b = (int)(r / Hq), h = (int)(r % Hq);\n        int kvh = h / G;",
+                        "int b = (int)(r / Hq), h = (int)(r % Hq);\n        int kvh = h % Hkv;"),
     "states_head_map_modulo": ("b, h / G, t0, t1", "b, h % Hkv, t0, t1"),
     "page_offset_shifted": ("offset = t % c->block_size;", "offset = (t + 1) % c->block_size;"),
     "block_index_shifted": ("t / c->block_size];", "(t / c->block_size) ^ 1];"),
@@ -26,8 +27,12 @@ MUTANTS = {
     "first_key_skipped": ("for (int64_t i = 0; i < n; ++i) {\n        double w",
                           "for (int64_t i = 1; i < n; ++i) {\n        double w"),
     "normaliser_unweighted": ("l += w;", "l += 1.0;"),
-    "query_head_zero": ("rc = attention_state(&c, q + r * D, scale, b, kvh,",
-                        "rc = attention_state(&c, q + (r / Hq) * Hq * D, scale, b, kvh,"),
+    "query_head_zero": ("rc = attention_state(&c, q + r * D, scale, b, kvh, 0, L, o, &m, &l);",
+                        "rc = attention_state(&c, q + (r / Hq) * Hq * D, scale, b, kvh, 0, L, o, &m, &l);"),
+    "multi_mask_off_by_one": ("0, L - Q + i + 1, o,", "0, L - Q + i, o,"),
+    "multi_token_order": ("int b = (int)(bi / Q), i = (int)(bi % Q);",
+                          "int i = (int)(bi / B), b = (int)(bi % B);"),
+    "multi_mask_reversed": ("0, L - Q + i + 1, o,", "0, L - i, o,"),
     "merge_weight_sign": ("exp(mi - mstar)", "exp(mstar - mi)"),
     "merge_normaliser_unweighted": ("lstar += w * l[", "lstar += l["),
     "merge_lse_dropped_max": ("mstar + log(lstar)", "log(lstar)"),
