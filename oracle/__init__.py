@@ -61,6 +61,20 @@ def _bits(x) -> np.ndarray:
     return arr
 
 
+def _bytes8(x) -> np.ndarray:
+    """Contiguous uint8 view of FP8 E4M3 data (torch float8_e4m3fn or uint8, numpy uint8)."""
+    if hasattr(x, "detach"):
+        import torch
+        x = x.detach().to("cpu").contiguous()
+        if x.dtype != torch.uint8:
+            x = x.view(torch.uint8)
+        x = x.numpy()
+    arr = np.ascontiguousarray(np.asarray(x))
+    if arr.dtype != np.uint8:
+        raise TypeError(f"expected FP8 E4M3 bytes (uint8), got {arr.dtype}")
+    return arr
+
+
 def _i32(x) -> np.ndarray | None:
     if x is None:
         return None
@@ -112,6 +126,11 @@ class Oracle:
         lib.oracle_gqa_decode_states.restype = I
         lib.oracle_merge_states.argtypes = [P, P, P, I, I, I, P, P]
         lib.oracle_merge_states.restype = I
+        lib.oracle_gqa_decode_fp8.argtypes = [P, P, P, Dbl, Dbl, P, P, I, I, I, I, I, I, I, Dbl,
+                                              I64, I64, P]
+        lib.oracle_gqa_decode_fp8.restype = I
+        lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_double.restype = Dbl
         lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
         lib.oracle_bf16_to_double.restype = Dbl
         self.lib = lib
@@ -145,6 +164,34 @@ class Oracle:
 
         _run_spans(run, _split(r1 - r0, threads))
         return out.reshape(B, Hq, D) if rows is None else out
+
+    def gqa_decode_fp8(self, q, k8, v8, k_scale: float, v_scale: float, block_table, seq_lens,
+                       scale: float, rows=None, threads: int | None = None) -> np.ndarray:
+        """Decode over an FP8 E4M3 cache (values e4m3 * k_scale, e4m3 * v_scale); k8, v8
+        have the bf16 caches' shapes with one byte per element.  Returns [B, Hq, D]."""
+        lib = self.lib
+        qb, kb, vb = _bits(q), _bytes8(k8), _bytes8(v8)
+        bt, sl = _i32(block_table), _i32(seq_lens)
+        B, Hq, Hkv, D, bs, max_blocks, num_blocks = _shape(qb, kb, bt)
+        r0, r1 = (0, B * Hq) if rows is None else rows
+        out = np.zeros((r1 - r0, D), dtype=np.float64)
+        threads = host_threads() if threads is None else threads
+
+        def run(span):
+            a, b = span
+            rc = lib.oracle_gqa_decode_fp8(_ptr(qb), _ptr(kb), _ptr(vb), float(k_scale),
+                                           float(v_scale), _ptr(bt), _ptr(sl), B, Hq, Hkv, D, bs,
+                                           max_blocks, num_blocks, float(scale), r0 + a, r0 + b,
+                                           ctypes.c_void_p(out.ctypes.data + a * D * 8))
+            if rc:
+                raise RuntimeError(f"oracle_gqa_decode_fp8: {ORACLE_ERRORS.get(rc, rc)}")
+
+        _run_spans(run, _split(r1 - r0, threads))
+        return out.reshape(B, Hq, D) if rows is None else out
+
+    def e4m3_to_double(self, bits: int) -> float:
+        """Exact widening of one FP8 E4M3 byte."""
+        return self.lib.oracle_e4m3_to_double(int(bits))
 
     def gqa_decode_multi(self, q, k_cache, v_cache, block_table, seq_lens, scale: float,
                          rows=None, threads: int | None = None) -> np.ndarray:
@@ -237,6 +284,14 @@ def default() -> Oracle:
 
 def gqa_decode(*args, **kw):
     return default().gqa_decode(*args, **kw)
+
+
+def gqa_decode_fp8(*args, **kw):
+    return default().gqa_decode_fp8(*args, **kw)
+
+
+def e4m3_to_double(bits: int) -> float:
+    return default().e4m3_to_double(bits)
 
 
 def gqa_decode_multi(*args, **kw):

@@ -60,11 +60,45 @@ static double bf16_to_double(uint16_t bits)
 
 double oracle_bf16_to_double(uint16_t bits) { return bf16_to_double(bits); }
 
+/* FP8 E4M3 (the "fn" encoding: 1 sign bit, 4 exponent bits with bias 7, 3
+ * mantissa bits, no infinities, S.1111.111 is NaN), widened exactly:
+ * normal (-1)^s 2^(e-7) (1 + m/8), subnormal (e = 0) (-1)^s 2^-6 (m/8). */
+static double e4m3_to_double(uint8_t bits)
+{
+    int s = bits >> 7, e = (bits >> 3) & 15, m = bits & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+double oracle_e4m3_to_double(uint8_t bits) { return e4m3_to_double(bits); }
+
+/* One cache holds bf16 rows, or FP8 E4M3 rows with one scale per tensor (the
+ * value is the E4M3 number times k_scale or v_scale): FP8 caches halve the bytes
+ * a decode step reads (Attention co-design for long-context inference, the
+ * FP8 KV cache in its list of techniques). */
 typedef struct {
     const uint16_t *k, *v;
+    const uint8_t *k8, *v8;     /* non-NULL: FP8 cache (k, v unused) */
+    double k_scale, v_scale;
     const int32_t *block_table; /* NULL: contiguous cache */
     int Hkv, D, block_size, max_blocks, num_blocks;
 } kv_cache;
+
+static double key_at(const kv_cache *c, int64_t i)
+{
+    return c->k8 ? e4m3_to_double(c->k8[i]) * c->k_scale : bf16_to_double(c->k[i]);
+}
+
+static double value_at(const kv_cache *c, int64_t i)
+{
+    return c->v8 ? e4m3_to_double(c->v8[i]) * c->v_scale : bf16_to_double(c->v[i]);
+}
 
 /* Element offset of key/value row t of (request b, kv head kvh); -1 when the
  * block table names a block outside the pool. */
@@ -117,7 +151,7 @@ static int attention_state(const kv_cache *c, const uint16_t *qrow, double scale
         rows[i] = row;
         double dot = 0.0;
         for (int d = 0; d < D; ++d)
-            dot += bf16_to_double(qrow[d]) * bf16_to_double(c->k[row + d]);
+            dot += bf16_to_double(qrow[d]) * key_at(c, row + d);
         s[i] = scale * dot;
     }
 
@@ -134,7 +168,7 @@ static int attention_state(const kv_cache *c, const uint16_t *qrow, double scale
         double w = exp(s[i] - m);
         l += w;
         for (int d = 0; d < D; ++d)
-            acc[d] += w * bf16_to_double(c->v[rows[i] + d]);
+            acc[d] += w * value_at(c, rows[i] + d);
     }
 
     *m_out = m;
@@ -174,7 +208,7 @@ int oracle_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t
         return rc;
     if (row_begin < 0 || row_end > (int64_t)B * Hq || row_begin > row_end)
         return ORACLE_BAD_ARG;
-    kv_cache c = {k_cache, v_cache, block_table, Hkv, D, block_size, max_blocks, num_blocks};
+    kv_cache c = {k_cache, v_cache, NULL, NULL, 1.0, 1.0, block_table, Hkv, D, block_size, max_blocks, num_blocks};
     const int G = Hq / Hkv;
     int64_t capacity = block_table ? (int64_t)max_blocks * block_size : block_size;
 
@@ -187,6 +221,44 @@ int oracle_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t
         double m, l;
         double *o = out + (r - row_begin) * D;
         rc = attention_state(&c, q + r * D, scale, b, kvh, 0, L, o, &m, &l);
+        if (rc)
+            return rc;
+        for (int d = 0; d < D; ++d)
+            o[d] = l > 0.0 ? o[d] / l : 0.0;
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * oracle_gqa_decode over an FP8 E4M3 cache: k8, v8 hold one byte per element
+ * (same layouts as the bf16 caches), their values are e4m3(byte) * k_scale and
+ * e4m3(byte) * v_scale.  q stays bf16.
+ */
+int oracle_gqa_decode_fp8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8,
+                          double k_scale, double v_scale, const int32_t *block_table,
+                          const int32_t *seq_lens, int B, int Hq, int Hkv, int D,
+                          int block_size, int max_blocks, int num_blocks, double scale,
+                          int64_t row_begin, int64_t row_end, double *out)
+{
+    int rc = check_shape(B, Hq, Hkv, D, block_size, block_table, max_blocks, num_blocks);
+    if (rc)
+        return rc;
+    if (row_begin < 0 || row_end > (int64_t)B * Hq || row_begin > row_end)
+        return ORACLE_BAD_ARG;
+    kv_cache c = {NULL, NULL, k8, v8, k_scale, v_scale, block_table, Hkv, D, block_size,
+                  max_blocks, num_blocks};
+    const int G = Hq / Hkv;
+    int64_t capacity = block_table ? (int64_t)max_blocks * block_size : block_size;
+
+    for (int64_t r = row_begin; r < row_end; ++r) {
+        int b = (int)(r / Hq), kvh = (int)(r % Hq) / G;
+        int64_t L = seq_lens[b];
+        if (L < 0 || L > capacity)
+            return ORACLE_BAD_ARG;
+        double m, l;
+        double *o = out + (r - row_begin) * D;
+        const uint16_t *qrow = q + r * D;
+        rc = attention_state(&c, qrow, scale, b, kvh, 0, L, o, &m, &l);
         if (rc)
             return rc;
         for (int d = 0; d < D; ++d)
@@ -220,7 +292,7 @@ int oracle_gqa_decode_multi(const uint16_t *q, const uint16_t *k_cache, const ui
         return rc;
     if (Q <= 0 || row_begin < 0 || row_end > (int64_t)B * Q * Hq || row_begin > row_end)
         return ORACLE_BAD_ARG;
-    kv_cache c = {k_cache, v_cache, block_table, Hkv, D, block_size, max_blocks, num_blocks};
+    kv_cache c = {k_cache, v_cache, NULL, NULL, 1.0, 1.0, block_table, Hkv, D, block_size, max_blocks, num_blocks};
     const int G = Hq / Hkv;
     int64_t capacity = block_table ? (int64_t)max_blocks * block_size : block_size;
 
@@ -261,7 +333,7 @@ int oracle_gqa_decode_states(const uint16_t *q, const uint16_t *k_cache, const u
         return rc;
     if (row_begin < 0 || row_end > (int64_t)B * Hq || row_begin > row_end)
         return ORACLE_BAD_ARG;
-    kv_cache c = {k_cache, v_cache, block_table, Hkv, D, block_size, max_blocks, num_blocks};
+    kv_cache c = {k_cache, v_cache, NULL, NULL, 1.0, 1.0, block_table, Hkv, D, block_size, max_blocks, num_blocks};
     const int G = Hq / Hkv;
     int64_t capacity = block_table ? (int64_t)max_blocks * block_size : block_size;
 

@@ -360,4 +360,35 @@ def pin_multi_too_short_rejected(o):
     raise AssertionError("L < Q accepted")
 
 
+# --------------------------------------------------------------------------- FP8 E4M3 cache
+
+def pin_e4m3_widening(o):
+    """All 256 FP8 E4M3 codes widen exactly as torch's float8_e4m3fn does."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([o.e4m3_to_double(c) for c in range(256)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    assert np.array_equal(got[fin], ref[fin])
+
+
+def pin_fp8_equals_dequantized_bf16(o):
+    """An FP8 cache with power-of-two scales gives exactly the result of the bf16
+    oracle on the dequantized cache (every e4m3 value times 2^k is a bf16 value)."""
+    for (B, Hq, Hkv, D, lens, bs, ks, vs) in [(2, 8, 2, 16, [37, 5], 4, 0.25, 2.0),
+                                              (1, 4, 1, 8, [20], None, 1.0, 0.5)]:
+        p = make_problem("fp8", B, Hq, Hkv, D, lens, seed=41 + D, block_size=bs)
+        gen = torch.Generator().manual_seed(99 + D)
+        k8 = torch.randint(0, 256, p.k_cache.shape, generator=gen, dtype=torch.int32).to(torch.uint8)
+        v8 = torch.randint(0, 256, p.v_cache.shape, generator=gen, dtype=torch.int32).to(torch.uint8)
+        k8[(k8 & 0x7F) == 0x7F] -= 1   # no NaN codes
+        v8[(v8 & 0x7F) == 0x7F] -= 1
+        kd = (k8.view(torch.float8_e4m3fn).to(torch.float64) * ks).to(torch.bfloat16)
+        vd = (v8.view(torch.float8_e4m3fn).to(torch.float64) * vs).to(torch.bfloat16)
+        assert torch.equal(kd.to(torch.float64), k8.view(torch.float8_e4m3fn).to(torch.float64) * ks)
+        got = o.gqa_decode_fp8(p.q, k8, v8, ks, vs, p.block_table, p.seq_lens, p.scale)
+        ref = o.gqa_decode(p.q, kd, vd, p.block_table, p.seq_lens, p.scale)
+        assert np.array_equal(got, ref)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -23,7 +23,13 @@ MUTANTS = {
     "states_head_map_modulo": ("b, h / G, t0, t1", "b, h % Hkv, t0, t1"),
     "page_offset_shifted": ("offset = t % c->block_size;", "offset = (t + 1) % c->block_size;"),
     "block_index_shifted": ("t / c->block_size];", "(t / c->block_size) ^ 1];"),
-    "key_replaced_by_value": ("bf16_to_double(c->k[row + d]);", "bf16_to_double(c->v[row + d]);"),
+    "key_replaced_by_value": ("dot += bf16_to_double(qrow[d]) * key_at(c, row + d);",
+                              "dot += bf16_to_double(qrow[d]) * value_at(c, row + d);"),
+    "e4m3_bias_off_by_one": ("ldexp(1.0 + (double)m / 8.0, e - 7)", "ldexp(1.0 + (double)m / 8.0, e - 8)"),
+    "e4m3_subnormal_exponent": ("ldexp((double)m / 8.0, -6)", "ldexp((double)m / 8.0, -7)"),
+    "e4m3_mantissa_width": ("1.0 + (double)m / 8.0, e - 7", "1.0 + (double)m / 16.0, e - 7"),
+    "fp8_value_scale_dropped": ("e4m3_to_double(c->v8[i]) * c->v_scale", "e4m3_to_double(c->v8[i])"),
+    "fp8_key_scale_dropped": ("e4m3_to_double(c->k8[i]) * c->k_scale", "e4m3_to_double(c->k8[i])"),
     "first_key_skipped": ("for (int64_t i = 0; i < n; ++i) {\n        double w",
                           "for (int64_t i = 1; i < n; ++i) {\n        double w"),
     "normaliser_unweighted": ("l += w;", "l += 1.0;"),
