@@ -48,7 +48,9 @@ KERNEL_SOURCES = ["gqa_decode_attention_attn_b200/csrc/decode_simt.cuh",
 def kernel_for(p) -> str:
     """Which decode kernel the library runs for this problem (mirrors the library's
     dispatch: tensor cores for D = 128 with at least 4 query heads per KV head and
-    pages that tile into 128-token boxes, CUDA cores otherwise)."""
+    pages that tile into 128-token boxes, CUDA cores otherwise and for FP8 caches)."""
+    if p.meta.get("kv_elem_bytes") == 1:
+        return "gqa_decode_simt_kernel (FP8 E4M3 cache)"
     bs = p.block_size
     boxes = (not p.paged) or (bs % 128 == 0 if bs >= 128 else (bs >= 8 and 128 % bs == 0))
     if p.D == 128 and p.G >= 4 and p.B <= 1024 and boxes:
@@ -195,7 +197,8 @@ def _oracle_chunk(p, threads: int) -> int:
 
 def _sample_bytes(p, b0: int, b1: int) -> int:
     L = sum(int(x) for x in p.seq_lens[b0:b1])
-    return 4 * p.Hkv * p.D * L + 4 * (b1 - b0) * p.Hq * p.D
+    eb = int(p.meta.get("kv_elem_bytes", 2))
+    return 2 * eb * p.Hkv * p.D * L + 4 * (b1 - b0) * p.Hq * p.D
 
 
 def cpu_oracle_sample(p, target_s: float):
@@ -234,12 +237,17 @@ def run_reference(args, rank: int):
     oracle.default()
     chunk = _oracle_chunk(p, threads)
     per_step, total_bytes = [], 0
+    fp8 = workloads.fp8_caches(p) if p.meta.get("kv_elem_bytes") == 1 else None
 
     def step(i):
         b0 = (i * chunk) % p.B
         b1 = min(p.B, b0 + chunk)
-        oracle.gqa_decode(p.q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, p.scale,
-                          rows=(b0 * p.Hq, b1 * p.Hq), threads=threads)
+        if fp8:
+            oracle.gqa_decode_fp8(p.q, fp8[0], fp8[1], fp8[2], fp8[3], p.block_table, p.seq_lens,
+                                  p.scale, rows=(b0 * p.Hq, b1 * p.Hq), threads=threads)
+        else:
+            oracle.gqa_decode(p.q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, p.scale,
+                              rows=(b0 * p.Hq, b1 * p.Hq), threads=threads)
         return _sample_bytes(p, b0, b1)
 
     for i in range(args.warmup):
@@ -289,7 +297,13 @@ def main():
         pg = dist
 
     p = workloads.workload(args.workload)
+    fp8 = p.meta.get("kv_elem_bytes") == 1
     d = p.to(dev)
+    if fp8:  # the cache as FP8 E4M3 bytes with per-tensor scales
+        k8, v8, k_scale, v_scale = workloads.fp8_caches(p)
+        d.k_cache, d.v_cache = k8.to(dev), v8.to(dev)
+        args.no_e2e = True  # the host-buffer entry point takes bf16 caches
+        args.no_cpu_baseline = True  # (bench.py --impl reference times the FP8 oracle)
     out = torch.empty_like(d.q)
     ws = gq.Workspace(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -298,7 +312,9 @@ def main():
     splits = 0
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     lens_host = p.seq_lens.to(torch.int32).contiguous()
-    if args.schedule == "fixed":
+    if fp8:
+        schedule = "stream-K (FP8 cache)"
+    elif args.schedule == "fixed":
         segs = p.B * p.Hkv * -(-p.G // 16)
         splits = args.splits if args.splits > 0 else max(1, -(-sms // segs))
         schedule = f"fixed-split x{splits}"
@@ -309,7 +325,10 @@ def main():
         schedule = "stream-K"
 
     def step():
-        if splits:
+        if fp8:
+            gq.gqa_decode_fp8(d.q, d.k_cache, d.v_cache, k_scale, v_scale, d.block_table,
+                              d.seq_lens, out=out, scale=p.scale, workspace=ws, stream=stream)
+        elif splits:
             gq.gqa_decode_fixed_split(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,
                                       splits, out=out, scale=p.scale, workspace=ws, stream=stream)
         elif args.schedule == "auto":

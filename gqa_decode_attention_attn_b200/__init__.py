@@ -33,7 +33,8 @@ DEV_TIMEOUT = 4
 EXPORTED = ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states", "gqa_merge_states",
             "gqa_status", "gqa_decode_host_buffer_bytes", "gqa_decode_host", "gqa_error_string",
             "gqa_decode_noalloc", "gqa_decode_fixed_split_workspace_size",
-            "gqa_decode_fixed_split", "gqa_select_schedule", "gqa_decode_auto")
+            "gqa_decode_fixed_split", "gqa_select_schedule", "gqa_decode_auto",
+            "gqa_decode_multi", "gqa_decode_fp8")
 GQA_ERR_SCRATCH_LIMIT = 6
 
 _lib = None
@@ -67,12 +68,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_decode_fixed_split.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, SZ, P]
     lib.gqa_select_schedule.argtypes = [I, I, I, I, P, I, I, ctypes.POINTER(I), P]
     lib.gqa_decode_auto.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, SZ, P]
+    lib.gqa_decode_multi.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, P, SZ, P]
+    lib.gqa_decode_fp8.argtypes = [P, P, P, F, F, P, P, P, I, I, I, I, I, F, I, I, P, SZ, P]
     lib.gqa_error_string.argtypes = [I]
     lib.gqa_error_string.restype = ctypes.c_char_p
     for name in ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states",
                  "gqa_merge_states", "gqa_status", "gqa_decode_host",
                  "gqa_decode_fixed_split_workspace_size", "gqa_decode_fixed_split",
-                 "gqa_select_schedule", "gqa_decode_auto"):
+                 "gqa_select_schedule", "gqa_decode_auto", "gqa_decode_multi",
+                 "gqa_decode_fp8"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -251,6 +255,65 @@ def gqa_decode_auto(q, k_cache, v_cache, block_table, seq_lens, seq_lens_host=No
                                  Hkv, D, bs, scale, mb, nb, _ptr(buf), buf.numel(),
                                  _stream_ptr(stream))
     _check("gqa_decode_auto", rc)
+    return out
+
+
+def gqa_decode_fp8(q, k8, v8, k_scale: float, v_scale: float, block_table, seq_lens, out=None,
+                   scale=None, workspace: Optional[Workspace] = None, stream=None) -> torch.Tensor:
+    """Decode over an FP8 E4M3 cache: k8, v8 uint8 (or float8_e4m3fn) in the bf16 caches'
+    layouts, values e4m3 * k_scale / e4m3 * v_scale.  Returns out [B, Hq, D] bf16."""
+    import torch as _t
+    lib = load_library()
+    k8 = k8.view(_t.uint8) if k8.dtype != _t.uint8 else k8
+    v8 = v8.view(_t.uint8) if v8.dtype != _t.uint8 else v8
+    B, Hq, Hkv, D, bs, mb, nb = _shape(q, k8, block_table)
+    dev = q.device
+    _require(q, "q", _t.bfloat16, dev)
+    _require(k8, "k_cache", _t.uint8, dev)
+    _require(v8, "v_cache", _t.uint8, dev)
+    _require(seq_lens, "seq_lens", _t.int32, dev)
+    if block_table is not None:
+        _require(block_table, "block_table", _t.int32, dev)
+    if out is None:
+        out = _t.empty_like(q)
+    _require(out, "out", _t.bfloat16, dev)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    ws = default_workspace(dev) if workspace is None else workspace
+    buf = ws.get(workspace_size(B, Hq, Hkv, D, dev.index))
+    with _t.cuda.device(dev):
+        rc = lib.gqa_decode_fp8(_ptr(q), _ptr(k8), _ptr(v8), float(k_scale), float(v_scale),
+                                _ptr(block_table), _ptr(seq_lens), _ptr(out), B, Hq, Hkv, D, bs,
+                                scale, mb, nb, _ptr(buf), buf.numel(), _stream_ptr(stream))
+    _check("gqa_decode_fp8", rc)
+    return out
+
+
+def gqa_decode_multi(q, k_cache, v_cache, block_table, seq_lens, out=None, scale=None,
+                     workspace: Optional[Workspace] = None, stream=None) -> torch.Tensor:
+    """Several query tokens per request (speculative verification): q [B, Q, Hq, D] bf16;
+    token i of request b sees keys t <= L_b - Q + i.  Returns out [B, Q, Hq, D]."""
+    lib = load_library()
+    if q.dim() != 4:
+        raise ValueError("q must be [B, Q, Hq, D]")
+    B, Q, Hq, D = q.shape
+    _, _, Hkv, _, bs, mb, nb = _shape(q.view(B, Q * Hq, D), k_cache, block_table)
+    dev = q.device
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _require(t, n, torch.bfloat16, dev)
+    _require(seq_lens, "seq_lens", torch.int32, dev)
+    if block_table is not None:
+        _require(block_table, "block_table", torch.int32, dev)
+    if out is None:
+        out = torch.empty_like(q)
+    _require(out, "out", torch.bfloat16, dev)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    ws = default_workspace(dev) if workspace is None else workspace
+    buf = ws.get(workspace_size(B, Hq, Hkv, D, dev.index))
+    with torch.cuda.device(dev):
+        rc = lib.gqa_decode_multi(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                  _ptr(seq_lens), _ptr(out), B, Q, Hq, Hkv, D, bs, scale, mb, nb,
+                                  _ptr(buf), buf.numel(), _stream_ptr(stream))
+    _check("gqa_decode_multi", rc)
     return out
 
 

@@ -52,10 +52,10 @@ int head_chunk(int G)
 
 using KernelFn = void (*)(Params);
 
-template <int D, int GC, bool ST>
+template <int D, int GC, bool ST, bool F8>
 KernelFn simt_fn()
 {
-    return gqa_decode_simt_kernel<D, GC, ST>;
+    return gqa_decode_simt_kernel<D, GC, ST, F8>;
 }
 
 struct Variant {
@@ -66,20 +66,20 @@ struct Variant {
     int slot_floats;
 };
 
-template <int D, int GC, bool ST>
+template <int D, int GC, bool ST, bool F8>
 Variant make_variant()
 {
-    using C = SimtCfg<D, GC>;
-    return Variant{simt_fn<D, GC, ST>(), C::THREADS, C::smem_bytes(GQA_MAX_BATCH), &C::smem_bytes,
+    using C = SimtCfg<D, GC, F8>;
+    return Variant{simt_fn<D, GC, ST, F8>(), C::THREADS, C::smem_bytes(GQA_MAX_BATCH), &C::smem_bytes,
                    C::SLOT_FLOATS};
 }
 
-template <bool ST>
+template <bool ST, bool F8>
 bool pick_gc(int D, int GC, Variant &v)
 {
 #define GQA_CASE(DD, GG)                       \
     if (D == DD && GC == GG) {                 \
-        v = make_variant<DD, GG, ST>();        \
+        v = make_variant<DD, GG, ST, F8>();    \
         return true;                           \
     }
     GQA_CASE(64, 1) GQA_CASE(64, 2) GQA_CASE(64, 4) GQA_CASE(64, 8)
@@ -89,10 +89,12 @@ bool pick_gc(int D, int GC, Variant &v)
     return false;
 }
 
-bool pick_variant(int D, int G, bool states, Variant &v)
+bool pick_variant(int D, int G, bool states, Variant &v, bool fp8 = false)
 {
     const int gc = head_chunk(G);
-    return states ? pick_gc<true>(D, gc, v) : pick_gc<false>(D, gc, v);
+    if (fp8)
+        return !states && pick_gc<false, true>(D, gc, v);
+    return states ? pick_gc<true, false>(D, gc, v) : pick_gc<false, false>(D, gc, v);
 }
 
 // Per-device cache: SM count and, per kernel, resident CTAs per SM.
@@ -204,10 +206,11 @@ int tc_box_rows(const int32_t *block_table, int block_size)
     return (block_size >= 8 && 128 % block_size == 0) ? block_size : 0;
 }
 
+// R = query rows per KV head (query tokens x G).
 bool tc_applicable(bool states, int B, int Hq, int Hkv, int D, int block_size,
-                   const int32_t *block_table, int num_blocks)
+                   const int32_t *block_table, int num_blocks, int R)
 {
-    if (states || D != TcCfg::D || Hq / Hkv < TC_MIN_G || B > TcCfg::MAX_BATCH)
+    if (states || D != TcCfg::D || R < TC_MIN_G || B > TcCfg::MAX_BATCH)
         return false;
     if (tc_box_rows(block_table, block_size) == 0)
         return false;
@@ -298,7 +301,8 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
                const int32_t *block_table, const int32_t *seq_lens, const int32_t *kv_begin,
                const int32_t *kv_end, void *out, float *acc, float *m, float *l, int B, int Hq,
                int Hkv, int D, int block_size, float scale, int max_blocks, int num_blocks,
-               void *workspace, size_t workspace_bytes, void *stream, int nsplit = 0)
+               void *workspace, size_t workspace_bytes, void *stream, int nsplit = 0,
+               int qlen = 1, bool fp8 = false, float k_scale = 1.0f, float v_scale = 1.0f)
 {
     int rc = check_shape(B, Hq, Hkv, D, block_size, block_table, max_blocks, num_blocks, scale);
     if (rc)
@@ -314,19 +318,26 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || (out && !aligned16(out)))
         return GQA_ERR_MISALIGNED;
     const int G = Hq / Hkv;
-    const bool use_tc = tc_applicable(states, B, Hq, Hkv, D, block_size, block_table, num_blocks);
+    if (qlen < 1 || qlen > GQA_MAX_QLEN)
+        return GQA_ERR_INVALID_ARG;
+    const int R = qlen * G;  // query rows per KV head
+    // FP8 caches run on the CUDA-core kernel.
+    const bool use_tc =
+        !fp8 && tc_applicable(states, B, Hq, Hkv, D, block_size, block_table, num_blocks, R);
     Variant v;
-    if (!use_tc && !pick_variant(D, G, states, v))
+    if (!use_tc && !pick_variant(D, G, states, v, fp8))
+        return GQA_ERR_UNSUPPORTED;
+    if (!use_tc && qlen > 1)  // several query tokens run on the tensor-core kernel only
         return GQA_ERR_UNSUPPORTED;
     int dev = 0;
     if ((rc = current_device(dev)))
         return rc;
     int ctas = 0;
-    if ((rc = use_tc ? tc_ctas(G, dev, ctas) : persistent_ctas(v, dev, ctas)))
+    if ((rc = use_tc ? tc_ctas(R, dev, ctas) : persistent_ctas(v, dev, ctas)))
         return rc;
     if (nsplit > 0 && !use_tc)
         return GQA_ERR_UNSUPPORTED;
-    const int hch_tc = (G + TcCfg::NP - 1) / TcCfg::NP;
+    const int hch_tc = (R + TcCfg::NP - 1) / TcCfg::NP;
     const int64_t items = nsplit > 0 ? (int64_t)B * Hkv * hch_tc * nsplit : 0;
     if (items > (int64_t)1 << 30)
         return GQA_ERR_INVALID_ARG;
@@ -358,13 +369,16 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     p.Hq = Hq;
     p.Hkv = Hkv;
     p.G = G;
+    p.qlen = qlen;
+    p.R = R;
     p.block_size = block_size;
     p.max_blocks = block_table ? max_blocks : 1;
     p.num_blocks = block_table ? num_blocks : B;
     p.hch = use_tc ? hch_tc : (G + head_chunk(G) - 1) / head_chunk(G);
     p.nsplit = nsplit > 0 ? nsplit : 0;
     p.capacity = block_table ? (int64_t)max_blocks * block_size : (int64_t)block_size;
-    p.qscale = scale * LOG2E;
+    p.qscale = scale * LOG2E * (fp8 ? k_scale : 1.0f);
+    p.vscale = fp8 ? v_scale : 1.0f;
     p.timeline = nullptr;
     // Magic number for t / block_size (t < 2^31): see page_of().
     {
@@ -385,12 +399,12 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         if (nsplit > 0) {
             // Fixed split: as many CTAs as chunks, in waves; no CTA waits for another.
             const cudaStream_t st = static_cast<cudaStream_t>(stream);
-            tc_kernel_for(G)<<<(unsigned)items, TcCfg::THREADS, TcCfg::smem_bytes(B), st>>>(p, tmk, tmv,
+            tc_kernel_for(R)<<<(unsigned)items, TcCfg::THREADS, TcCfg::smem_bytes(B), st>>>(p, tmk, tmv,
                                                                                         box_rows);
             if (B > 0 && nsplit > 1) {
-                const int nv = G <= 4 ? 4 : (G <= 8 ? 8 : 16);
+                const int nv = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
                 const int64_t threads = (int64_t)B * Hkv * hch_tc * nv * TcCfg::D;
-                tc_merge_for(G)<<<(unsigned)((threads + 127) / 128), 128, 0, st>>>(p);
+                tc_merge_for(R)<<<(unsigned)((threads + 127) / 128), 128, 0, st>>>(p);
             }
             return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
         }
@@ -407,7 +421,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, tc_kernel_for(G), p, tmk, tmv, box_rows) != cudaSuccess)
+        if (cudaLaunchKernelEx(&cfg, tc_kernel_for(R), p, tmk, tmv, box_rows) != cudaSuccess)
             return GQA_ERR_CUDA;
     } else {
         v.fn<<<ctas, v.threads, v.smem(B), static_cast<cudaStream_t>(stream)>>>(p);
@@ -534,9 +548,9 @@ int gqa_decode_workspace_size(int B, int Hq, int Hkv, int D, int device, size_t 
         const size_t t = layout_for(ctas, v.slot_floats).total;
         best = t > best ? t : best;
     }
-    if (D == TcCfg::D && Hq / Hkv >= TC_MIN_G) {
+    if (D == TcCfg::D) {  // the tensor-core kernel (also for several query tokens)
         int ctas = 0;
-        if ((rc = tc_ctas(Hq / Hkv, device, ctas)))
+        if ((rc = tc_ctas(TC_MIN_G, device, ctas)))
             return rc;
         const size_t t = layout_for(ctas, TcCfg::SLOT_FLOATS).total;
         best = t > best ? t : best;
@@ -611,6 +625,31 @@ int gqa_decode_auto(const void *q, const void *k_cache, const void *v_cache,
     return run_decode(false, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, out,
                       nullptr, nullptr, nullptr, B, Hq, Hkv, D, block_size, scale,
                       max_blocks_per_seq, num_blocks, workspace, workspace_bytes, stream, ns);
+}
+
+int gqa_decode_multi(const void *q, const void *k_cache, const void *v_cache,
+                     const int32_t *block_table, const int32_t *seq_lens, void *out, int B,
+                     int qlen, int Hq, int Hkv, int D, int block_size, float scale,
+                     int max_blocks_per_seq, int num_blocks, void *workspace,
+                     size_t workspace_bytes, void *stream)
+{
+    return run_decode(false, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, out,
+                      nullptr, nullptr, nullptr, B, Hq, Hkv, D, block_size, scale,
+                      max_blocks_per_seq, num_blocks, workspace, workspace_bytes, stream, 0, qlen);
+}
+
+int gqa_decode_fp8(const void *q, const void *k_cache, const void *v_cache, float k_scale,
+                   float v_scale, const int32_t *block_table, const int32_t *seq_lens, void *out,
+                   int B, int Hq, int Hkv, int D, int block_size, float scale,
+                   int max_blocks_per_seq, int num_blocks, void *workspace,
+                   size_t workspace_bytes, void *stream)
+{
+    if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || k_scale <= 0.f || v_scale <= 0.f)
+        return GQA_ERR_INVALID_ARG;
+    return run_decode(false, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, out,
+                      nullptr, nullptr, nullptr, B, Hq, Hkv, D, block_size, scale,
+                      max_blocks_per_seq, num_blocks, workspace, workspace_bytes, stream, 0, 1,
+                      true, k_scale, v_scale);
 }
 
 int gqa_decode_states(const void *q, const void *k_cache, const void *v_cache,

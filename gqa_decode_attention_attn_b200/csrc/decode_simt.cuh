@@ -29,13 +29,17 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include "schedule.cuh"
 
 namespace gqa {
 
-template <int D, int GC>
+// F8: the cache holds FP8 E4M3 bytes (one scale per tensor, folded into q for K
+// and applied at the output for V) instead of bf16.
+template <int D, int GC, bool F8 = false>
 struct SimtCfg {
+    static constexpr int KB = F8 ? 1 : 2;              // bytes per cache element
     // 7 consumer warps + 1 producer = 256 threads: the register allocator grants
     // up to 255 registers per thread only to CTAs of at most 256 threads, and each
     // warp needs ~200 to keep 8 steps (16 tokens at D = 128) in flight per tile.
@@ -46,7 +50,8 @@ struct SimtCfg {
     static constexpr int TPW = 32 / LPT;               // tokens per warp step
     static constexpr int TOKW = STEPS * TPW;           // tokens per warp per tile
     static constexpr int T = NC * TOKW;                // tokens per tile: 56 KB of K+V
-    static constexpr int STAGES = (D == 256 && GC == 8) ? 2 : 3;  // shared-memory budget
+    // Shared-memory budget: the FP8 ring holds twice the tiles in the same bytes.
+    static constexpr int STAGES = ((D == 256 && GC == 8) ? 2 : 3) * (F8 ? 2 : 1);
     static constexpr int NV = STEPS * GC;              // partial dots per lane
     static constexpr int NF = NV >= LPT ? NV / LPT : 1;  // whole scores per lane
     static constexpr int REP = NV >= LPT ? 1 : LPT / NV; // lanes sharing one score
@@ -55,7 +60,7 @@ struct SimtCfg {
     static constexpr int TILE_ELEMS = T * D;
     static constexpr int SCRATCH_PER_WARP = GC * D + ((2 * GC + 3) / 4) * 4;  // 16-byte multiple
     static constexpr int PSCR_PER_WARP = ((NS + GC + 3) / 4) * 4;              // scores + alphas
-    static constexpr size_t RING_BYTES = 2ull * STAGES * TILE_ELEMS * sizeof(uint16_t);
+    static constexpr size_t RING_BYTES = 2ull * STAGES * TILE_ELEMS * KB;
     static constexpr size_t BAR_OFF = RING_BYTES;
     static constexpr size_t FLAG_OFF = BAR_OFF + 2 * STAGES * sizeof(uint64_t);
     static constexpr size_t SCRATCH_OFF = FLAG_OFF + 32 * sizeof(int);
@@ -97,14 +102,44 @@ __device__ __forceinline__ void transpose_reduce(float (&v)[NV], int lane)
     }
 }
 
-template <int D, int GC, bool STATES>
-__global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
+// Eight consecutive cache elements at `src` (16 bytes of bf16 or 8 of FP8 E4M3)
+// as four float2, exactly.
+template <bool F8>
+__device__ __forceinline__ void load8(const unsigned char *src, float2 &a, float2 &b, float2 &c,
+                                      float2 &d)
+{
+    if constexpr (F8) {
+        const uint2 w = *reinterpret_cast<const uint2 *>(src);
+        const uint32_t ww[2] = {w.x, w.y};
+        float2 f[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(
+                (__nv_fp8x2_storage_t)((ww[j >> 1] >> (16 * (j & 1))) & 0xffffu), __NV_E4M3);
+            f[j] = __half22float2(*reinterpret_cast<const __half2 *>(&h));
+        }
+        a = f[0];
+        b = f[1];
+        c = f[2];
+        d = f[3];
+    } else {
+        const uint4 w = *reinterpret_cast<const uint4 *>(src);
+        a = bf16x2_to_float2(w.x);
+        b = bf16x2_to_float2(w.y);
+        c = bf16x2_to_float2(w.z);
+        d = bf16x2_to_float2(w.w);
+    }
+}
+
+template <int D, int GC, bool STATES, bool F8 = false>
+__global__ void __launch_bounds__(SimtCfg<D, GC, F8>::THREADS, 1)
     gqa_decode_simt_kernel(const Params p)
 {
-    using C = SimtCfg<D, GC>;
+    using C = SimtCfg<D, GC, F8>;
+    constexpr int KB = C::KB;
     extern __shared__ __align__(128) unsigned char smem[];
-    uint16_t *kring = reinterpret_cast<uint16_t *>(smem);
-    uint16_t *vring = kring + C::STAGES * C::TILE_ELEMS;
+    unsigned char *kring = smem;
+    unsigned char *vring = kring + (size_t)C::STAGES * C::TILE_ELEMS * KB;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
     uint64_t *empty = full + C::STAGES;
     int *stage_bad = reinterpret_cast<int *>(smem + C::FLAG_OFF);  // [STAGES]
@@ -229,7 +264,7 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
                 if (row && (blk < 0 || blk >= p.num_blocks))
                     bad = true;
             }
-            uint32_t bytes = (uint32_t)n * D * 4;
+            uint32_t bytes = (uint32_t)n * D * 2 * KB;
             if (__any_sync(0xffffffffu, bad)) {
                 uint32_t skip = 0;
                 for (int pc = lane; pc < npieces; pc += 32) {
@@ -237,7 +272,7 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
                     if (blk < 0 || blk >= p.num_blocks) {
                         const int pg = pg0 + pc;
                         skip += (uint32_t)(min((int64_t)tok0 + n, (int64_t)(pg + 1) * bs) -
-                                           max((int64_t)tok0, (int64_t)pg * bs)) * D * 4;
+                                           max((int64_t)tok0, (int64_t)pg * bs)) * D * 2 * KB;
                     }
                 }
 #pragma unroll
@@ -248,7 +283,7 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
                     atomicOr(p.status, DEV_BAD_BLOCK);
             }
             if (lane == 0) {
-                stage_bad[s] = bytes != (uint32_t)n * D * 4;
+                stage_bad[s] = bytes != (uint32_t)n * D * 2 * KB;
                 stage_n[s] = n;
                 mbar_arrive_expect_tx(&full[s], bytes);
             }
@@ -263,9 +298,11 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
                 const int z = (int)min((int64_t)tok0 + n, (int64_t)(pg + 1) * bs);
                 const int64_t src = ((blk * p.Hkv + it.kvh) * (int64_t)bs + (a - pg * bs)) * D;
                 const int dst = s * C::TILE_ELEMS + (a - tok0) * D;
-                const uint32_t nb = (uint32_t)(z - a) * D * 2;
-                bulk_copy_g2s(kring + dst, p.k + src, nb, &full[s], pol);
-                bulk_copy_g2s(vring + dst, p.v + src, nb, &full[s], pol);
+                const uint32_t nb = (uint32_t)(z - a) * D * KB;
+                bulk_copy_g2s(kring + (size_t)dst * KB,
+                              reinterpret_cast<const unsigned char *>(p.k) + src * KB, nb, &full[s], pol);
+                bulk_copy_g2s(vring + (size_t)dst * KB,
+                              reinterpret_cast<const unsigned char *>(p.v) + src * KB, nb, &full[s], pol);
             }
         }
         // Never leave copies in flight: wait for the last issued phase of each slot.
@@ -336,8 +373,8 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
         } else {
             poisoned |= stage_bad[s] != 0;
             const int n = stage_n[s];
-            const uint16_t *Ks = kring + s * C::TILE_ELEMS;
-            const uint16_t *Vs = vring + s * C::TILE_ELEMS;
+            const unsigned char *Ks = kring + (size_t)s * C::TILE_ELEMS * KB;
+            const unsigned char *Vs = vring + (size_t)s * C::TILE_ELEMS * KB;
             const int tok_base = cw * C::TOKW;  // this warp's first token in the tile
 
             // BMM1: partial dots over this lane's 8 dimensions.
@@ -345,11 +382,9 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
 #pragma unroll
             for (int st = 0; st < C::STEPS; ++st) {
                 const int tt = tok_base + st * C::TPW + grp;
-                uint4 w = make_uint4(0, 0, 0, 0);
+                float2 k0 = make_float2(0.f, 0.f), k1 = k0, k2 = k0, k3 = k0;
                 if (tt < n)
-                    w = *reinterpret_cast<const uint4 *>(Ks + tt * D + d0);
-                const float2 k0 = bf16x2_to_float2(w.x), k1 = bf16x2_to_float2(w.y);
-                const float2 k2 = bf16x2_to_float2(w.z), k3 = bf16x2_to_float2(w.w);
+                    load8<F8>(Ks + (size_t)(tt * D + d0) * KB, k0, k1, k2, k3);
 #pragma unroll
                 for (int g = 0; g < GC; ++g) {
                     float2 a = __fmul2_rn(q2[g][0], k0);
@@ -418,9 +453,8 @@ __global__ void __launch_bounds__(SimtCfg<D, GC>::THREADS, 1)
                 const int tl = st * C::TPW + grp;  // token inside this warp's share
                 if (tok_base + tl >= n)
                     continue;
-                const uint4 w = *reinterpret_cast<const uint4 *>(Vs + (tok_base + tl) * D + d0);
-                const float2 v0 = bf16x2_to_float2(w.x), v1 = bf16x2_to_float2(w.y);
-                const float2 v2 = bf16x2_to_float2(w.z), v3 = bf16x2_to_float2(w.w);
+                float2 v0, v1, v2, v3;
+                load8<F8>(Vs + (size_t)((tok_base + tl) * D + d0) * KB, v0, v1, v2, v3);
                 float pv[GC];
                 if constexpr (GC % 4 == 0) {
 #pragma unroll

@@ -222,8 +222,8 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             continue;
         int64_t begin, len;
         const bool bad = !request_range<false>(p, b, begin, len);
-        for (int e = tid; e < p.Hq * D; e += C::THREADS)
-            write_result<false>(p, (int64_t)b * p.Hq + e / D, e % D, D, 0.f, -INFINITY, 0.f, bad);
+        for (int e = tid; e < p.qlen * p.Hq * D; e += C::THREADS)
+            write_result<false>(p, (int64_t)b * p.qlen * p.Hq + e / D, e % D, D, 0.f, -INFINITY, 0.f, bad);
     }
 
     if (start < end && (warp == 0 || warp == 6)) {
@@ -477,15 +477,16 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 lsum[g] = lred[g] + lred[NV + g] + lred[2 * NV + g] + lred[3 * NV + g];
             const bool pois = *reinterpret_cast<volatile int *>(poison_flag) != 0;
             const bool complete = piece_first == cur.seg0 && last_excl == cur.seg0 + cur.nb;
-            const int rows = min(NV, G - cur.hc * NP);
-            const int64_t row0 = (int64_t)cur.b * p.Hq + (int64_t)cur.kvh * G + (int64_t)cur.hc * NP;
+            const int rows = min(NV, p.R - cur.hc * NP);
+            const int r0 = cur.hc * NP;
             const int64_t vseg = ((int64_t)cur.b * p.Hkv + cur.kvh) * p.hch + cur.hc;
             float *slot = p.slots + (p.nsplit ? c : 2 * c + (piece_first == start ? 0 : 1)) * (int64_t)SLOT;
             if (complete) {
 #pragma unroll
                 for (int g = 0; g < NV; ++g)
                     if (g < rows)
-                        write_result<false>(p, row0 + g, ti, D, acc[g], m_ref[g], lsum[g], pois);
+                        write_result<false>(p, out_row(p, cur.b, cur.kvh, r0 + g), ti, D, acc[g], m_ref[g],
+                                            lsum[g], pois);
             } else {
 #pragma unroll
                 for (int g = 0; g < NV; ++g)
@@ -506,7 +507,8 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             if (!complete) {
                 if (stid == 0)
                     *poison_flag = 0;
-                pending[npending++] = PendingPiece{cur.seg0, piece_first, last_excl, vseg, row0, cur.nb, rows};
+                pending[npending++] =
+                    PendingPiece{cur.seg0, piece_first, last_excl, vseg, 0, cur.nb, rows, cur.b, cur.kvh, r0};
             } else if (stid == 0) {
                 *poison_flag = 0;
             }
@@ -524,6 +526,8 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             fold_pend = false;
         };
 
+        int len_b = -1;
+        int64_t req_len = 0;
         int k = 0;
         for (int64_t i = start; i < end; ++i, ++k) {
             if (i > start)
@@ -542,10 +546,9 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                     const int x = stid + 128 * r;
                     const int half = x >> 7, g = (x & 127) >> 3, cc = x & 7;
                     uint4 w = make_uint4(0, 0, 0, 0);
-                    if (it.hc * NP + g < G)
+                    if (it.hc * NP + g < p.R)
                         w = __ldg(reinterpret_cast<const uint4 *>(
-                            p.q + (((int64_t)it.b * p.Hq + (int64_t)it.kvh * G + it.hc * NP + g) * D +
-                                   half * 64 + cc * 8)));
+                            p.q + (out_row(p, it.b, it.kvh, it.hc * NP + g) * D + half * 64 + cc * 8)));
                     *reinterpret_cast<uint4 *>(qd + half * NP * 128 + g * 128 + ((cc ^ (g & 7)) << 4)) = w;
                 }
                 fence_proxy_async_smem();
@@ -582,6 +585,27 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             mbar_arrive(&s_free[b]);
             flush_fold();  // before this tile may rescale acc again
             const bool valid = ti < n;
+            // Several query tokens (qlen > 1): query row r is token r / G at position
+            // L - qlen + r / G and sees keys up to its own position, so a key `past`
+            // places beyond L - qlen is hidden from the rows of tokens before it.
+            bool see[NV];
+#pragma unroll
+            for (int g = 0; g < NV; ++g)
+                see[g] = valid;
+            if (p.qlen > 1) {
+                if (it.b != len_b) {
+                    len_b = it.b;
+                    int64_t b0, l0;
+                    request_range<false>(p, len_b, b0, l0);
+                    req_len = l0;
+                }
+                const int64_t past = (int64_t)it.j * T + ti - (req_len - p.qlen);
+                if (past > 0) {  // only the last qlen - 1 keys of a request
+#pragma unroll
+                    for (int g = 0; g < NV; ++g)
+                        see[g] = see[g] && past <= (it.hc * NP + g) / G;
+                }
+            }
             // x = scaled score relative to the reference.  While no score of the tile
             // exceeds its reference by more than 2^LAZY, P = 2^x <= 2^LAZY is used as
             // is and nothing is rescaled: one barrier-OR decides that for the CTA.
@@ -589,7 +613,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             float xmax = -INFINITY;
 #pragma unroll
             for (int g = 0; g < NV; ++g) {
-                x[g] = valid ? fmaf(sc[g], qscale, -m_ref[g]) : -INFINITY;
+                x[g] = see[g] ? fmaf(sc[g], qscale, -m_ref[g]) : -INFINITY;
                 xmax = fmaxf(xmax, x[g]);
             }
             const bool moved = named_barrier_or(1, 128, !(xmax <= C::LAZY));
@@ -599,7 +623,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 float mx[NV];
 #pragma unroll
                 for (int g = 0; g < NV; ++g)
-                    mx[g] = valid ? sc[g] * qscale : -INFINITY;
+                    mx[g] = see[g] ? sc[g] * qscale : -INFINITY;
                 const float wmax = warp_transpose_reduce<NV, true>(mx, lane);
                 float *tred = red + (k & 1) * 4 * NP;
                 if (lane % LPH == 0)
@@ -611,7 +635,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                     const float m_new = tm > m_ref[g] + C::LAZY ? tm : m_ref[g];
                     alpha[g] = m_new == m_ref[g] ? 1.f : fast_exp2(m_ref[g] - m_new);
                     m_ref[g] = m_new;
-                    x[g] = (valid && m_new != -INFINITY) ? fmaf(sc[g], qscale, -m_new) : -INFINITY;
+                    x[g] = (see[g] && m_new != -INFINITY) ? fmaf(sc[g], qscale, -m_new) : -INFINITY;
                     l_t[g] *= alpha[g];
                     acc[g] *= alpha[g];
                 }
@@ -692,7 +716,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         for (int x = 0; x < npending; ++x) {
             const PendingPiece &pp = pending[x];
             merge_segment_gather<NV, D, 128>(p, c, pp.seg0, pp.nb, pp.first, pp.vseg, W, P, pp.rows,
-                                             pp.row0, reinterpret_cast<int *>(pbuf),
+                                             pp.b, pp.kvh, pp.r0, reinterpret_cast<int *>(pbuf),
                                              reinterpret_cast<float *>(ring), misc + 20, stid, 1,
                                              abort_flag);
         }
@@ -736,8 +760,7 @@ __global__ void __launch_bounds__(128)
     const int e = (int)(gid - j * (NV * D)), g = e / D, d = e - g * D;
     const int b = (int)(j / units);
     const int u = (int)(j - (int64_t)b * units), kvh = u / p.hch, hc = u - kvh * p.hch;
-    const int G = p.G;
-    if (g >= min(NV, G - hc * NP))
+    if (g >= min(NV, p.R - hc * NP))
         return;
     int64_t begin, len;
     request_range<false>(p, b, begin, len);
@@ -776,8 +799,7 @@ __global__ void __launch_bounds__(128)
             ls = fmaf(w, lv[q], ls);
         }
     }
-    const int64_t row = (int64_t)b * p.Hq + (int64_t)kvh * G + (int64_t)hc * NP + g;
-    write_result<false>(p, row, d, D, a, mx, ls, ls != ls);
+    write_result<false>(p, out_row(p, b, kvh, hc * NP + g), d, D, a, mx, ls, ls != ls);
 }
 
 }  // namespace gqa

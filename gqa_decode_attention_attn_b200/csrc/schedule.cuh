@@ -48,10 +48,13 @@ struct Params {
     int B, Hq, Hkv, G, block_size, max_blocks, num_blocks;
     int hch;                      // head chunks per KV head
     int nsplit;                   // 0: stream-K runs; n > 0: fixed split, CTA = (segment, chunk)
+    int qlen;                     // query tokens per request (1: decode; > 1: speculative verify)
+    int R;                        // query rows per KV head: qlen * G
     int64_t capacity;             // tokens a request can hold
     uint32_t bs_magic;            // token -> page division by block_size (see page_of)
     int bs_shift;
-    float qscale;                 // scale * log2(e): scores are kept in log2 units
+    float qscale;                 // scale * log2(e) (* k_scale for FP8): scores in log2 units
+    float vscale;                 // FP8 cache: v_scale, applied to the output (1 for bf16)
     unsigned long long *timeline; // optional [grid][4]: start ns, end ns, SM id, tiles
 };
 
@@ -171,10 +174,19 @@ __device__ __forceinline__ bool request_range(const Params &p, int b, int64_t &b
     } else {
         b1 = p.seq_lens[b];
     }
-    bool ok = b0 >= 0 && b1 >= b0 && b1 <= p.capacity;
+    // With qlen > 1 query tokens the request must hold at least qlen tokens.
+    bool ok = b0 >= 0 && b1 >= b0 && b1 <= p.capacity && (STATES || p.qlen <= 1 || b1 >= p.qlen);
     begin = ok ? b0 : 0;
     len = ok ? b1 - b0 : 0;
     return ok;
+}
+
+// Output row of query row r (0 <= r < R) of (request b, KV head kvh): query token
+// r / G, head kvh * G + r % G, in the [B, qlen, Hq] row order of q and out.
+__device__ __forceinline__ int64_t out_row(const Params &p, int b, int kvh, int r)
+{
+    const int i = r / p.G, h = r - i * p.G;
+    return ((int64_t)b * p.qlen + i) * p.Hq + (int64_t)kvh * p.G + h;
 }
 
 // Bounded wait on an mbarrier phase.  On timeout: status bit, CTA abort flag.
@@ -210,7 +222,7 @@ __device__ __forceinline__ void write_result(const Params &p, int64_t row, int d
             p.st_l[row] = poisoned ? __int_as_float(0x7fc00000) : ls;
         }
     } else {
-        float o = poisoned ? __int_as_float(0x7fc00000) : (ls > 0.f ? a / ls : 0.f);
+        float o = poisoned ? __int_as_float(0x7fc00000) : (ls > 0.f ? p.vscale * a / ls : 0.f);
         __nv_bfloat16 h = __float2bfloat16_rn(o);
         p.out[row * D + d] = *reinterpret_cast<uint16_t *>(&h);
     }
@@ -349,8 +361,9 @@ __device__ __forceinline__ int ticket_add(int *counter, int v)
 // its tiles: the segment cannot complete before its other owners reach the end
 // of their runs anyway, and a merge in mid-run would stall this CTA's pipeline.
 struct PendingPiece {
-    int64_t seg0, first, end, vseg, row0;
+    int64_t seg0, first, end, vseg, row0;  // row0: first output row (qlen = 1 kernels)
     int nb, rows;
+    int b, kvh, r0;                        // request, KV head, first query row (any qlen)
 };
 
 // Slot of CTA cc's piece of the segment starting at tile seg0, or -1 if cc owns

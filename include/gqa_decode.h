@@ -73,6 +73,7 @@ extern "C" {
 
 #define GQA_MAX_BATCH 4096   /* requests per call */
 #define GQA_MAX_QHEADS 256   /* query heads per request */
+#define GQA_MAX_QLEN 16      /* query tokens per request (gqa_decode_multi) */
 
 /*
  * Bytes of device workspace gqa_decode / gqa_decode_states need for this shape
@@ -162,6 +163,42 @@ GQA_API int gqa_decode_auto(const void *q, const void *k_cache, const void *v_ca
                             const int32_t *seq_lens_host, void *out, int B, int Hq, int Hkv, int D,
                             int block_size, float scale, int max_blocks_per_seq, int num_blocks,
                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Several query tokens per request: the verification pass of speculative
+ * decoding, where the large model scores the qlen drafted positions in one pass
+ * (Inference optimization: KV cache, MQA/GQA, batching..., section 5
+ * "Speculative decoding").  The drafted tokens' keys and values are already in
+ * the cache: request b holds L_b >= qlen tokens and query token i sits at
+ * position L_b - qlen + i, seeing the keys t <= L_b - qlen + i (causal inside the
+ * qlen new tokens).
+ *   q, out  [B, qlen, Hq, D] bf16; everything else as gqa_decode.
+ * 1 <= qlen <= GQA_MAX_QLEN; qlen = 1 is gqa_decode.  Runs on the tensor-core
+ * kernel (D = 128, qlen * Hq / Hkv >= 4, its page sizes, B <= 1024), the query
+ * rows of one KV head (qlen x G) sharing every K/V tile; other shapes return
+ * GQA_ERR_UNSUPPORTED for qlen > 1.  A request with L_b < qlen gets NaN rows and
+ * GQA_DEV_BAD_LENGTH.  Workspace: gqa_decode_workspace_size(B, Hq, Hkv, D, ...).
+ */
+GQA_API int gqa_decode_multi(const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *block_table, const int32_t *seq_lens, void *out,
+                             int B, int qlen, int Hq, int Hkv, int D, int block_size, float scale,
+                             int max_blocks_per_seq, int num_blocks, void *workspace,
+                             size_t workspace_bytes, void *stream);
+
+/*
+ * gqa_decode over an FP8 E4M3 cache (the FP8 KV cache of Attention co-design for
+ * long-context inference, list of techniques): k_cache and v_cache hold one byte
+ * per element in the bf16 caches' layouts; element values are e4m3(byte) * k_scale
+ * and e4m3(byte) * v_scale (one scale per tensor, > 0).  q and out stay bf16.  A
+ * decode step reads half the bytes.  Runs on the CUDA-core kernel, the E4M3 bytes
+ * widened exactly in registers (k_scale folded into q, v_scale applied to the
+ * output).  Workspace: gqa_decode_workspace_size.  Errors as gqa_decode.
+ */
+GQA_API int gqa_decode_fp8(const void *q, const void *k_cache, const void *v_cache, float k_scale,
+                           float v_scale, const int32_t *block_table, const int32_t *seq_lens,
+                           void *out, int B, int Hq, int Hkv, int D, int block_size, float scale,
+                           int max_blocks_per_seq, int num_blocks, void *workspace,
+                           size_t workspace_bytes, void *stream);
 
 /*
  * Partial softmax states of every query row over the key range

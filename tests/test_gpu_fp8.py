@@ -1,0 +1,49 @@
+"""GPU parity of the FP8 E4M3 cache path (gqa_decode_fp8) against the fp64 oracle
+on the same E4M3 bytes and scales."""
+import pytest
+import torch
+
+import gqa_decode_attention_attn_b200 as gq
+import oracle
+import workloads
+from gpu_util import parity
+from workloads import fp8_caches, make_problem
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # B, Hq, Hkv, D, lens, block_size
+    (3, 8, 2, 128, [1, 63, 700], None),
+    (2, 32, 8, 128, [3000, 129], 16),       # G = 4
+    (2, 8, 8, 128, [500, 64], 32),          # MHA
+    (2, 16, 1, 128, [1000, 7], 64),         # G = 16: two head chunks
+    (3, 4, 2, 64, [128, 127, 900], 8),
+    (2, 16, 4, 256, [777, 2], 16),
+    (1, 4, 1, 128, [60000], None),          # one long segment over every CTA
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}_Hq{c[1]}_Hkv{c[2]}_D{c[3]}_bs{c[5]}")
+def test_fp8_matches_oracle(case):
+    B, Hq, Hkv, D, lens, bs = case
+    p = make_problem("fp8", B, Hq, Hkv, D, lens, seed=500 + sum(lens) + D, block_size=bs,
+                     spare_blocks=2 if bs else 0, key_outlier_frac=0.01)
+    k8, v8, ks, vs = fp8_caches(p)
+    d = p.to("cuda")
+    ws = gq.Workspace(d.q.device)
+    out = gq.gqa_decode_fp8(d.q, k8.cuda(), v8.cuda(), ks, vs, d.block_table, d.seq_lens,
+                            scale=p.scale, workspace=ws)
+    assert ws.status() == 0
+    ref = oracle.gqa_decode_fp8(p.q, k8, v8, ks, vs, p.block_table, p.seq_lens, p.scale)
+    parity(out.cpu(), ref, str(case), bf16_scaled=True)
+
+
+def test_fp8_llama3_shape_sampled_rows():
+    p = workloads.workload("llama3_8b_fp8")
+    k8, v8, ks, vs = fp8_caches(p)
+    d = p.to("cuda")
+    out = gq.gqa_decode_fp8(d.q, k8.cuda(), v8.cuda(), ks, vs, d.block_table, d.seq_lens,
+                            scale=p.scale).cpu()
+    rows = (0, 24)  # one request's first query heads
+    ref = oracle.gqa_decode_fp8(p.q, k8, v8, ks, vs, p.block_table, p.seq_lens, p.scale, rows=rows)
+    parity(out.reshape(-1, 128)[rows[0]:rows[1]], ref, "llama3_8b_fp8 rows")

@@ -84,8 +84,10 @@ class Problem:
         return int(self.seq_lens.to(torch.int64).sum())
 
     def algorithmic_bytes(self) -> int:
-        """K + V rows of valid tokens, plus q read and out written, all bf16."""
-        return kv_bytes(self.seq_lens, self.Hkv, self.D) + 2 * 2 * self.B * self.Hq * self.D
+        """K + V rows of valid tokens (bf16, or one byte per element for an FP8 cache),
+        plus q read and out written (bf16)."""
+        eb = int(self.meta.get("kv_elem_bytes", 2))
+        return kv_bytes(self.seq_lens, self.Hkv, self.D, eb) + 2 * 2 * self.B * self.Hq * self.D
 
     def block_table_bytes(self) -> int:
         if self.block_table is None:
@@ -218,12 +220,28 @@ def varlen_lengths(B: int, seed: int, lo: int = 1024, hi: int = 131072):
     return [int(x) for x in L.clamp(lo, hi).tolist()]
 
 
+def fp8_caches(p: Problem):
+    """The problem's caches stored as FP8 E4M3 with one scale per tensor (the largest
+    finite magnitude maps to 448, E4M3's largest finite value): returns (k8, v8,
+    k_scale, v_scale), k8/v8 uint8 in the bf16 caches' layouts.  Poisoned slots
+    stay NaN (E4M3 0x7F)."""
+    out = []
+    for c in (p.k_cache, p.v_cache):
+        f = c.to(torch.float32)
+        fin = f[torch.isfinite(f)]
+        amax = float(fin.abs().max()) if fin.numel() else 1.0
+        sc = amax / 448.0 if amax > 0 else 1.0
+        out.append(((f / sc).to(torch.float8_e4m3fn).view(torch.uint8), sc))
+    return out[0][0], out[1][0], out[0][1], out[1][1]
+
+
 WORKLOADS = {
     "tiny": "B=1, Hq=4, Hkv=1, D=128, L=512, contiguous",
     "llama3_8b": "B=16, Hq=32, Hkv=8, D=128, L=8192, contiguous, 1% of keys x8",
     "long_256k": "B=1, Hq=32, Hkv=2, D=128, L=262144, 64-token pages, permuted table",
     "varlen_paged": "B=64, Hq=32, Hkv=8, D=128, L log-uniform [1024, 131072], 16-token pages",
 }
+WORKLOADS["llama3_8b_fp8"] = "llama3_8b's shape and values, K/V stored as FP8 E4M3"
 for _i, (_hq, _hkv, _d) in enumerate(SWEEP):
     WORKLOADS[f"sweep_{_hq}_{_hkv}_{_d}"] = f"B=8, Hq={_hq}, Hkv={_hkv}, D={_d}, L=32768, contiguous"
 
@@ -234,6 +252,10 @@ def workload(name: str) -> Problem:
         return make_problem(name, 1, 4, 1, 128, [512], seed=1000)
     if name == "llama3_8b":
         return make_problem(name, 16, 32, 8, 128, [8192] * 16, seed=1001, key_outlier_frac=0.01)
+    if name == "llama3_8b_fp8":
+        p = make_problem(name, 16, 32, 8, 128, [8192] * 16, seed=1001, key_outlier_frac=0.01)
+        p.meta["kv_elem_bytes"] = 1
+        return p
     if name == "long_256k":
         return make_problem(name, 1, 32, 2, 128, [262144], seed=1002, block_size=64)
     if name == "varlen_paged":
