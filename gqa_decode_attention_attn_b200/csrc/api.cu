@@ -169,13 +169,16 @@ int persistent_ctas(const Variant &v, int dev, int &ctas)
 // Tensor-core kernel for G query heads per KV head: the softmax carries 4, 8 or
 // 16 heads (the smallest that holds G, capped at the MMA width 16).
 using TcKernelFn = void (*)(Params, CUtensorMap, CUtensorMap, int);
-TcKernelFn tc_kernel_for(int G)
+TcKernelFn tc_kernel_for(int G, bool mq = false)
 {
+    if (mq)
+        return G <= 4 ? gqa_decode_tc_kernel<4, true>
+                      : (G <= 8 ? gqa_decode_tc_kernel<8, true> : gqa_decode_tc_kernel<16, true>);
     if (G <= 4)
-        return gqa_decode_tc_kernel<4>;
+        return gqa_decode_tc_kernel<4, false>;
     if (G <= 8)
-        return gqa_decode_tc_kernel<8>;
-    return gqa_decode_tc_kernel<16>;
+        return gqa_decode_tc_kernel<8, false>;
+    return gqa_decode_tc_kernel<16, false>;
 }
 
 using MergeFn = void (*)(Params);
@@ -188,9 +191,9 @@ MergeFn tc_merge_for(int G)
     return merge_split_kernel<16>;
 }
 
-int tc_ctas(int G, int dev, int &ctas)
+int tc_ctas(int G, int dev, int &ctas, bool mq = false)
 {
-    return persistent_ctas_fn(reinterpret_cast<const void *>(tc_kernel_for(G)), TcCfg::THREADS,
+    return persistent_ctas_fn(reinterpret_cast<const void *>(tc_kernel_for(G, mq)), TcCfg::THREADS,
                               TcCfg::smem_bytes(TcCfg::MAX_BATCH), dev, ctas);
 }
 
@@ -333,7 +336,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     if ((rc = current_device(dev)))
         return rc;
     int ctas = 0;
-    if ((rc = use_tc ? tc_ctas(R, dev, ctas) : persistent_ctas(v, dev, ctas)))
+    if ((rc = use_tc ? tc_ctas(R, dev, ctas, qlen > 1) : persistent_ctas(v, dev, ctas)))
         return rc;
     if (nsplit > 0 && !use_tc)
         return GQA_ERR_UNSUPPORTED;
@@ -399,7 +402,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         if (nsplit > 0) {
             // Fixed split: as many CTAs as chunks, in waves; no CTA waits for another.
             const cudaStream_t st = static_cast<cudaStream_t>(stream);
-            tc_kernel_for(R)<<<(unsigned)items, TcCfg::THREADS, TcCfg::smem_bytes(B), st>>>(p, tmk, tmv,
+            tc_kernel_for(R, qlen > 1)<<<(unsigned)items, TcCfg::THREADS, TcCfg::smem_bytes(B), st>>>(p, tmk, tmv,
                                                                                         box_rows);
             if (B > 0 && nsplit > 1) {
                 const int nv = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
@@ -421,7 +424,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, tc_kernel_for(R), p, tmk, tmv, box_rows) != cudaSuccess)
+        if (cudaLaunchKernelEx(&cfg, tc_kernel_for(R, qlen > 1), p, tmk, tmv, box_rows) != cudaSuccess)
             return GQA_ERR_CUDA;
     } else {
         v.fn<<<ctas, v.threads, v.smem(B), static_cast<cudaStream_t>(stream)>>>(p);

@@ -105,7 +105,9 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[NV], int lane)
 // NV: query heads the softmax threads carry (4, 8 or 16 = the MMA width NP);
 // the MMAs always run NP = 16 columns, and columns NV..NP-1 of S and O are
 // never read (zero Q rows in, P left as is: an O column depends on its P column only).
-template <int NV>
+// MQ: several query tokens per request (causal mask inside them); the one-token
+// decode instantiation carries no mask code.
+template <int NV, bool MQ>
 __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     gqa_decode_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv, int box_rows)
@@ -232,7 +234,10 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         const CUtensorMap *map = is_k ? &tmk : &tmv;
         unsigned char *base = ring + (is_k ? 0 : C::V_RING_OFF);
         uint64_t *full = is_k ? k_full : v_full, *emptyb = is_k ? k_empty : v_empty;
-        const uint64_t pol = l2_evict_first_policy();
+        // K/V are read once, except when several 16-head chunks of a KV head (G > 16)
+        // stream the same tiles at about the same time: then L2 keeps them for the
+        // other chunks.
+        const uint64_t pol = p.hch > 1 ? l2_evict_normal_policy() : l2_evict_first_policy();
         TileIter it;
         it.init(start, prefix, B, units, p.hch);
         // Global row of this lane's box of tile `ti` (lane < boxes), or -1 for a
@@ -592,7 +597,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
 #pragma unroll
             for (int g = 0; g < NV; ++g)
                 see[g] = valid;
-            if (p.qlen > 1) {
+            if (MQ) {
                 if (it.b != len_b) {
                     len_b = it.b;
                     int64_t b0, l0;

@@ -80,6 +80,14 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy()
     return pol;
 }
 
+// L2 policy for data read again soon by other CTAs: evict normally.
+__device__ __forceinline__ uint64_t l2_evict_normal_policy()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 // Bulk copy of `bytes` (multiple of 16; both addresses 16-byte aligned) from
 // global to this CTA's shared memory; completion is signalled on `bar` as
 // transaction bytes.  No multicast.
