@@ -37,12 +37,14 @@ METRIC = "decode-attn KV GB/s & % of B200 HBM peak; µs/step at 1 GPU"
 SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
-KERNEL_SOURCES = ["gqa_decode_attention_attn_b200/csrc/decode_simt.cuh",
-                  "gqa_decode_attention_attn_b200/csrc/decode_tc.cuh",
-                  "gqa_decode_attention_attn_b200/csrc/gather_merge.cuh",
-                  "gqa_decode_attention_attn_b200/csrc/schedule.cuh",
-                  "gqa_decode_attention_attn_b200/csrc/tc.cuh",
-                  "gqa_decode_attention_attn_b200/csrc/ptx.cuh"]
+_CSRC = "gqa_decode_attention_attn_b200/csrc/"
+# The sources each kernel is compiled from (a traffic record is valid while they
+# are unchanged).
+KERNEL_SOURCES = {
+    "tc": [_CSRC + f for f in ("decode_tc.cuh", "gather_merge.cuh", "schedule.cuh", "tc.cuh",
+                               "ptx.cuh")],
+    "simt": [_CSRC + f for f in ("decode_simt.cuh", "schedule.cuh", "ptx.cuh")],
+}
 
 
 def kernel_for(p) -> str:
@@ -89,24 +91,25 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the sources of the named kernel (a kernel_for() name)."""
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES["tc" if "tc_kernel" in kernel else "simt"]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, kernel: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on the
-    current kernel source (else None)."""
+    current source of the kernel (else None)."""
     path = os.path.join(ROOT, "profiles", f"decode_{workload}_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
     except (OSError, ValueError):
         return None
-    if rec.get("kernel_source_sha256_16") != kernel_source_hash():
+    if rec.get("kernel_source_sha256_16") != kernel_source_hash(kernel):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -389,7 +392,7 @@ def main():
 
     line = None
     if rank == 0:
-        traffic = profiled_traffic(p.name)
+        traffic = profiled_traffic(p.name, kernel_for(p))
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
