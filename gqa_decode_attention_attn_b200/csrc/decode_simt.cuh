@@ -31,6 +31,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include <type_traits>
+
 #include "schedule.cuh"
 
 namespace gqa {
@@ -102,14 +104,17 @@ __device__ __forceinline__ void transpose_reduce(float (&v)[NV], int lane)
     }
 }
 
-// Eight consecutive cache elements at `src` (16 bytes of bf16 or 8 of FP8 E4M3)
-// as four float2, exactly.
+// Eight consecutive cache elements: one uint4 of bf16 or one uint2 of FP8 E4M3.
+// Typed (not char) so that the compiler may keep shared-memory loads and stores
+// of other types apart.
 template <bool F8>
-__device__ __forceinline__ void load8(const unsigned char *src, float2 &a, float2 &b, float2 &c,
-                                      float2 &d)
+using Vec8 = typename std::conditional<F8, uint2, uint4>::type;
+
+// Eight cache elements as four float2, exactly.
+template <bool F8>
+__device__ __forceinline__ void load8(const Vec8<F8> &w, float2 &a, float2 &b, float2 &c, float2 &d)
 {
     if constexpr (F8) {
-        const uint2 w = *reinterpret_cast<const uint2 *>(src);
         const uint32_t ww[2] = {w.x, w.y};
         float2 f[4];
 #pragma unroll
@@ -123,7 +128,6 @@ __device__ __forceinline__ void load8(const unsigned char *src, float2 &a, float
         c = f[2];
         d = f[3];
     } else {
-        const uint4 w = *reinterpret_cast<const uint4 *>(src);
         a = bf16x2_to_float2(w.x);
         b = bf16x2_to_float2(w.y);
         c = bf16x2_to_float2(w.z);
@@ -138,8 +142,11 @@ __global__ void __launch_bounds__(SimtCfg<D, GC, F8>::THREADS, 1)
     using C = SimtCfg<D, GC, F8>;
     constexpr int KB = C::KB;
     extern __shared__ __align__(128) unsigned char smem[];
-    unsigned char *kring = smem;
-    unsigned char *vring = kring + (size_t)C::STAGES * C::TILE_ELEMS * KB;
+    // The rings, typed by element (bf16 bits or FP8 bytes; the other pair unused).
+    uint16_t *kring = reinterpret_cast<uint16_t *>(smem);
+    uint16_t *vring = kring + C::STAGES * C::TILE_ELEMS;
+    uint8_t *kring8 = smem;
+    uint8_t *vring8 = kring8 + C::STAGES * C::TILE_ELEMS;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
     uint64_t *empty = full + C::STAGES;
     int *stage_bad = reinterpret_cast<int *>(smem + C::FLAG_OFF);  // [STAGES]
@@ -299,10 +306,13 @@ __global__ void __launch_bounds__(SimtCfg<D, GC, F8>::THREADS, 1)
                 const int64_t src = ((blk * p.Hkv + it.kvh) * (int64_t)bs + (a - pg * bs)) * D;
                 const int dst = s * C::TILE_ELEMS + (a - tok0) * D;
                 const uint32_t nb = (uint32_t)(z - a) * D * KB;
-                bulk_copy_g2s(kring + (size_t)dst * KB,
-                              reinterpret_cast<const unsigned char *>(p.k) + src * KB, nb, &full[s], pol);
-                bulk_copy_g2s(vring + (size_t)dst * KB,
-                              reinterpret_cast<const unsigned char *>(p.v) + src * KB, nb, &full[s], pol);
+                if constexpr (F8) {
+                    bulk_copy_g2s(kring8 + dst, reinterpret_cast<const uint8_t *>(p.k) + src, nb, &full[s], pol);
+                    bulk_copy_g2s(vring8 + dst, reinterpret_cast<const uint8_t *>(p.v) + src, nb, &full[s], pol);
+                } else {
+                    bulk_copy_g2s(kring + dst, p.k + src, nb, &full[s], pol);
+                    bulk_copy_g2s(vring + dst, p.v + src, nb, &full[s], pol);
+                }
             }
         }
         // Never leave copies in flight: wait for the last issued phase of each slot.
@@ -373,8 +383,10 @@ __global__ void __launch_bounds__(SimtCfg<D, GC, F8>::THREADS, 1)
         } else {
             poisoned |= stage_bad[s] != 0;
             const int n = stage_n[s];
-            const unsigned char *Ks = kring + (size_t)s * C::TILE_ELEMS * KB;
-            const unsigned char *Vs = vring + (size_t)s * C::TILE_ELEMS * KB;
+            const uint16_t *Ks = kring + s * C::TILE_ELEMS;
+            const uint16_t *Vs = vring + s * C::TILE_ELEMS;
+            const uint8_t *Ks8 = kring8 + s * C::TILE_ELEMS;
+            const uint8_t *Vs8 = vring8 + s * C::TILE_ELEMS;
             const int tok_base = cw * C::TOKW;  // this warp's first token in the tile
 
             // BMM1: partial dots over this lane's 8 dimensions.
@@ -382,9 +394,21 @@ __global__ void __launch_bounds__(SimtCfg<D, GC, F8>::THREADS, 1)
 #pragma unroll
             for (int st = 0; st < C::STEPS; ++st) {
                 const int tt = tok_base + st * C::TPW + grp;
-                float2 k0 = make_float2(0.f, 0.f), k1 = k0, k2 = k0, k3 = k0;
-                if (tt < n)
-                    load8<F8>(Ks + (size_t)(tt * D + d0) * KB, k0, k1, k2, k3);
+                float2 k0, k1, k2, k3;
+                if constexpr (F8) {
+                    uint2 w = make_uint2(0, 0);
+                    if (tt < n)
+                        w = *reinterpret_cast<const uint2 *>(Ks8 + tt * D + d0);
+                    load8<true>(w, k0, k1, k2, k3);
+                } else {
+                    uint4 w = make_uint4(0, 0, 0, 0);
+                    if (tt < n)
+                        w = *reinterpret_cast<const uint4 *>(Ks + tt * D + d0);
+                    k0 = bf16x2_to_float2(w.x);
+                    k1 = bf16x2_to_float2(w.y);
+                    k2 = bf16x2_to_float2(w.z);
+                    k3 = bf16x2_to_float2(w.w);
+                }
 #pragma unroll
                 for (int g = 0; g < GC; ++g) {
                     float2 a = __fmul2_rn(q2[g][0], k0);
@@ -454,7 +478,16 @@ __global__ void __launch_bounds__(SimtCfg<D, GC, F8>::THREADS, 1)
                 if (tok_base + tl >= n)
                     continue;
                 float2 v0, v1, v2, v3;
-                load8<F8>(Vs + (size_t)((tok_base + tl) * D + d0) * KB, v0, v1, v2, v3);
+                if constexpr (F8) {
+                    load8<true>(*reinterpret_cast<const uint2 *>(Vs8 + (tok_base + tl) * D + d0), v0, v1,
+                                v2, v3);
+                } else {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(Vs + (tok_base + tl) * D + d0);
+                    v0 = bf16x2_to_float2(w.x);
+                    v1 = bf16x2_to_float2(w.y);
+                    v2 = bf16x2_to_float2(w.z);
+                    v3 = bf16x2_to_float2(w.w);
+                }
                 float pv[GC];
                 if constexpr (GC % 4 == 0) {
 #pragma unroll
