@@ -1,0 +1,53 @@
+"""CPU checks of host-side helpers: FP8 cache preparation, the bench's kernel
+mapping and traffic-record keying, workspace sizes."""
+import os
+import sys
+
+import torch
+
+import gqa_decode_attention_attn_b200 as gq
+import workloads
+from workloads import fp8_caches, make_problem
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def test_fp8_caches_range_scale_and_poison():
+    p = make_problem("fp8h", 2, 8, 2, 64, [37, 5], seed=3, block_size=8, spare_blocks=2,
+                     key_outlier_frac=0.05)
+    k8, v8, ks, vs = fp8_caches(p)
+    assert k8.dtype == torch.uint8 and k8.shape == p.k_cache.shape
+    assert ks > 0 and vs > 0
+    kf = k8.view(torch.float8_e4m3fn).to(torch.float32)
+    fin = torch.isfinite(p.k_cache.float())
+    assert torch.all(torch.isnan(kf[~fin]))          # poison stays NaN
+    assert torch.all(kf[fin].abs() <= 448)          # every finite value representable
+    assert kf[fin].abs().max() == 448               # the largest maps to E4M3's maximum
+    # dequantised values track the bf16 originals within E4M3 precision (3 mantissa bits)
+    err = (kf[fin] * ks - p.k_cache.float()[fin]).abs()
+    assert torch.all(err <= p.k_cache.float()[fin].abs() * 2 ** -4 + ks * 2 ** -9)
+
+
+def test_bench_kernel_mapping():
+    import bench
+    assert bench.kernel_for(workloads.make_problem("a", 1, 32, 8, 128, [10], seed=1)).startswith(
+        "gqa_decode_tc_kernel")
+    assert bench.kernel_for(workloads.make_problem("b", 1, 32, 32, 128, [10], seed=1)) == \
+        "gqa_decode_simt_kernel"                     # G = 1
+    assert bench.kernel_for(workloads.make_problem("c", 1, 32, 8, 64, [10], seed=1)) == \
+        "gqa_decode_simt_kernel"                     # D = 64
+    assert bench.kernel_for(workloads.make_problem("d", 1, 32, 8, 128, [10], seed=1,
+                                                   block_size=48)) == "gqa_decode_simt_kernel"
+    p = workloads.make_problem("e", 1, 32, 8, 128, [10], seed=1)
+    p.meta["kv_elem_bytes"] = 1
+    assert "FP8" in bench.kernel_for(p)
+    # traffic records are keyed to each kernel's own sources
+    assert bench.kernel_source_hash("gqa_decode_tc_kernel<4>") != \
+        bench.kernel_source_hash("gqa_decode_simt_kernel")
+
+
+def test_fixed_split_workspace_grows_with_splits():
+    sizes = [gq.fixed_split_workspace_size(16, 32, 8, 128, s, 0) for s in (1, 2, 8, 32)]
+    assert sizes == sorted(sizes) and sizes[0] < sizes[-1]
