@@ -169,32 +169,49 @@ int persistent_ctas(const Variant &v, int dev, int &ctas)
 // Tensor-core kernel for G query heads per KV head: the softmax carries 4, 8 or
 // 16 heads (the smallest that holds G, capped at the MMA width 16).
 using TcKernelFn = void (*)(Params, CUtensorMap, CUtensorMap, int);
-TcKernelFn tc_kernel_for(int G, bool mq = false)
+template <bool MQ, int DH>
+TcKernelFn tc_kernel_nv(int G)
 {
-    if (mq)
-        return G <= 4 ? gqa_decode_tc_kernel<4, true>
-                      : (G <= 8 ? gqa_decode_tc_kernel<8, true> : gqa_decode_tc_kernel<16, true>);
     if (G <= 4)
-        return gqa_decode_tc_kernel<4, false>;
+        return gqa_decode_tc_kernel<4, MQ, DH>;
     if (G <= 8)
-        return gqa_decode_tc_kernel<8, false>;
-    return gqa_decode_tc_kernel<16, false>;
+        return gqa_decode_tc_kernel<8, MQ, DH>;
+    return gqa_decode_tc_kernel<16, MQ, DH>;
+}
+
+TcKernelFn tc_kernel_for(int G, bool mq = false, int D = 128)
+{
+    if (D == 64)
+        return mq ? tc_kernel_nv<true, 64>(G) : tc_kernel_nv<false, 64>(G);
+    return mq ? tc_kernel_nv<true, 128>(G) : tc_kernel_nv<false, 128>(G);
 }
 
 using MergeFn = void (*)(Params);
-MergeFn tc_merge_for(int G)
+template <int DH>
+MergeFn tc_merge_nv(int G)
 {
     if (G <= 4)
-        return merge_split_kernel<4>;
+        return merge_split_kernel<4, DH>;
     if (G <= 8)
-        return merge_split_kernel<8>;
-    return merge_split_kernel<16>;
+        return merge_split_kernel<8, DH>;
+    return merge_split_kernel<16, DH>;
 }
 
-int tc_ctas(int G, int dev, int &ctas, bool mq = false)
+MergeFn tc_merge_for(int G, int D = 128)
 {
-    return persistent_ctas_fn(reinterpret_cast<const void *>(tc_kernel_for(G, mq)), TcCfg::THREADS,
+    return D == 64 ? tc_merge_nv<64>(G) : tc_merge_nv<128>(G);
+}
+
+int tc_ctas(int G, int dev, int &ctas, bool mq = false, int D = 128)
+{
+    return persistent_ctas_fn(reinterpret_cast<const void *>(tc_kernel_for(G, mq, D)), TcCfg::THREADS,
                               TcCfg::smem_bytes(TcCfg::MAX_BATCH), dev, ctas);
+}
+
+// Head dimensions the tensor-core kernel is built for.
+bool tc_head_dim(int D)
+{
+    return D == 64 || D == 128;
 }
 
 // ---- tensor-core path: applicability and tensor maps -------------------------
@@ -213,7 +230,7 @@ int tc_box_rows(const int32_t *block_table, int block_size)
 bool tc_applicable(bool states, int B, int Hq, int Hkv, int D, int block_size,
                    const int32_t *block_table, int num_blocks, int R)
 {
-    if (states || D != TcCfg::D || R < TC_MIN_G || B > TcCfg::MAX_BATCH)
+    if (states || !tc_head_dim(D) || R < TC_MIN_G || B > TcCfg::MAX_BATCH)
         return false;
     if (tc_box_rows(block_table, block_size) == 0)
         return false;
@@ -242,15 +259,15 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// 2-D view of a cache as [rows, 128] bf16; boxes of 64 columns x box_rows rows,
+// 2-D view of a cache as [rows, D] bf16; boxes of 64 columns x box_rows rows,
 // 128-byte swizzle (the layout the tensor cores read), zero fill out of range.
-bool encode_kv_map(CUtensorMap *map, const void *base, int64_t rows, int box_rows)
+bool encode_kv_map(CUtensorMap *map, const void *base, int64_t rows, int box_rows, int D)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn)
         return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)TcCfg::D, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)TcCfg::D * 2};
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
     const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
@@ -336,7 +353,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     if ((rc = current_device(dev)))
         return rc;
     int ctas = 0;
-    if ((rc = use_tc ? tc_ctas(R, dev, ctas, qlen > 1) : persistent_ctas(v, dev, ctas)))
+    if ((rc = use_tc ? tc_ctas(R, dev, ctas, qlen > 1, D) : persistent_ctas(v, dev, ctas)))
         return rc;
     if (nsplit > 0 && !use_tc)
         return GQA_ERR_UNSUPPORTED;
@@ -397,17 +414,17 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         const int box_rows = tc_box_rows(block_table, block_size);
         const int64_t rows = (block_table ? (int64_t)num_blocks : (int64_t)B) * Hkv * block_size;
         CUtensorMap tmk, tmv;
-        if (!encode_kv_map(&tmk, k_cache, rows, box_rows) || !encode_kv_map(&tmv, v_cache, rows, box_rows))
+        if (!encode_kv_map(&tmk, k_cache, rows, box_rows, D) || !encode_kv_map(&tmv, v_cache, rows, box_rows, D))
             return GQA_ERR_CUDA;
         if (nsplit > 0) {
             // Fixed split: as many CTAs as chunks, in waves; no CTA waits for another.
             const cudaStream_t st = static_cast<cudaStream_t>(stream);
-            tc_kernel_for(R, qlen > 1)<<<(unsigned)items, TcCfg::THREADS, TcCfg::smem_bytes(B), st>>>(p, tmk, tmv,
-                                                                                        box_rows);
+            tc_kernel_for(R, qlen > 1, D)<<<(unsigned)items, TcCfg::THREADS, TcCfg::smem_bytes(B), st>>>(
+                p, tmk, tmv, box_rows);
             if (B > 0 && nsplit > 1) {
                 const int nv = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
-                const int64_t threads = (int64_t)B * Hkv * hch_tc * nv * TcCfg::D;
-                tc_merge_for(R)<<<(unsigned)((threads + 127) / 128), 128, 0, st>>>(p);
+                const int64_t threads = (int64_t)B * Hkv * hch_tc * nv * D;
+                tc_merge_for(R, D)<<<(unsigned)((threads + 127) / 128), 128, 0, st>>>(p);
             }
             return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
         }
@@ -424,7 +441,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, tc_kernel_for(R, qlen > 1), p, tmk, tmv, box_rows) != cudaSuccess)
+        if (cudaLaunchKernelEx(&cfg, tc_kernel_for(R, qlen > 1, D), p, tmk, tmv, box_rows) != cudaSuccess)
             return GQA_ERR_CUDA;
     } else {
         v.fn<<<ctas, v.threads, v.smem(B), static_cast<cudaStream_t>(stream)>>>(p);
@@ -451,7 +468,7 @@ int select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int 
         if (seq_lens[b] < 0)
             return GQA_ERR_INVALID_ARG;
     const int G = Hq / Hkv;
-    const bool tc = D == TcCfg::D && G >= TC_MIN_G && B <= TcCfg::MAX_BATCH;
+    const bool tc = tc_head_dim(D) && G >= TC_MIN_G && B <= TcCfg::MAX_BATCH;
     const int64_t units = (int64_t)Hkv * (tc ? (G + TcCfg::NP - 1) / TcCfg::NP
                                              : (G + head_chunk(G) - 1) / head_chunk(G));
     // Microseconds per 128-token K+V tile for a CTA while `active` CTAs stream.
@@ -551,7 +568,7 @@ int gqa_decode_workspace_size(int B, int Hq, int Hkv, int D, int device, size_t 
         const size_t t = layout_for(ctas, v.slot_floats).total;
         best = t > best ? t : best;
     }
-    if (D == TcCfg::D) {  // the tensor-core kernel (also for several query tokens)
+    if (tc_head_dim(D)) {  // the tensor-core kernel (also for several query tokens)
         int ctas = 0;
         if ((rc = tc_ctas(TC_MIN_G, device, ctas)))
             return rc;

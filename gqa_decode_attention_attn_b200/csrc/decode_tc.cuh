@@ -1,5 +1,5 @@
 // decode_tc.cuh -- persistent stream-K decode attention on the 5th-generation
-// tensor cores (tcgen05), for groups of G >= 4 query heads per KV head (D = 128).
+// tensor cores (tcgen05), for groups of G >= 4 query heads per KV head (D = 128 or 64).
 // The MMAs run M = 128 tokens by N = 16 heads; the softmax threads carry only
 // the NV <= 16 heads that exist.
 //
@@ -107,13 +107,19 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[NV], int lane)
 // never read (zero Q rows in, P left as is: an O column depends on its P column only).
 // MQ: several query tokens per request (causal mask inside them); the one-token
 // decode instantiation carries no mask code.
-template <int NV, bool MQ>
+// DH: head dimension, 128 or 64.  At 64, BMM1 takes 4 K-steps over the one
+// 64-column half that is loaded, and BMM2 still runs M = 128 over V^T with rows
+// 64..127 held at zero in shared memory (written once, never loaded), so the
+// O rows 64..127 are zero and are not read back.
+template <int NV, bool MQ, int DH = 128>
 __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     gqa_decode_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv, int box_rows)
 {
     using C = TcCfg;
-    constexpr int S = C::STAGES, NP = C::NP, D = C::D, T = C::T;
+    constexpr int S = C::STAGES, NP = C::NP, D = DH, T = C::T;
+    constexpr int HALVES = D / 64;  // 64-column halves loaded per tile
+    static_assert(D == 64 || D == 128, "head dimension");
     constexpr int SLOT = slot_floats(NV, D);
     constexpr int LPH = 32 / NV;  // lanes per head after a transposed warp reduction
     static_assert(NV == 4 || NV == 8 || NV == 16, "softmax head count");
@@ -167,6 +173,18 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
+    }
+    if constexpr (HALVES == 1) {
+        // V^T rows 64..127 (the upper half of every V slot) stay zero for the whole
+        // launch; the TMA loads only the lower half.  Likewise Q's upper half.
+        for (int x = tid; x < S * C::BOX_BYTES / 16; x += C::THREADS) {
+            const int slot = x / (C::BOX_BYTES / 16), off = x % (C::BOX_BYTES / 16);
+            reinterpret_cast<uint4 *>(ring + C::V_RING_OFF + (size_t)slot * C::TILE_BYTES + C::BOX_BYTES)[off] =
+                make_uint4(0, 0, 0, 0);
+        }
+        for (int x = tid; x < 2 * C::QBUF_BYTES / 16; x += C::THREADS)
+            reinterpret_cast<uint4 *>(qbuf)[x] = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();
     }
     for (int b = tid; b < B; b += C::THREADS) {
         int64_t begin, len;
@@ -288,13 +306,14 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                         atomicOr(p.status, DEV_BAD_BLOCK);
                 }
                 const uint32_t boxes = (uint32_t)(nbox - __popc(badmask));
-                mbar_arrive_expect_tx(&full[s], boxes * 2u * (uint32_t)box_rows * 128u);
+                mbar_arrive_expect_tx(&full[s], boxes * (uint32_t)HALVES * (uint32_t)box_rows * 128u);
             }
             __syncwarp();
             if (lane < nbox && !bad) {
                 unsigned char *d = base + (size_t)s * C::TILE_BYTES + (size_t)lane * box_rows * 128;
                 tma_load_2d(d, map, 0, row, &full[s], pol);
-                tma_load_2d(d + C::BOX_BYTES, map, 64, row, &full[s], pol);
+                if constexpr (HALVES == 2)
+                    tma_load_2d(d + C::BOX_BYTES, map, 64, row, &full[s], pol);
             }
         }
         if (lane == 0) {
@@ -489,13 +508,14 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             if (complete) {
 #pragma unroll
                 for (int g = 0; g < NV; ++g)
-                    if (g < rows)
+                    if (g < rows && ti < D)
                         write_result<false>(p, out_row(p, cur.b, cur.kvh, r0 + g), ti, D, acc[g], m_ref[g],
                                             lsum[g], pois);
             } else {
 #pragma unroll
                 for (int g = 0; g < NV; ++g)
-                    slot[g * D + ti] = acc[g];
+                    if (ti < D)
+                        slot[g * D + ti] = acc[g];
                 if (ti < NV) {
                     float mv = m_ref[0], lvv = lsum[0];
 #pragma unroll
@@ -547,7 +567,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 ++piece;
                 unsigned char *qd = qbuf + ((piece - 1) & 1) * C::QBUF_BYTES;
 #pragma unroll
-                for (int r = 0; r < 2; ++r) {
+                for (int r = 0; r < HALVES; ++r) {
                     const int x = stid + 128 * r;
                     const int half = x >> 7, g = (x & 127) >> 3, cc = x & 7;
                     uint4 w = make_uint4(0, 0, 0, 0);
@@ -690,7 +710,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             if (!valid) {
                 unsigned char *vr = ring + C::V_RING_OFF + (size_t)s * C::TILE_BYTES + ti * 128;
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
+                for (int h = 0; h < HALVES; ++h)
 #pragma unroll
                     for (int cc = 0; cc < 8; ++cc)
                         *reinterpret_cast<uint4 *>(vr + h * C::BOX_BYTES + cc * 16) = make_uint4(0, 0, 0, 0);
@@ -750,11 +770,11 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
 // c) in chunk order; a segment with fewer than two non-empty chunks was written by
 // the decode kernel itself.  (Attention co-design for long-context inference,
 // section "FlashAttention and GEMM shapes": FlashDecoding's split-KV reduction.)
-template <int NV>
+template <int NV, int DH = 128>
 __global__ void __launch_bounds__(128)
     merge_split_kernel(const Params p)
 {
-    constexpr int D = TcCfg::D, NP = TcCfg::NP, T = TcCfg::T;
+    constexpr int D = DH, NP = TcCfg::NP, T = TcCfg::T;
     constexpr int SLOT = slot_floats(NV, D);
     constexpr int U = 8;  // chunks per batch of independent loads
     const int64_t units = (int64_t)p.Hkv * p.hch;

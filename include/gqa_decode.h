@@ -96,7 +96,7 @@ GQA_API int gqa_decode_workspace_size(int B, int Hq, int Hkv, int D, int device,
  * requests spread over many SMs (LeanAttention decode tiles digest, sections
  * "Exact softmax that merges piece by piece" and "Hardware-sized work units").
  * A (request, KV head) split across CTAs is merged exactly from the partial
- * states.  On the tensor-core kernel (D = 128, at least 4 query heads per KV head,
+ * states.  On the tensor-core kernel (D = 64 or 128, at least 4 query heads per KV head,
  * pages of 8..128 tokens dividing 128 or multiples of 128, B <= 1024) the launch
  * is cooperative: every CTA is resident, and the owners of a split segment wait
  * (bounded, GQA_DEV_TIMEOUT on expiry) for one another and merge one slice of its
@@ -174,7 +174,7 @@ GQA_API int gqa_decode_auto(const void *q, const void *k_cache, const void *v_ca
  * qlen new tokens).
  *   q, out  [B, qlen, Hq, D] bf16; everything else as gqa_decode.
  * 1 <= qlen <= GQA_MAX_QLEN; qlen = 1 is gqa_decode.  Runs on the tensor-core
- * kernel (D = 128, qlen * Hq / Hkv >= 4, its page sizes, B <= 1024), the query
+ * kernel (D = 64 or 128, qlen * Hq / Hkv >= 4, its page sizes, B <= 1024), the query
  * rows of one KV head (qlen x G) sharing every K/V tile; other shapes return
  * GQA_ERR_UNSUPPORTED for qlen > 1.  A request with L_b < qlen gets NaN rows and
  * GQA_DEV_BAD_LENGTH.  Workspace: gqa_decode_workspace_size(B, Hq, Hkv, D, ...).

@@ -18,13 +18,15 @@ CASES = [
     (3, 16, 1, [100, 5000, 1280], 16, 64),     # more chunks than tiles: empty chunks
     (2, 64, 2, [4000, 999], 32, 4),             # G = 32: two head chunks
     (5, 8, 1, [0, 17, 0, 2500, 64], 16, 5),     # empty requests
+    (2, 32, 4, [9000, 130], 16, 5, 64),         # D = 64
 ]
 
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}_Hq{c[1]}_Hkv{c[2]}_bs{c[4]}_s{c[5]}")
 def test_fixed_split_matches_oracle_and_stream_k(case):
-    B, Hq, Hkv, lens, bs, splits = case
-    p = make_problem("fixed", B, Hq, Hkv, 128, lens, seed=700 + sum(lens) + splits, block_size=bs,
+    B, Hq, Hkv, lens, bs, splits, *rest = case
+    D = rest[0] if rest else 128
+    p = make_problem("fixed", B, Hq, Hkv, D, lens, seed=700 + sum(lens) + splits, block_size=bs,
                      key_outlier_frac=0.01)
     d = p.to("cuda")
     ws = gq.Workspace(d.q.device)
@@ -39,7 +41,7 @@ def test_fixed_split_matches_oracle_and_stream_k(case):
 
 
 def test_fixed_split_rejects_cuda_core_shapes():
-    p = make_problem("fixed64", 2, 8, 2, 64, [100, 50], seed=3)
+    p = make_problem("fixedg1", 2, 8, 8, 128, [100, 50], seed=3)    # G = 1
     d = p.to("cuda")
     with pytest.raises(gq.GqaError):
         gq.gqa_decode_fixed_split(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens, 2,

@@ -19,19 +19,21 @@ CASES = [
     (2, 2, 32, 2, [40000, 777], 64),            # G = 16: 32 rows, two chunks; long: split segments
     (1, 5, 24, 8, [100000], None),              # G = 3, 15 rows; one long segment over every CTA
     (4, 3, 16, 4, [3, 130, 128, 1], 8),         # a request shorter than Q -> error row
+    (2, 2, 16, 2, [6000, 301], 16, 64),         # D = 64: 16 rows per KV head
 ]
 
 
-def _problem(B, Q, Hq, Hkv, lens, bs, seed):
-    p = make_problem("multi", B, Q * Hq, Hkv, 128, lens, seed=seed, block_size=bs,
+def _problem(B, Q, Hq, Hkv, lens, bs, seed, D=128):
+    p = make_problem("multi", B, Q * Hq, Hkv, D, lens, seed=seed, block_size=bs,
                      key_outlier_frac=0.01)
-    return p, p.q.reshape(B, Q, Hq, 128).contiguous()
+    return p, p.q.reshape(B, Q, Hq, D).contiguous()
 
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}_Q{c[1]}_Hq{c[2]}_Hkv{c[3]}_bs{c[5]}")
 def test_multi_matches_oracle(case):
-    B, Q, Hq, Hkv, lens, bs = case
-    p, q = _problem(B, Q, Hq, Hkv, lens, bs, 1200 + sum(lens) + Q)
+    B, Q, Hq, Hkv, lens, bs, *rest = case
+    D = rest[0] if rest else 128
+    p, q = _problem(B, Q, Hq, Hkv, lens, bs, 1200 + sum(lens) + Q, D)
     d = p.to("cuda")
     qd = q.cuda()
     ws = gq.Workspace(qd.device)
@@ -50,7 +52,7 @@ def test_multi_matches_oracle(case):
         for b in short:
             assert torch.isnan(o[b]).all()
         keep = [b for b in range(B) if lens[b] >= Q]
-        sub = make_problem("multi", B, Q * Hq, Hkv, 128, lens, seed=1200 + sum(lens) + Q,
+        sub = make_problem("multi", B, Q * Hq, Hkv, D, lens, seed=1200 + sum(lens) + Q,
                            block_size=bs, key_outlier_frac=0.01)
         lens_ok = sub.seq_lens.clone()
         for b in short:

@@ -73,6 +73,10 @@ SMALL = [
     (1, 4, 1, 128, [100000], None),
     (1, 16, 1, 128, [200000], 64),
     (1, 2, 1, 64, [150000], 16),
+    # tensor-core path at D = 64
+    (2, 32, 4, 64, [3001, 77], 32),                     # G = 8
+    (2, 16, 2, 64, [1000, 999], None),                  # contiguous
+    (1, 8, 1, 64, [120000], 64),                        # one long segment over every CTA
 ]
 
 

@@ -36,8 +36,10 @@ def test_bench_kernel_mapping():
         "gqa_decode_tc_kernel")
     assert bench.kernel_for(workloads.make_problem("b", 1, 32, 32, 128, [10], seed=1)) == \
         "gqa_decode_simt_kernel"                     # G = 1
-    assert bench.kernel_for(workloads.make_problem("c", 1, 32, 8, 64, [10], seed=1)) == \
-        "gqa_decode_simt_kernel"                     # D = 64
+    assert bench.kernel_for(workloads.make_problem("c", 1, 32, 8, 64, [10], seed=1)).startswith(
+        "gqa_decode_tc_kernel")                      # D = 64
+    assert bench.kernel_for(workloads.make_problem("c", 1, 32, 8, 256, [10], seed=1)) == \
+        "gqa_decode_simt_kernel"                     # D = 256
     assert bench.kernel_for(workloads.make_problem("d", 1, 32, 8, 128, [10], seed=1,
                                                    block_size=48)) == "gqa_decode_simt_kernel"
     p = workloads.make_problem("e", 1, 32, 8, 128, [10], seed=1)

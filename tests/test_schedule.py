@@ -28,7 +28,7 @@ def test_selector_estimates_scale_with_work():
 
 
 def test_selector_fixed_split_not_applicable_off_the_tensor_core_shapes():
-    n, (sk, fs) = gq.select_schedule([4096] * 4, 32, 8, 64, 148)   # D = 64
+    n, (sk, fs) = gq.select_schedule([4096] * 4, 32, 8, 256, 148)  # D = 256
     assert n == 0 and fs == -1.0 and sk > 0
     n, (_, fs) = gq.select_schedule([4096] * 4, 32, 32, 128, 148)  # G = 1
     assert n == 0 and fs == -1.0
