@@ -34,6 +34,15 @@ def test_selector_fixed_split_not_applicable_off_the_tensor_core_shapes():
     assert n == 0 and fs == -1.0
 
 
+def test_selector_covers_head_dim_64_on_the_tensor_cores():
+    # D = 64 runs on the tensor-core kernel, so the fixed split is a candidate too,
+    # and a tile costs half the bytes of D = 128.
+    n, (sk, fs) = gq.select_schedule([8192] * 16, 32, 8, 64, 148)
+    assert n == 1 and 0 < fs < sk
+    _, (sk128, _) = gq.select_schedule([8192] * 16, 32, 8, 128, 148)
+    assert 0.4 < sk / sk128 < 0.6
+
+
 def test_selector_empty_and_bad_arguments():
     n, (sk, _) = gq.select_schedule([], 32, 8, 128, 148)
     assert n == 0 and sk >= 0
