@@ -276,6 +276,24 @@ def run_reference(args, rank: int):
     print(json.dumps(line), flush=True)
 
 
+def step_timeline(gq, d, p, out, ws, stream, flush, splits, schedule):
+    """One more step, untimed and after an L2 flush, through gqa_decode_timeline with
+    the schedule the timed steps ran: per-CTA start/end (%globaltimer) and SM, summed
+    up as span, busy fraction and tail idle."""
+    ns = splits if splits else (1 if schedule.startswith("auto: one CTA") else 0)
+    flush.fill_(0)
+    _, tl = gq.gqa_decode_timeline(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,
+                                   num_splits=ns, out=out, scale=p.scale, workspace=ws,
+                                   stream=stream)
+    torch.cuda.synchronize()
+    if ws.status():
+        raise SystemExit("device status error during the timeline step")
+    summary = gq.timeline_summary(tl)
+    summary["source"] = ("one untimed step through gqa_decode_timeline, same schedule: "
+                         "per-CTA %globaltimer at entry and exit, %smid")
+    return summary
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -410,6 +428,8 @@ def main():
             "timed_region_ms": region_ms,
             "clocks": clocks,
         }
+    if rank == 0 and not fp8:
+        line["timeline"] = step_timeline(gq, d, p, out, ws, stream, flush, splits, schedule)
     if splits:  # comparator runs report the kernel numbers only
         args.no_e2e = args.no_cpu_baseline = True
     if rank == 0 and not args.no_e2e:

@@ -34,7 +34,7 @@ EXPORTED = ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states", "gqa
             "gqa_status", "gqa_decode_host_buffer_bytes", "gqa_decode_host", "gqa_error_string",
             "gqa_decode_noalloc", "gqa_decode_fixed_split_workspace_size",
             "gqa_decode_fixed_split", "gqa_select_schedule", "gqa_decode_auto",
-            "gqa_decode_multi", "gqa_decode_fp8")
+            "gqa_decode_multi", "gqa_decode_fp8", "gqa_decode_timeline")
 GQA_ERR_SCRATCH_LIMIT = 6
 
 _lib = None
@@ -70,6 +70,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_decode_auto.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, SZ, P]
     lib.gqa_decode_multi.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, P, SZ, P]
     lib.gqa_decode_fp8.argtypes = [P, P, P, F, F, P, P, P, I, I, I, I, I, F, I, I, P, SZ, P]
+    lib.gqa_decode_timeline.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, I,
+                                        ctypes.POINTER(I), P, SZ, P]
     lib.gqa_error_string.argtypes = [I]
     lib.gqa_error_string.restype = ctypes.c_char_p
     for name in ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states",
@@ -225,6 +227,73 @@ def gqa_decode_fixed_split(q, k_cache, v_cache, block_table, seq_lens, num_split
                                         _stream_ptr(stream))
     _check("gqa_decode_fixed_split", rc)
     return out
+
+
+def gqa_decode_timeline(q, k_cache, v_cache, block_table, seq_lens, num_splits: int = 0,
+                        out=None, scale=None, workspace: Optional[Workspace] = None,
+                        stream=None):
+    """gqa_decode (num_splits = 0, stream-K) or the fixed split (num_splits >= 1) that
+    also records the decode kernel's per-CTA timeline (see include/gqa_decode.h).
+    Returns (out, timeline): timeline is int64 [grid, 4] on the device, rows
+    (start ns, end ns, SM id, tiles)."""
+    lib = load_library()
+    B, Hq, Hkv, D, bs, mb, nb = _shape(q, k_cache, block_table)
+    dev = q.device
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _require(t, n, torch.bfloat16, dev)
+    _require(seq_lens, "seq_lens", torch.int32, dev)
+    if block_table is not None:
+        _require(block_table, "block_table", torch.int32, dev)
+    if out is None:
+        out = torch.empty_like(q)
+    _require(out, "out", torch.bfloat16, dev)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    ws = default_workspace(dev) if workspace is None else workspace
+    need = (fixed_split_workspace_size(B, Hq, Hkv, D, num_splits, dev.index) if num_splits > 0
+            else workspace_size(B, Hq, Hkv, D, dev.index))
+    buf = ws.get(need)
+    grid = ctypes.c_int(0)
+    # A buffer too small for the grid is refused before launch, with the grid reported.
+    tl = torch.zeros((1, 4), dtype=torch.int64, device=dev)
+    with torch.cuda.device(dev):
+        for _ in range(2):
+            rc = lib.gqa_decode_timeline(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                         _ptr(seq_lens), _ptr(out), B, Hq, Hkv, D, bs, scale, mb,
+                                         nb, int(num_splits), _ptr(tl), tl.shape[0],
+                                         ctypes.byref(grid), _ptr(buf), buf.numel(),
+                                         _stream_ptr(stream))
+            if rc == GQA_ERR_WORKSPACE_TOO_SMALL and grid.value > tl.shape[0]:
+                tl = torch.zeros((grid.value, 4), dtype=torch.int64, device=dev)
+                continue
+            break
+    _check("gqa_decode_timeline", rc)
+    return out, tl[:grid.value]
+
+
+def timeline_summary(timeline) -> dict:
+    """Tail-wave figures of one step's timeline (rows start ns, end ns, SM id, tiles):
+    span = last CTA end - first CTA start; busy = sum of CTA durations over
+    (CTAs x span); tail idle = 1 - busy; start and end times of the CTAs relative to
+    the first start (ends over the CTAs that had tiles)."""
+    import numpy as np
+    t = np.asarray(timeline.cpu() if hasattr(timeline, "cpu") else timeline, dtype=np.int64)
+    if t.ndim != 2 or t.shape[1] != 4 or t.shape[0] == 0:
+        raise ValueError("timeline must be a non-empty [rows, 4] array")
+    start, end, sm, tiles = t[:, 0], t[:, 1], t[:, 2], t[:, 3]
+    if np.any(end < start):
+        raise ValueError("a CTA ends before it starts")
+    t0 = start.min()
+    span = float(end.max() - t0)
+    busy = float((end - start).sum()) / (len(t) * span) if span > 0 else 1.0
+    work = tiles > 0
+    ends = (end[work] if work.any() else end) - t0
+    return {
+        "ctas": int(len(t)), "ctas_with_work": int(work.sum()), "sms": int(len(np.unique(sm))),
+        "tiles": int(tiles.sum()), "span_us": span / 1e3, "busy_frac": busy,
+        "tail_idle": 1.0 - busy, "start_us_max": float(start.max() - t0) / 1e3,
+        "end_us_min": float(ends.min()) / 1e3, "end_us_median": float(np.median(ends)) / 1e3,
+        "end_us_max": float(ends.max()) / 1e3,
+    }
 
 
 def gqa_decode_auto(q, k_cache, v_cache, block_table, seq_lens, seq_lens_host=None, out=None,

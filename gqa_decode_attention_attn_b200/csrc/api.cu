@@ -322,11 +322,15 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
                const int32_t *kv_end, void *out, float *acc, float *m, float *l, int B, int Hq,
                int Hkv, int D, int block_size, float scale, int max_blocks, int num_blocks,
                void *workspace, size_t workspace_bytes, void *stream, int nsplit = 0,
-               int qlen = 1, bool fp8 = false, float k_scale = 1.0f, float v_scale = 1.0f)
+               int qlen = 1, bool fp8 = false, float k_scale = 1.0f, float v_scale = 1.0f,
+               unsigned long long *timeline = nullptr, int timeline_rows = 0,
+               int *grid_out = nullptr)
 {
     int rc = check_shape(B, Hq, Hkv, D, block_size, block_table, max_blocks, num_blocks, scale);
     if (rc)
         return rc;
+    if (grid_out)
+        *grid_out = 0;
     if (B == 0)
         return GQA_OK;
     // An empty pool (num_blocks == 0) is never read: its caches may be null.
@@ -367,6 +371,12 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
                                             : layout_for(ctas, use_tc ? TcCfg::SLOT_FLOATS : v.slot_floats);
     if (workspace_bytes < w.total)
         return GQA_ERR_WORKSPACE_TOO_SMALL;
+    // The decode kernel's grid: one timeline row per CTA.
+    const int64_t grid = nsplit > 0 ? items : ctas;
+    if (grid_out)
+        *grid_out = (int)grid;
+    if (timeline && timeline_rows < grid)
+        return GQA_ERR_WORKSPACE_TOO_SMALL;
 
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     Params p{};
@@ -399,7 +409,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     p.capacity = block_table ? (int64_t)max_blocks * block_size : (int64_t)block_size;
     p.qscale = scale * LOG2E * (fp8 ? k_scale : 1.0f);
     p.vscale = fp8 ? v_scale : 1.0f;
-    p.timeline = nullptr;
+    p.timeline = timeline;
     // Magic number for t / block_size (t < 2^31): see page_of().
     {
         int l = 0;
@@ -604,6 +614,22 @@ int gqa_decode_fixed_split_workspace_size(int B, int Hq, int Hkv, int D, int num
         return GQA_ERR_INVALID_ARG;
     *bytes = layout_for(num_splits > 1 ? (int)((items + 1) / 2) : 0, TcCfg::SLOT_FLOATS).total;
     return GQA_OK;
+}
+
+int gqa_decode_timeline(const void *q, const void *k_cache, const void *v_cache,
+                        const int32_t *block_table, const int32_t *seq_lens, void *out, int B,
+                        int Hq, int Hkv, int D, int block_size, float scale,
+                        int max_blocks_per_seq, int num_blocks, int num_splits,
+                        unsigned long long *timeline, int timeline_rows, int *grid,
+                        void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!timeline || timeline_rows < 0 || num_splits < 0 ||
+        reinterpret_cast<uintptr_t>(timeline) % alignof(unsigned long long) != 0)
+        return GQA_ERR_INVALID_ARG;
+    return run_decode(false, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, out,
+                      nullptr, nullptr, nullptr, B, Hq, Hkv, D, block_size, scale,
+                      max_blocks_per_seq, num_blocks, workspace, workspace_bytes, stream,
+                      num_splits, 1, false, 1.0f, 1.0f, timeline, timeline_rows, grid);
 }
 
 int gqa_decode_fixed_split(const void *q, const void *k_cache, const void *v_cache,

@@ -134,6 +134,33 @@ GQA_API int gqa_decode_fixed_split(const void *q, const void *k_cache, const voi
                                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Per-CTA timeline of one decode step, for measuring how evenly the work units
+ * spread over the SMs and how long the last CTA trails (the tail wave the
+ * LeanAttention decode tiles digest sets out to remove, sections "Hardware-sized
+ * work units" and "Evaluation figures and their scope").  Computes exactly what
+ * gqa_decode (num_splits = 0, the stream-K schedule) or gqa_decode_fixed_split
+ * (num_splits >= 1) computes, with the same arguments, workspace and errors, and
+ * in addition writes one row per CTA of the decode kernel's grid:
+ *   timeline  DEVICE buffer, unsigned 64-bit [timeline_rows][4], 8-byte aligned,
+ *             borrowed.  Row c = { start ns, end ns, SM id, tiles }: the GPU's
+ *             global nanosecond timer when CTA c began and when it finished
+ *             (after any merge it took part in), the SM it ran on, and the
+ *             number of tiles (work units) in its run: 128 tokens each on the
+ *             tensor-core kernel, the kernel's own tile size on the CUDA cores.
+ *   grid      HOST int or NULL; receives the number of rows written (0 for B = 0).
+ * timeline_rows below the grid returns GQA_ERR_WORKSPACE_TOO_SMALL without
+ * launching (grid is still set), so a caller may size the buffer from a first
+ * call.  A NULL or misaligned timeline, or num_splits < 0, is GQA_ERR_INVALID_ARG.
+ * The second kernel of the fixed split records no rows.
+ */
+GQA_API int gqa_decode_timeline(const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *block_table, const int32_t *seq_lens, void *out,
+                                int B, int Hq, int Hkv, int D, int block_size, float scale,
+                                int max_blocks_per_seq, int num_blocks, int num_splits,
+                                unsigned long long *timeline, int timeline_rows, int *grid,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Runtime schedule selection on the host (LeanAttention decode tiles digest,
  * section "Runtime selection policy": the choice depends on the batch's context
  * length distribution, the heads per device, the head dimension and the SM

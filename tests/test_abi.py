@@ -66,3 +66,20 @@ def test_host_argument_checks(lib):
     assert lib.gqa_merge_states(None, None, None, 1, 0, 8, None, None, None) == 0   # N = 0
     assert lib.gqa_merge_states(None, None, None, 1, 4, 8, None, None, None) == 1
     assert lib.gqa_decode_host_buffer_bytes(2, 4, 1, 128, 64, 0, 0, 0) > 2 * 4 * 128 * 2
+
+
+def test_timeline_argument_checks(lib):
+    P, I = ctypes.c_void_p, ctypes.c_int
+    grid = I(-5)
+
+    def rc(timeline=16, rows=8, splits=0, B=1):
+        return lib.gqa_decode_timeline(P(16), P(16), P(16), None, P(16), P(16), B, 4, 1, 128, 16,
+                                       0.1, 0, 0, splits, None if timeline is None else P(timeline),
+                                       rows, ctypes.byref(grid), P(16), 1 << 20, None)
+
+    assert rc(timeline=None) == 1       # no timeline buffer
+    assert rc(timeline=20) == 1         # not 8-byte aligned
+    assert rc(splits=-1) == 1
+    assert rc(rows=-1) == 1
+    assert rc(B=-1) == 1                # the shape checks of gqa_decode
+    assert rc(B=0) == 0 and grid.value == 0   # empty batch: nothing launched, no rows

@@ -3,6 +3,7 @@ mapping and traffic-record keying, workspace sizes."""
 import os
 import sys
 
+import pytest
 import torch
 
 import gqa_decode_attention_attn_b200 as gq
@@ -53,3 +54,22 @@ def test_bench_kernel_mapping():
 def test_fixed_split_workspace_grows_with_splits():
     sizes = [gq.fixed_split_workspace_size(16, 32, 8, 128, s, 0) for s in (1, 2, 8, 32)]
     assert sizes == sorted(sizes) and sizes[0] < sizes[-1]
+
+
+def test_timeline_summary():
+    import numpy as np
+    # Three CTAs over a 10 us span: busy 10 + 8 + 2 = 20 of 30 us; the idle one has no tiles.
+    tl = np.array([[1000, 11000, 0, 5],
+                   [2000, 10000, 1, 4],
+                   [1000, 3000, 2, 0]])
+    s = gq.timeline_summary(tl)
+    assert s["ctas"] == 3 and s["ctas_with_work"] == 2 and s["sms"] == 3 and s["tiles"] == 9
+    assert abs(s["span_us"] - 10.0) < 1e-12
+    assert abs(s["busy_frac"] - 20.0 / 30.0) < 1e-12
+    assert abs(s["tail_idle"] - 10.0 / 30.0) < 1e-12
+    assert s["start_us_max"] == 1.0
+    assert s["end_us_min"] == 9.0 and s["end_us_max"] == 10.0   # CTAs with tiles only
+    with pytest.raises(ValueError):
+        gq.timeline_summary(np.array([[5, 4, 0, 1]]))             # ends before it starts
+    with pytest.raises(ValueError):
+        gq.timeline_summary(np.zeros((0, 4)))
