@@ -44,6 +44,9 @@ def test_stream_k_timeline_on_the_tensor_cores():
     t = _rows_ok(tl, 2 * sum(math.ceil(L / 128) for L in lens))
     # The cooperative grid holds one CTA per SM, each on its own SM, all with work.
     assert len(set(t[:, 2].tolist())) == t.shape[0]
+    # Stream-K partition of the W tiles over the P CTAs: CTA c runs [cW/P, (c+1)W/P).
+    W, P = 2 * sum(math.ceil(L / 128) for L in lens), t.shape[0]
+    assert t[:, 3].tolist() == [(c + 1) * W // P - c * W // P for c in range(P)]
     s = gq.timeline_summary(tl)
     assert s["ctas_with_work"] == t.shape[0] and 0.0 <= s["tail_idle"] < 1.0
 
@@ -62,6 +65,10 @@ def test_fixed_split_timeline():
     assert torch.equal(out, ref)
     t = _rows_ok(tl, 8 * sum(math.ceil(L / 128) for L in lens))
     assert t.shape[0] == 4 * 8 * 3  # one CTA per (request, KV head, chunk)
+    # Chunk i of a segment of nb tiles holds tiles [i nb / 3, (i + 1) nb / 3).
+    nb = [math.ceil(L / 128) for L in lens]
+    assert t[:, 3].tolist() == [(i + 1) * nb[b] // 3 - i * nb[b] // 3
+                                for b in range(4) for _ in range(8) for i in range(3)]
 
 
 def test_cuda_core_timeline():
