@@ -29,6 +29,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 import workloads  # noqa: E402
@@ -204,29 +205,45 @@ def _sample_bytes(p, b0: int, b1: int) -> int:
     return 2 * eb * p.Hkv * p.D * L + 4 * (b1 - b0) * p.Hq * p.D
 
 
-def cpu_oracle_sample(p, target_s: float):
+def cpu_oracle_sample(p, target_s: float, gpu_out=None):
     """Time the fp64 oracle as it stands on a bounded sample of the workload: groups
-    of whole requests, in order, until about target_s seconds have passed."""
+    of whole requests, in order, until about target_s seconds have passed.  With
+    gpu_out (the timed steps' output), the oracle rows it computed are also compared
+    with it: max-abs and rel-RMS error over the sampled requests."""
     import oracle
     threads = oracle.host_threads()
     oracle.default()
     chunk = _oracle_chunk(p, threads)
+    got = None if gpu_out is None else gpu_out.float().cpu().double().numpy().reshape(-1, p.D)
+    max_abs, sq_err, sq_ref, rows_cmp = 0.0, 0.0, 0.0, 0
     done_bytes, reqs, b = 0, 0, 0
     t0 = time.perf_counter()
     while True:
         b1 = min(p.B, b + chunk)
-        oracle.gqa_decode(p.q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, p.scale,
-                          rows=(b * p.Hq, b1 * p.Hq), threads=threads)
+        ref = oracle.gqa_decode(p.q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, p.scale,
+                                rows=(b * p.Hq, b1 * p.Hq), threads=threads)
+        if got is not None and reqs < p.B:  # each request compared once
+            d = got[b * p.Hq:b1 * p.Hq] - ref
+            max_abs = max(max_abs, float(np.abs(d).max()) if d.size else 0.0)
+            sq_err += float((d * d).sum())
+            sq_ref += float((ref * ref).sum())
+            rows_cmp += (b1 - b) * p.Hq
         done_bytes += _sample_bytes(p, b, b1)
         reqs += b1 - b
         b = 0 if b1 == p.B else b1
         if time.perf_counter() - t0 >= target_s:
             break
     dt = time.perf_counter() - t0
-    return {"value": done_bytes / dt / 1e9, "unit": "GB/s",
-            "cores": min(threads, chunk * p.Hq), "kind": "oracle",
-            "sample": f"{reqs} whole requests (all {p.Hq} heads each) of {p.name}, "
-                      f"{done_bytes / 1e6:.1f} MB of K+V+Q+O in {dt:.1f} s"}
+    res = {"value": done_bytes / dt / 1e9, "unit": "GB/s",
+           "cores": min(threads, chunk * p.Hq), "kind": "oracle",
+           "sample": f"{reqs} whole requests (all {p.Hq} heads each) of {p.name}, "
+                     f"{done_bytes / 1e6:.1f} MB of K+V+Q+O in {dt:.1f} s"}
+    if got is not None:
+        res["parity_of_sample"] = {
+            "rows": rows_cmp, "max_abs": max_abs,
+            "rel_rms": (sq_err / sq_ref) ** 0.5 if sq_ref > 0 else 0.0,
+            "bar": "max-abs <= 1e-2, rel-RMS <= 2e-3 (gpu bf16 output vs fp64 oracle)"}
+    return res
 
 
 def run_reference(args, rank: int):
@@ -435,7 +452,7 @@ def main():
     if rank == 0 and not args.no_e2e:
         line["e2e"] = measure_e2e(gq, p, dev, args, stream)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_oracle_sample(p, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_oracle_sample(p, args.cpu_seconds, gpu_out=out)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg:

@@ -73,3 +73,19 @@ def test_timeline_summary():
         gq.timeline_summary(np.array([[5, 4, 0, 1]]))             # ends before it starts
     with pytest.raises(ValueError):
         gq.timeline_summary(np.zeros((0, 4)))
+
+
+def test_cpu_baseline_reports_parity_of_its_sample():
+    import bench
+    import oracle
+    p = make_problem("cb", 3, 8, 2, 128, [300, 5, 900], seed=5, block_size=16)
+    ref = oracle.gqa_decode(p.q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, p.scale)
+    exact = torch.from_numpy(ref).to(torch.bfloat16)    # the correctly rounded result
+    r = bench.cpu_oracle_sample(p, 0.2, gpu_out=exact)
+    par = r["parity_of_sample"]
+    assert par["rows"] == 3 * 8                         # every request compared once
+    assert par["max_abs"] <= 1e-2 and par["rel_rms"] <= 2e-3
+    wrong = exact.clone()
+    wrong[1, 3, 7] += 1.0                               # one wrong element is seen
+    assert bench.cpu_oracle_sample(p, 0.2, gpu_out=wrong)["parity_of_sample"]["max_abs"] > 0.9
+    assert "parity_of_sample" not in bench.cpu_oracle_sample(p, 0.05)
