@@ -202,10 +202,15 @@ MergeFn tc_merge_for(int G, int D = 128)
     return D == 64 ? tc_merge_nv<64>(G) : tc_merge_nv<128>(G);
 }
 
+size_t tc_smem_bytes(int D, int B)
+{
+    return D == 64 ? TcGeom<64>::smem_bytes(B) : TcGeom<128>::smem_bytes(B);
+}
+
 int tc_ctas(int G, int dev, int &ctas, bool mq = false, int D = 128)
 {
     return persistent_ctas_fn(reinterpret_cast<const void *>(tc_kernel_for(G, mq, D)), TcCfg::THREADS,
-                              TcCfg::smem_bytes(TcCfg::MAX_BATCH), dev, ctas);
+                              tc_smem_bytes(D, TcCfg::MAX_BATCH), dev, ctas);
 }
 
 // Head dimensions the tensor-core kernel is built for.
@@ -429,7 +434,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         if (nsplit > 0) {
             // Fixed split: as many CTAs as chunks, in waves; no CTA waits for another.
             const cudaStream_t st = static_cast<cudaStream_t>(stream);
-            tc_kernel_for(R, qlen > 1, D)<<<(unsigned)items, TcCfg::THREADS, TcCfg::smem_bytes(B), st>>>(
+            tc_kernel_for(R, qlen > 1, D)<<<(unsigned)items, TcCfg::THREADS, tc_smem_bytes(D, B), st>>>(
                 p, tmk, tmv, box_rows);
             if (B > 0 && nsplit > 1) {
                 const int nv = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
@@ -444,7 +449,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)ctas);
         cfg.blockDim = dim3(TcCfg::THREADS);
-        cfg.dynamicSmemBytes = TcCfg::smem_bytes(B);
+        cfg.dynamicSmemBytes = tc_smem_bytes(D, B);
         cfg.stream = static_cast<cudaStream_t>(stream);
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeCooperative;

@@ -42,12 +42,9 @@ namespace gqa {
 
 struct TcCfg {
     // (merge scratch lives in the P buffers: checked below)
-    static constexpr int D = 128, T = 128, NP = 16;  // head dim, tile tokens, heads per MMA
-    static constexpr int STAGES = 3;                   // slots per ring (K ring, V ring)
+    static constexpr int T = 128, NP = 16;             // tile tokens, heads per MMA
     static constexpr int THREADS = 256;
     static constexpr int BOX_BYTES = T * 128;          // one 64-column half of a tile: 16 KB
-    static constexpr int TILE_BYTES = 2 * BOX_BYTES;   // K or V tile
-    static constexpr int V_RING_OFF = STAGES * TILE_BYTES;
     static constexpr int QBUF_BYTES = 2 * NP * 128;    // two halves, NP rows of 128 B
     static constexpr int NO = 2 * NP;                  // BMM2 columns: P_hi heads, P_lo heads
     static constexpr int P_LBO = (NO / 8) * 128;       // P: stride between 8-token groups
@@ -55,26 +52,45 @@ struct TcCfg {
     static constexpr int S_COL = 0, O_COL = 2 * NP;    // TMEM columns: S x2, O x2 (NO wide)
     static constexpr int TMEM_COLS = 128;              // >= 2 * NP + 2 * NO, power of two
     static constexpr float LAZY = 8.f;                 // rescale only when max grows > 2^8
-    static constexpr size_t Q_OFF = (size_t)2 * STAGES * TILE_BYTES;
-    static constexpr size_t P_OFF = Q_OFF + 2 * QBUF_BYTES;
-    static constexpr size_t BAR_OFF = P_OFF + 2 * PBUF_BYTES;
+    static constexpr int SLOT_FLOATS = slot_floats(NP, 128);  // the larger head dimension
+    static constexpr int MAX_BATCH = 1024;
+};
+static_assert(TcCfg::O_COL + 2 * TcCfg::NO <= TcCfg::TMEM_COLS, "tensor memory columns");
+
+// Shared-memory layout for head dimension D.  A ring slot holds one K or V tile:
+// both 64-column halves at D = 128 (32 KB, three slots per ring), the one half at
+// D = 64 (16 KB, five slots per ring, so that as many bytes stay in flight).  At
+// D = 64 BMM2 still runs M = 128 over V^T; its rows 64..127 come from one 16 KB
+// block of zeros shared by every V slot (the operand's leading-byte offset points
+// there).
+template <int D>
+struct TcGeom {
+    static constexpr int HALVES = D / 64;
+    static constexpr int STAGES = D == 64 ? 5 : 3;    // slots per ring (K ring, V ring)
+    static constexpr int SLOT_BYTES = HALVES * TcCfg::BOX_BYTES;
+    static constexpr size_t V_RING_OFF = (size_t)STAGES * SLOT_BYTES;
+    static constexpr size_t ZERO_OFF = 2 * V_RING_OFF;                 // D = 64 only
+    static constexpr size_t Q_OFF = ZERO_OFF + (D == 64 ? TcCfg::BOX_BYTES : 0);
+    static constexpr size_t P_OFF = Q_OFF + 2 * TcCfg::QBUF_BYTES;
+    static constexpr size_t BAR_OFF = P_OFF + 2 * TcCfg::PBUF_BYTES;
     static constexpr int NBAR = 4 * STAGES + 16;
     static constexpr size_t MISC_OFF = BAR_OFF + NBAR * 8;
     // floats: tile maxima [2][4][NP], piece sums [4][NP], merge maxima [NP]
     static constexpr size_t RED_OFF = MISC_OFF + 64 * 4;
-    static constexpr size_t PREFIX_OFF = RED_OFF + 13 * NP * 4 + 64;
-    static constexpr int SLOT_FLOATS = slot_floats(NP, D);
-    static constexpr int MAX_BATCH = 1024;
+    static constexpr size_t PREFIX_OFF = RED_OFF + 13 * TcCfg::NP * 4 + 64;
     // +1024: the dynamic shared-memory base is re-aligned to 1024 bytes in-kernel.
     static size_t smem_bytes(int B) { return PREFIX_OFF + (size_t)(B + 1) * sizeof(int) + 1024; }
+    // Segment merge: the owner list (<= 512 ints) in the P buffers; the gathered
+    // slices, at most E + 4 no + 3 no (E / D + 2) + 2 NP floats (E <= NP x D
+    // outputs, no <= 512 owners, slices rounded to 4 elements), in the rings.
+    static_assert(512 * 4 <= 2 * TcCfg::PBUF_BYTES, "owner list must fit in the P buffers");
+    static_assert((16 * D + 4 * 512 + 3 * 512 * (16 + 2) + 32) * 4 <= 2 * V_RING_OFF,
+                  "gathered slices must fit in the rings");
+    static_assert(STAGES <= 8, "stage_n and stage_bad hold 8 slots");
+    static_assert(Q_OFF % 1024 == 0 && ZERO_OFF % 1024 == 0, "swizzled buffers are 1024-byte aligned");
+    static_assert(PREFIX_OFF + (TcCfg::MAX_BATCH + 1) * sizeof(int) + 1024 <= 227 * 1024,
+                  "shared memory per CTA");
 };
-// Segment merge: the owner list (<= 512 ints) in the P buffers; the gathered
-// slices, at most E + 4 no + 3 no (E / D + 2) + 2 NP floats (E <= NP x D outputs,
-// no <= 512 owners, slices rounded to 4 elements), in the rings.
-static_assert(512 * 4 <= 2 * TcCfg::PBUF_BYTES, "owner list must fit in the P buffers");
-static_assert((16 * 128 + 4 * 512 + 3 * 512 * (16 + 2) + 32) * 4 <= 2 * TcCfg::STAGES * TcCfg::TILE_BYTES,
-              "gathered slices must fit in the rings");
-static_assert(TcCfg::O_COL + 2 * TcCfg::NO <= TcCfg::TMEM_COLS, "tensor memory columns");
 
 // Max or sum of NV per-lane values across the 32 lanes of a warp, transposed so
 // that lane l ends with the result for index l / (32 / NV) (NV <= 32).
@@ -109,16 +125,17 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[NV], int lane)
 // decode instantiation carries no mask code.
 // DH: head dimension, 128 or 64.  At 64, BMM1 takes 4 K-steps over the one
 // 64-column half that is loaded, and BMM2 still runs M = 128 over V^T with rows
-// 64..127 held at zero in shared memory (written once, never loaded), so the
-// O rows 64..127 are zero and are not read back.
+// 64..127 read from a block of zeros (written once, never loaded), so the O rows
+// 64..127 are zero and are not read back.
 template <int NV, bool MQ, int DH = 128>
 __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     gqa_decode_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv, int box_rows)
 {
     using C = TcCfg;
-    constexpr int S = C::STAGES, NP = C::NP, D = DH, T = C::T;
-    constexpr int HALVES = D / 64;  // 64-column halves loaded per tile
+    using L = TcGeom<DH>;
+    constexpr int S = L::STAGES, NP = C::NP, D = DH, T = C::T;
+    constexpr int HALVES = L::HALVES;  // 64-column halves loaded per tile
     static_assert(D == 64 || D == 128, "head dimension");
     constexpr int SLOT = slot_floats(NV, D);
     constexpr int LPH = 32 / NV;  // lanes per head after a transposed warp reduction
@@ -126,21 +143,21 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     unsigned char *ring = smem;
-    unsigned char *qbuf = smem + C::Q_OFF;
-    unsigned char *pbuf = smem + C::P_OFF;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    unsigned char *qbuf = smem + L::Q_OFF;
+    unsigned char *pbuf = smem + L::P_OFF;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
     uint64_t *k_full = bars, *k_empty = bars + S, *v_full = bars + 2 * S, *v_empty = bars + 3 * S;
     uint64_t *s_full = bars + 4 * S, *s_free = s_full + 2, *p_full = s_free + 2;
     uint64_t *o_full = p_full + 2, *o_free = o_full + 2, *q_full = o_free + 2, *p_free = q_full + 2;
     uint64_t *drain = p_free + 2;  // two: one per MMA-issuing thread
-    int *misc = reinterpret_cast<int *>(smem + C::MISC_OFF);
+    int *misc = reinterpret_cast<int *>(smem + L::MISC_OFF);
     int *stage_n = misc, *stage_bad = misc + 8;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 16);
     volatile int *abort_flag = misc + 17;
     int *last_flag = misc + 18, *poison_flag = misc + 19;
     volatile int *ctl = misc + 28;  // per P buffer: the softmax moved its reference max
-    float *red = reinterpret_cast<float *>(smem + C::RED_OFF);
-    int *prefix = reinterpret_cast<int *>(smem + C::PREFIX_OFF);
+    float *red = reinterpret_cast<float *>(smem + L::RED_OFF);
+    int *prefix = reinterpret_cast<int *>(smem + L::PREFIX_OFF);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = p.B;
@@ -175,13 +192,10 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         tmem_relinquish();
     }
     if constexpr (HALVES == 1) {
-        // V^T rows 64..127 (the upper half of every V slot) stay zero for the whole
-        // launch; the TMA loads only the lower half.  Likewise Q's upper half.
-        for (int x = tid; x < S * C::BOX_BYTES / 16; x += C::THREADS) {
-            const int slot = x / (C::BOX_BYTES / 16), off = x % (C::BOX_BYTES / 16);
-            reinterpret_cast<uint4 *>(ring + C::V_RING_OFF + (size_t)slot * C::TILE_BYTES + C::BOX_BYTES)[off] =
-                make_uint4(0, 0, 0, 0);
-        }
+        // The block BMM2 reads as V^T rows 64..127 stays zero for the whole launch.
+        // Likewise Q's upper half.
+        for (int x = tid; x < C::BOX_BYTES / 16; x += C::THREADS)
+            reinterpret_cast<uint4 *>(ring + L::ZERO_OFF)[x] = make_uint4(0, 0, 0, 0);
         for (int x = tid; x < 2 * C::QBUF_BYTES / 16; x += C::THREADS)
             reinterpret_cast<uint4 *>(qbuf)[x] = make_uint4(0, 0, 0, 0);
         fence_proxy_async_smem();
@@ -250,7 +264,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         // ---------------------------------------------------------------- TMA
         const bool is_k = warp == 0;
         const CUtensorMap *map = is_k ? &tmk : &tmv;
-        unsigned char *base = ring + (is_k ? 0 : C::V_RING_OFF);
+        unsigned char *base = ring + (is_k ? 0 : L::V_RING_OFF);
         uint64_t *full = is_k ? k_full : v_full, *emptyb = is_k ? k_empty : v_empty;
         // K/V are read once, except when several 16-head chunks of a KV head (G > 16)
         // stream the same tiles at about the same time: then L2 keeps them for the
@@ -310,7 +324,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             }
             __syncwarp();
             if (lane < nbox && !bad) {
-                unsigned char *d = base + (size_t)s * C::TILE_BYTES + (size_t)lane * box_rows * 128;
+                unsigned char *d = base + (size_t)s * L::SLOT_BYTES + (size_t)lane * box_rows * 128;
                 tma_load_2d(d, map, 0, row, &full[s], pol);
                 if constexpr (HALVES == 2)
                     tma_load_2d(d + C::BOX_BYTES, map, 64, row, &full[s], pol);
@@ -354,7 +368,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                     if (!ok)
                         break;
                     tc_fence_after_sync();
-                    const uint32_t ka = ring_a + (uint32_t)(s * C::TILE_BYTES);
+                    const uint32_t ka = ring_a + (uint32_t)(s * L::SLOT_BYTES);
                     const uint32_t qa = q_a + (uint32_t)(qb * C::QBUF_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
@@ -403,12 +417,15 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                         segp = itp.seg0;
                     }
                     tc_fence_after_sync();
-                    const uint32_t va = ring_a + (uint32_t)(C::V_RING_OFF + s * C::TILE_BYTES);
+                    const uint32_t va_off = (uint32_t)(L::V_RING_OFF + s * L::SLOT_BYTES);
+                    const uint32_t va = ring_a + va_off;
+                    // V^T rows 64..127: the slot's upper half, or the zero block at D = 64.
+                    const uint32_t vlbo = HALVES == 2 ? (uint32_t)C::BOX_BYTES : (uint32_t)L::ZERO_OFF - va_off;
                     const uint32_t pa = p_a + (uint32_t)(b * C::PBUF_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < T / 16; ++kk) {
                         umma_bf16(tbase + (uint32_t)(C::O_COL + (u & 1) * C::NO),
-                                  umma_smem_desc(va + (uint32_t)(kk * 2048), C::BOX_BYTES, 1024, SMEM_LAYOUT_SW128),
+                                  umma_smem_desc(va + (uint32_t)(kk * 2048), vlbo, 1024, SMEM_LAYOUT_SW128),
                                   umma_smem_desc(pa + (uint32_t)(2 * kk * C::P_LBO), C::P_LBO, 128, SMEM_LAYOUT_NONE),
                                   idesc2, kk > 0 || !fresh);
                     }
@@ -708,7 +725,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             // Rows past the valid tokens may hold anything (stale tiles, poison):
             // zero this token's V row so that 0-weight rows add exact zeros.
             if (!valid) {
-                unsigned char *vr = ring + C::V_RING_OFF + (size_t)s * C::TILE_BYTES + ti * 128;
+                unsigned char *vr = ring + L::V_RING_OFF + (size_t)s * L::SLOT_BYTES + ti * 128;
 #pragma unroll
                 for (int h = 0; h < HALVES; ++h)
 #pragma unroll
