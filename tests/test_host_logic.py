@@ -45,7 +45,10 @@ def test_bench_kernel_mapping():
                                                    block_size=48)) == "gqa_decode_simt_kernel"
     p = workloads.make_problem("e", 1, 32, 8, 128, [10], seed=1)
     p.meta["kv_elem_bytes"] = 1
-    assert "FP8" in bench.kernel_for(p)
+    assert bench.kernel_for(p) == "gqa_decode_tc_kernel<4> (FP8 E4M3 cache)"
+    p = workloads.make_problem("f", 1, 32, 8, 64, [10], seed=1)
+    p.meta["kv_elem_bytes"] = 1
+    assert bench.kernel_for(p) == "gqa_decode_simt_kernel (FP8 E4M3 cache)"   # D = 64
     # traffic records are keyed to each kernel's own sources
     assert bench.kernel_source_hash("gqa_decode_tc_kernel<4>") != \
         bench.kernel_source_hash("gqa_decode_simt_kernel")
