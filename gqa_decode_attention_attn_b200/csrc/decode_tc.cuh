@@ -146,6 +146,12 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     const int B = p.B;
     const uint64_t t_start = global_timer_ns();
 
+    // The tensor maps are fetched while the barriers, TMEM and the tile prefix sums
+    // are set up.
+    if (tid == 32 * 2)
+        tma_prefetch_map(&tmk);
+    else if (tid == 32 * 3)
+        tma_prefetch_map(&tmv);
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&k_full[s], 1);
