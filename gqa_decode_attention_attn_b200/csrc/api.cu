@@ -390,7 +390,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
                                             : layout_for(ctas, use_tc ? TcCfg::SLOT_FLOATS : v.slot_floats);
     if (workspace_bytes < w.total)
         return GQA_ERR_WORKSPACE_TOO_SMALL;
-    // The decode kernel's grid: one timeline row per CTA.
+    // The decode kernel's grid: one timeline row (TL_COLS values) per CTA.
     const int64_t grid = nsplit > 0 ? items : ctas;
     if (grid_out)
         *grid_out = (int)grid;

@@ -199,6 +199,12 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     const int B = p.B;
     const uint64_t t_start = global_timer_ns();
 
+    // The tensor maps are fetched while the barriers, TMEM and the tile prefix sums
+    // are set up.
+    if (tid == 32 * 2)
+        tma_prefetch_map(&tmk);
+    else if (tid == 32 * 3)
+        tma_prefetch_map(&tmv);
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&k_full[s], 1);
@@ -357,6 +363,8 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 }
                 const uint32_t boxes = (uint32_t)(nbox - __popc(badmask));
                 mbar_arrive_expect_tx(&full[s], boxes * (uint32_t)HALVES * (uint32_t)box_rows * 128u);
+                if (p.timeline && is_k && k == 0)
+                    p.timeline[TL_COLS * c + 4] = global_timer_ns();
             }
             __syncwarp();
             if (lane < nbox && !bad) {
@@ -684,6 +692,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
 
         int len_b = -1;
         int64_t req_len = 0;
+        uint64_t t_scores = 0;
         int k = 0;
         for (int64_t i = start; i < end; ++i, ++k) {
             if (i > start)
@@ -753,6 +762,8 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                     tmem_load<NV>(tlane + (uint32_t)(C::S_COL + b * SW), sc);
                 }
                 tc_fence_before_sync();
+                if (k == 0 && stid == 0 && p.timeline)
+                    t_scores = global_timer_ns();
             } else {
                 ok = false;
                 poisoned = true;
@@ -907,6 +918,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         }
         flush_fold();
         epilogue(end);
+        const uint64_t t_streamed = p.timeline ? global_timer_ns() : 0;
         // Split segments: publish every partial piece of this run, then merge this
         // CTA's share of each (all owners are resident: cooperative launch).  Every
         // tile has been consumed, so the P buffers and the rings are scratch.
@@ -921,6 +933,12 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                                              reinterpret_cast<float *>(ring), misc + 20, stid, 1,
                                              abort_flag);
         }
+        if (p.timeline && stid == 0) {
+            unsigned long long *rec = p.timeline + TL_COLS * c;
+            rec[5] = t_scores;
+            rec[6] = t_streamed;
+            rec[7] = global_timer_ns();
+        }
     }
 
     // Timeline record and tensor-memory release.
@@ -933,11 +951,14 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     if (p.timeline && tid == 0) {
         unsigned sm;
         asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
-        unsigned long long *rec = p.timeline + 4 * c;
+        unsigned long long *rec = p.timeline + TL_COLS * c;
         rec[0] = t_start;
         rec[1] = global_timer_ns();
         rec[2] = sm;
         rec[3] = (unsigned long long)(end - start);
+        if (start >= end)
+            for (int x = 4; x < TL_COLS; ++x)
+                rec[x] = 0;
     }
 }
 

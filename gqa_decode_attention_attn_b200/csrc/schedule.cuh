@@ -29,6 +29,11 @@ constexpr unsigned DEV_TIMEOUT = 4u;
 // Upper bound on any single in-kernel wait; a healthy wait lasts microseconds.
 constexpr uint64_t WAIT_LIMIT_NS = 1500000000ull;
 
+// Per-CTA timeline row (Params::timeline): start ns, end ns, SM id, tiles, then the
+// phases of a tensor-core CTA with work (0 elsewhere): first TMA issue, first
+// scores ready, end of streaming (last piece closed), end of merging.
+constexpr int TL_COLS = 8;
+
 struct Params {
     const uint16_t *q;            // [B, Hq, D] bf16
     const uint16_t *k;            // [num_blocks, Hkv, block_size, D] bf16
@@ -55,7 +60,7 @@ struct Params {
     int bs_shift;
     float qscale;                 // scale * log2(e) (* k_scale for FP8): scores in log2 units
     float vscale;                 // FP8 cache: v_scale, applied to the output (1 for bf16)
-    unsigned long long *timeline; // optional [grid][4]: start ns, end ns, SM id, tiles
+    unsigned long long *timeline; // optional [grid][TL_COLS], see TL_COLS
 };
 
 // floor(t / block_size) for 0 <= t < 2^31 without a divide: with l = ceil(log2 bs)

@@ -173,4 +173,11 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
                  : "memory");
 }
 
+// Fetch a tensor map (a kernel parameter) into the TMA unit's descriptor cache
+// ahead of its first use, so the first tile's load does not wait for it.
+__device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *map)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
 }  // namespace gqa
