@@ -50,12 +50,16 @@ KERNEL_SOURCES = {
 
 def kernel_for(p) -> str:
     """Which decode kernel the library runs for this problem (mirrors the library's
-    dispatch: tensor cores for D = 64 or 128 with at least 4 query heads per KV head and
-    pages that tile into 128-token boxes, CUDA cores otherwise and for FP8 caches)."""
-    if p.meta.get("kv_elem_bytes") == 1:
-        return "gqa_decode_simt_kernel (FP8 E4M3 cache)"
+    dispatch: tensor cores for D = 64 or 128 (FP8 caches: D = 128) with at least 4
+    query heads per KV head and pages that tile into 128-token boxes, CUDA cores
+    otherwise)."""
     bs = p.block_size
     boxes = (not p.paged) or (bs % 128 == 0 if bs >= 128 else (bs >= 8 and 128 % bs == 0))
+    if p.meta.get("kv_elem_bytes") == 1:
+        if p.D == 128 and p.G >= 4 and p.B <= 1024 and boxes:
+            nv = 4 if p.G <= 4 else (8 if p.G <= 8 else 16)
+            return f"gqa_decode_tc_kernel<{nv}> (FP8 E4M3 cache)"
+        return "gqa_decode_simt_kernel (FP8 E4M3 cache)"
     if p.D in (64, 128) and p.G >= 4 and p.B <= 1024 and boxes:
         nv = 4 if p.G <= 4 else (8 if p.G <= 8 else 16)
         return f"gqa_decode_tc_kernel<{nv}>"

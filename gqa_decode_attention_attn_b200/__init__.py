@@ -36,6 +36,7 @@ EXPORTED = ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states", "gqa
             "gqa_decode_fixed_split", "gqa_select_schedule", "gqa_decode_auto",
             "gqa_decode_multi", "gqa_decode_fp8", "gqa_decode_timeline")
 GQA_ERR_SCRATCH_LIMIT = 6
+TIMELINE_COLS = 8  # values per CTA row of gqa_decode_timeline
 
 _lib = None
 
@@ -234,8 +235,9 @@ def gqa_decode_timeline(q, k_cache, v_cache, block_table, seq_lens, num_splits: 
                         stream=None):
     """gqa_decode (num_splits = 0, stream-K) or the fixed split (num_splits >= 1) that
     also records the decode kernel's per-CTA timeline (see include/gqa_decode.h).
-    Returns (out, timeline): timeline is int64 [grid, 4] on the device, rows
-    (start ns, end ns, SM id, tiles)."""
+    Returns (out, timeline): timeline is int64 [grid, 8] on the device, rows
+    (start ns, end ns, SM id, tiles, first TMA ns, first scores ns, streamed ns,
+    merged ns); the last four are 0 where not recorded."""
     lib = load_library()
     B, Hq, Hkv, D, bs, mb, nb = _shape(q, k_cache, block_table)
     dev = q.device
@@ -254,7 +256,7 @@ def gqa_decode_timeline(q, k_cache, v_cache, block_table, seq_lens, num_splits: 
     buf = ws.get(need)
     grid = ctypes.c_int(0)
     # A buffer too small for the grid is refused before launch, with the grid reported.
-    tl = torch.zeros((1, 4), dtype=torch.int64, device=dev)
+    tl = torch.zeros((1, TIMELINE_COLS), dtype=torch.int64, device=dev)
     with torch.cuda.device(dev):
         for _ in range(2):
             rc = lib.gqa_decode_timeline(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
@@ -263,7 +265,7 @@ def gqa_decode_timeline(q, k_cache, v_cache, block_table, seq_lens, num_splits: 
                                          ctypes.byref(grid), _ptr(buf), buf.numel(),
                                          _stream_ptr(stream))
             if rc == GQA_ERR_WORKSPACE_TOO_SMALL and grid.value > tl.shape[0]:
-                tl = torch.zeros((grid.value, 4), dtype=torch.int64, device=dev)
+                tl = torch.zeros((grid.value, TIMELINE_COLS), dtype=torch.int64, device=dev)
                 continue
             break
     _check("gqa_decode_timeline", rc)
@@ -271,14 +273,15 @@ def gqa_decode_timeline(q, k_cache, v_cache, block_table, seq_lens, num_splits: 
 
 
 def timeline_summary(timeline) -> dict:
-    """Tail-wave figures of one step's timeline (rows start ns, end ns, SM id, tiles):
+    """Tail-wave figures of one step's timeline (rows as gqa_decode_timeline returns):
     span = last CTA end - first CTA start; busy = sum of CTA durations over
     (CTAs x span); tail idle = 1 - busy; start and end times of the CTAs relative to
-    the first start (ends over the CTAs that had tiles)."""
+    the first start (ends over the CTAs that had tiles); and, where the phases were
+    recorded, their median and maximum times after each CTA's own start."""
     import numpy as np
     t = np.asarray(timeline.cpu() if hasattr(timeline, "cpu") else timeline, dtype=np.int64)
-    if t.ndim != 2 or t.shape[1] != 4 or t.shape[0] == 0:
-        raise ValueError("timeline must be a non-empty [rows, 4] array")
+    if t.ndim != 2 or t.shape[1] != TIMELINE_COLS or t.shape[0] == 0:
+        raise ValueError(f"timeline must be a non-empty [rows, {TIMELINE_COLS}] array")
     start, end, sm, tiles = t[:, 0], t[:, 1], t[:, 2], t[:, 3]
     if np.any(end < start):
         raise ValueError("a CTA ends before it starts")
@@ -293,7 +296,19 @@ def timeline_summary(timeline) -> dict:
         "tail_idle": 1.0 - busy, "start_us_max": float(start.max() - t0) / 1e3,
         "end_us_min": float(ends.min()) / 1e3, "end_us_median": float(np.median(ends)) / 1e3,
         "end_us_max": float(ends.max()) / 1e3,
+        "phases_us": _phases(t),
     }
+
+
+def _phases(t) -> dict:
+    import numpy as np
+    out = {}
+    for col, name in ((4, "first_tma"), (5, "first_scores"), (6, "streamed"), (7, "merged")):
+        rec = t[:, col] > 0
+        if rec.any():
+            d = (t[rec, col] - t[rec, 0]) / 1e3
+            out[name] = {"median": float(np.median(d)), "max": float(d.max())}
+    return out
 
 
 def gqa_decode_auto(q, k_cache, v_cache, block_table, seq_lens, seq_lens_host=None, out=None,

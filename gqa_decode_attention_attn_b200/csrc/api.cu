@@ -179,8 +179,15 @@ TcKernelFn tc_kernel_nv(int G)
     return gqa_decode_tc_kernel<16, MQ, DH>;
 }
 
-TcKernelFn tc_kernel_for(int G, bool mq = false, int D = 128)
+TcKernelFn tc_kernel_for(int G, bool mq = false, int D = 128, bool fp8 = false)
 {
+    if (fp8) {  // FP8 E4M3 cache: D = 128, one query token
+        if (G <= 4)
+            return gqa_decode_tc_kernel<4, false, 128, true>;
+        if (G <= 8)
+            return gqa_decode_tc_kernel<8, false, 128, true>;
+        return gqa_decode_tc_kernel<16, false, 128, true>;
+    }
     if (D == 64)
         return mq ? tc_kernel_nv<true, 64>(G) : tc_kernel_nv<false, 64>(G);
     return mq ? tc_kernel_nv<true, 128>(G) : tc_kernel_nv<false, 128>(G);
@@ -202,10 +209,17 @@ MergeFn tc_merge_for(int G, int D = 128)
     return D == 64 ? tc_merge_nv<64>(G) : tc_merge_nv<128>(G);
 }
 
-int tc_ctas(int G, int dev, int &ctas, bool mq = false, int D = 128)
+size_t tc_smem_bytes(int D, int B, bool fp8 = false)
 {
-    return persistent_ctas_fn(reinterpret_cast<const void *>(tc_kernel_for(G, mq, D)), TcCfg::THREADS,
-                              TcCfg::smem_bytes(TcCfg::MAX_BATCH), dev, ctas);
+    if (fp8)
+        return TcGeom<128, true>::smem_bytes(B);
+    return D == 64 ? TcGeom<64>::smem_bytes(B) : TcGeom<128>::smem_bytes(B);
+}
+
+int tc_ctas(int G, int dev, int &ctas, bool mq = false, int D = 128, bool fp8 = false)
+{
+    return persistent_ctas_fn(reinterpret_cast<const void *>(tc_kernel_for(G, mq, D, fp8)),
+                              TcCfg::THREADS, tc_smem_bytes(D, TcCfg::MAX_BATCH, fp8), dev, ctas);
 }
 
 // Head dimensions the tensor-core kernel is built for.
@@ -259,18 +273,22 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// 2-D view of a cache as [rows, D] bf16; boxes of 64 columns x box_rows rows,
-// 128-byte swizzle (the layout the tensor cores read), zero fill out of range.
-bool encode_kv_map(CUtensorMap *map, const void *base, int64_t rows, int box_rows, int D)
+// 2-D view of a cache as [rows, D] bf16 (or FP8 bytes); boxes of 128 bytes (64
+// bf16 or 128 FP8 columns) x box_rows rows, 128-byte swizzle (the layout the
+// tensor cores read), zero fill out of range.
+bool encode_kv_map(CUtensorMap *map, const void *base, int64_t rows, int box_rows, int D,
+                   bool fp8 = false)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn)
         return false;
+    const int eb = fp8 ? 1 : 2;
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * eb};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 / eb), (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+    return fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+              const_cast<void *>(base), dims, strides,
               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -345,9 +363,10 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     if (qlen < 1 || qlen > GQA_MAX_QLEN)
         return GQA_ERR_INVALID_ARG;
     const int R = qlen * G;  // query rows per KV head
-    // FP8 caches run on the CUDA-core kernel.
-    const bool use_tc =
-        !fp8 && tc_applicable(states, B, Hq, Hkv, D, block_size, block_table, num_blocks, R);
+    // FP8 caches run on the tensor cores at D = 128 (one query token), else on the
+    // CUDA-core kernel.
+    const bool use_tc = (!fp8 || (D == 128 && qlen == 1)) &&
+                        tc_applicable(states, B, Hq, Hkv, D, block_size, block_table, num_blocks, R);
     Variant v;
     if (!use_tc && !pick_variant(D, G, states, v, fp8))
         return GQA_ERR_UNSUPPORTED;
@@ -357,7 +376,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     if ((rc = current_device(dev)))
         return rc;
     int ctas = 0;
-    if ((rc = use_tc ? tc_ctas(R, dev, ctas, qlen > 1, D) : persistent_ctas(v, dev, ctas)))
+    if ((rc = use_tc ? tc_ctas(R, dev, ctas, qlen > 1, D, fp8) : persistent_ctas(v, dev, ctas)))
         return rc;
     if (nsplit > 0 && !use_tc)
         return GQA_ERR_UNSUPPORTED;
@@ -371,7 +390,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
                                             : layout_for(ctas, use_tc ? TcCfg::SLOT_FLOATS : v.slot_floats);
     if (workspace_bytes < w.total)
         return GQA_ERR_WORKSPACE_TOO_SMALL;
-    // The decode kernel's grid: one timeline row per CTA.
+    // The decode kernel's grid: one timeline row (TL_COLS values) per CTA.
     const int64_t grid = nsplit > 0 ? items : ctas;
     if (grid_out)
         *grid_out = (int)grid;
@@ -424,12 +443,13 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         const int box_rows = tc_box_rows(block_table, block_size);
         const int64_t rows = (block_table ? (int64_t)num_blocks : (int64_t)B) * Hkv * block_size;
         CUtensorMap tmk, tmv;
-        if (!encode_kv_map(&tmk, k_cache, rows, box_rows, D) || !encode_kv_map(&tmv, v_cache, rows, box_rows, D))
+        if (!encode_kv_map(&tmk, k_cache, rows, box_rows, D, fp8) ||
+            !encode_kv_map(&tmv, v_cache, rows, box_rows, D, fp8))
             return GQA_ERR_CUDA;
         if (nsplit > 0) {
             // Fixed split: as many CTAs as chunks, in waves; no CTA waits for another.
             const cudaStream_t st = static_cast<cudaStream_t>(stream);
-            tc_kernel_for(R, qlen > 1, D)<<<(unsigned)items, TcCfg::THREADS, TcCfg::smem_bytes(B), st>>>(
+            tc_kernel_for(R, qlen > 1, D, fp8)<<<(unsigned)items, TcCfg::THREADS, tc_smem_bytes(D, B, fp8), st>>>(
                 p, tmk, tmv, box_rows);
             if (B > 0 && nsplit > 1) {
                 const int nv = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
@@ -444,14 +464,14 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)ctas);
         cfg.blockDim = dim3(TcCfg::THREADS);
-        cfg.dynamicSmemBytes = TcCfg::smem_bytes(B);
+        cfg.dynamicSmemBytes = tc_smem_bytes(D, B, fp8);
         cfg.stream = static_cast<cudaStream_t>(stream);
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeCooperative;
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, tc_kernel_for(R, qlen > 1, D), p, tmk, tmv, box_rows) != cudaSuccess)
+        if (cudaLaunchKernelEx(&cfg, tc_kernel_for(R, qlen > 1, D, fp8), p, tmk, tmv, box_rows) != cudaSuccess)
             return GQA_ERR_CUDA;
     } else {
         v.fn<<<ctas, v.threads, v.smem(B), static_cast<cudaStream_t>(stream)>>>(p);

@@ -222,11 +222,13 @@ __global__ void __launch_bounds__(SimtCfg<D, GC, F8>::THREADS, 1)
         if (p.timeline && tid == 0) {
             unsigned sm;
             asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
-            unsigned long long *rec = p.timeline + 4 * c;
+            unsigned long long *rec = p.timeline + TL_COLS * c;
             rec[0] = t_start;
             rec[1] = global_timer_ns();
             rec[2] = sm;
             rec[3] = 0;
+            for (int x = 4; x < TL_COLS; ++x)
+                rec[x] = 0;
         }
         return;
     }
@@ -613,11 +615,13 @@ __global__ void __launch_bounds__(SimtCfg<D, GC, F8>::THREADS, 1)
     if (p.timeline && ctid == 0) {
         unsigned sm;
         asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
-        unsigned long long *rec = p.timeline + 4 * c;
+        unsigned long long *rec = p.timeline + TL_COLS * c;
         rec[0] = t_start;
         rec[1] = global_timer_ns();
         rec[2] = sm;
         rec[3] = (unsigned long long)(end - start);
+        for (int x = 4; x < TL_COLS; ++x)
+            rec[x] = 0;
     }
 }
 

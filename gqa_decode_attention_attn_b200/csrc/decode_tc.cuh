@@ -34,6 +34,8 @@
 // softmax that merges piece by piece" and "Hardware-sized work units".)
 #pragma once
 
+#include <cuda_fp8.h>
+
 #include "gather_merge.cuh"
 #include "schedule.cuh"
 #include "tc.cuh"
@@ -42,12 +44,9 @@ namespace gqa {
 
 struct TcCfg {
     // (merge scratch lives in the P buffers: checked below)
-    static constexpr int D = 128, T = 128, NP = 16;  // head dim, tile tokens, heads per MMA
-    static constexpr int STAGES = 3;                   // slots per ring (K ring, V ring)
+    static constexpr int T = 128, NP = 16;             // tile tokens, heads per MMA
     static constexpr int THREADS = 256;
     static constexpr int BOX_BYTES = T * 128;          // one 64-column half of a tile: 16 KB
-    static constexpr int TILE_BYTES = 2 * BOX_BYTES;   // K or V tile
-    static constexpr int V_RING_OFF = STAGES * TILE_BYTES;
     static constexpr int QBUF_BYTES = 2 * NP * 128;    // two halves, NP rows of 128 B
     static constexpr int NO = 2 * NP;                  // BMM2 columns: P_hi heads, P_lo heads
     static constexpr int P_LBO = (NO / 8) * 128;       // P: stride between 8-token groups
@@ -55,26 +54,67 @@ struct TcCfg {
     static constexpr int S_COL = 0, O_COL = 2 * NP;    // TMEM columns: S x2, O x2 (NO wide)
     static constexpr int TMEM_COLS = 128;              // >= 2 * NP + 2 * NO, power of two
     static constexpr float LAZY = 8.f;                 // rescale only when max grows > 2^8
-    static constexpr size_t Q_OFF = (size_t)2 * STAGES * TILE_BYTES;
-    static constexpr size_t P_OFF = Q_OFF + 2 * QBUF_BYTES;
-    static constexpr size_t BAR_OFF = P_OFF + 2 * PBUF_BYTES;
+    static constexpr int SLOT_FLOATS = slot_floats(NP, 128);  // the larger head dimension
+    static constexpr int MAX_BATCH = 1024;
+};
+static_assert(TcCfg::O_COL + 2 * TcCfg::NO <= TcCfg::TMEM_COLS, "tensor memory columns");
+
+// Shared-memory layout for head dimension D (F8: an FP8 E4M3 cache, D = 128).  A
+// ring slot holds one K or V tile of 128-byte boxes (one box row per token):
+// two boxes at bf16 D = 128 (32 KB, three slots per ring), one at bf16 D = 64 and
+// at FP8 D = 128 (16 KB, five slots per ring, so that as many bytes stay in
+// flight).  At bf16 D = 64 BMM2 still runs M = 128 over V^T; its rows 64..127
+// come from one 16 KB block of zeros shared by every V slot (the operand's
+// leading-byte offset points there).  At 8 bits one box row spans all 128 rows
+// of V^T.
+template <int D, bool F8 = false>
+struct TcGeom {
+    static_assert(!F8 || D == 128, "FP8 tiles are built for D = 128");
+    static constexpr int BOXES = (F8 ? D : 2 * D) / 128;   // 128-byte boxes per token row
+    static constexpr bool NEED_ZERO = !F8 && D == 64;
+    static constexpr int STAGES = BOXES == 1 ? 5 : 3;      // slots per ring (K ring, V ring)
+    static constexpr int SLOT_BYTES = BOXES * TcCfg::BOX_BYTES;
+    static constexpr size_t V_RING_OFF = (size_t)STAGES * SLOT_BYTES;
+    static constexpr size_t ZERO_OFF = 2 * V_RING_OFF;                 // NEED_ZERO only
+    static constexpr size_t Q_OFF = ZERO_OFF + (NEED_ZERO ? TcCfg::BOX_BYTES : 0);
+    static constexpr size_t P_OFF = Q_OFF + 2 * TcCfg::QBUF_BYTES;
+    static constexpr size_t BAR_OFF = P_OFF + 2 * TcCfg::PBUF_BYTES;
     static constexpr int NBAR = 4 * STAGES + 16;
     static constexpr size_t MISC_OFF = BAR_OFF + NBAR * 8;
-    // floats: tile maxima [2][4][NP], piece sums [4][NP], merge maxima [NP]
+    // floats: tile maxima [2][4][NP], piece sums [4][NP], merge maxima [NP], then
+    // (FP8) the per-row scales of the piece's Q terms [NP]
     static constexpr size_t RED_OFF = MISC_OFF + 64 * 4;
-    static constexpr size_t PREFIX_OFF = RED_OFF + 13 * NP * 4 + 64;
-    static constexpr int SLOT_FLOATS = slot_floats(NP, D);
-    static constexpr int MAX_BATCH = 1024;
+    static constexpr size_t PREFIX_OFF = RED_OFF + 13 * TcCfg::NP * 4 + 64;
     // +1024: the dynamic shared-memory base is re-aligned to 1024 bytes in-kernel.
     static size_t smem_bytes(int B) { return PREFIX_OFF + (size_t)(B + 1) * sizeof(int) + 1024; }
+    // Segment merge: the owner list (<= 512 ints) in the P buffers; the gathered
+    // slices, at most E + 4 no + 3 no (E / D + 2) + 2 NP floats (E <= NP x D
+    // outputs, no <= 512 owners, slices rounded to 4 elements), in the rings.
+    static_assert(512 * 4 <= 2 * TcCfg::PBUF_BYTES, "owner list must fit in the P buffers");
+    static_assert((16 * D + 4 * 512 + 3 * 512 * (16 + 2) + 32) * 4 <= 2 * V_RING_OFF,
+                  "gathered slices must fit in the rings");
+    static_assert(STAGES <= 8, "stage_n and stage_bad hold 8 slots");
+    static_assert(Q_OFF % 1024 == 0 && ZERO_OFF % 1024 == 0, "swizzled buffers are 1024-byte aligned");
+    static_assert(PREFIX_OFF + (TcCfg::MAX_BATCH + 1) * sizeof(int) + 1024 <= 227 * 1024,
+                  "shared memory per CTA");
 };
-// Segment merge: the owner list (<= 512 ints) in the P buffers; the gathered
-// slices, at most E + 4 no + 3 no (E / D + 2) + 2 NP floats (E <= NP x D outputs,
-// no <= 512 owners, slices rounded to 4 elements), in the rings.
-static_assert(512 * 4 <= 2 * TcCfg::PBUF_BYTES, "owner list must fit in the P buffers");
-static_assert((16 * 128 + 4 * 512 + 3 * 512 * (16 + 2) + 32) * 4 <= 2 * TcCfg::STAGES * TcCfg::TILE_BYTES,
-              "gathered slices must fit in the rings");
-static_assert(TcCfg::O_COL + 2 * TcCfg::NO <= TcCfg::TMEM_COLS, "tensor memory columns");
+
+// One float to E4M3 (round to nearest even, saturating) and back, exactly.
+__device__ __forceinline__ uint32_t to_e4m3(float x)
+{
+    return (uint32_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+}
+__device__ __forceinline__ float e4m3_value(uint32_t b)
+{
+    const __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)b, __NV_E4M3);
+    return __half2float(__half(h));
+}
+// x as two E4M3 terms, x ~ hi + lo / 16 (lo carries the remainder scaled by 16).
+__device__ __forceinline__ void split_e4m3(float x, uint32_t &hi, uint32_t &lo)
+{
+    hi = to_e4m3(x);
+    lo = to_e4m3((x - e4m3_value(hi)) * 16.f);
+}
 
 // Max or sum of NV per-lane values across the 32 lanes of a warp, transposed so
 // that lane l ends with the result for index l / (32 / NV) (NV <= 32).
@@ -109,16 +149,29 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[NV], int lane)
 // decode instantiation carries no mask code.
 // DH: head dimension, 128 or 64.  At 64, BMM1 takes 4 K-steps over the one
 // 64-column half that is loaded, and BMM2 still runs M = 128 over V^T with rows
-// 64..127 held at zero in shared memory (written once, never loaded), so the
-// O rows 64..127 are zero and are not read back.
-template <int NV, bool MQ, int DH = 128>
+// 64..127 read from a block of zeros (written once, never loaded), so the O rows
+// 64..127 are zero and are not read back.
+// F8: the cache holds FP8 E4M3 (D = 128): the MMAs run kind::f8f6f4 (K = 32) on
+// the cache bytes as loaded; Q and P enter as two E4M3 terms each, t1 + t2 / 16,
+// side by side in N = 32 (one term per 16 columns), and the softmax and the fold
+// add the two column blocks back.  Scores are scaled by p.qscale (which holds the
+// K scale) and by the power of two that brought each Q row into E4M3's range.
+template <int NV, bool MQ, int DH = 128, bool F8 = false>
 __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     gqa_decode_tc_kernel(const Params p, const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv, int box_rows)
 {
     using C = TcCfg;
-    constexpr int S = C::STAGES, NP = C::NP, D = DH, T = C::T;
-    constexpr int HALVES = D / 64;  // 64-column halves loaded per tile
+    using L = TcGeom<DH, F8>;
+    constexpr int S = L::STAGES, NP = C::NP, D = DH, T = C::T;
+    constexpr int HALVES = L::BOXES;  // 128-byte boxes loaded per token row
+    constexpr int SW = F8 ? 2 * NP : NP;            // S columns per buffer
+    constexpr int OC = F8 ? 4 * NP : C::O_COL;      // first O column
+    constexpr int KSTEP = F8 ? 32 : 16;             // MMA K per instruction
+    // FP8 P: per 8-token group, two 128-byte core matrices along N (16 E4M3 heads
+    // per 16-byte row: term 1, then term 2).
+    constexpr int P8_LBO = (C::NO / 16) * 128;
+    static_assert(OC + 2 * C::NO <= C::TMEM_COLS, "tensor memory columns");
     static_assert(D == 64 || D == 128, "head dimension");
     constexpr int SLOT = slot_floats(NV, D);
     constexpr int LPH = 32 / NV;  // lanes per head after a transposed warp reduction
@@ -126,26 +179,32 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     unsigned char *ring = smem;
-    unsigned char *qbuf = smem + C::Q_OFF;
-    unsigned char *pbuf = smem + C::P_OFF;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    unsigned char *qbuf = smem + L::Q_OFF;
+    unsigned char *pbuf = smem + L::P_OFF;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
     uint64_t *k_full = bars, *k_empty = bars + S, *v_full = bars + 2 * S, *v_empty = bars + 3 * S;
     uint64_t *s_full = bars + 4 * S, *s_free = s_full + 2, *p_full = s_free + 2;
     uint64_t *o_full = p_full + 2, *o_free = o_full + 2, *q_full = o_free + 2, *p_free = q_full + 2;
     uint64_t *drain = p_free + 2;  // two: one per MMA-issuing thread
-    int *misc = reinterpret_cast<int *>(smem + C::MISC_OFF);
+    int *misc = reinterpret_cast<int *>(smem + L::MISC_OFF);
     int *stage_n = misc, *stage_bad = misc + 8;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 16);
     volatile int *abort_flag = misc + 17;
     int *last_flag = misc + 18, *poison_flag = misc + 19;
     volatile int *ctl = misc + 28;  // per P buffer: the softmax moved its reference max
-    float *red = reinterpret_cast<float *>(smem + C::RED_OFF);
-    int *prefix = reinterpret_cast<int *>(smem + C::PREFIX_OFF);
+    float *red = reinterpret_cast<float *>(smem + L::RED_OFF);
+    int *prefix = reinterpret_cast<int *>(smem + L::PREFIX_OFF);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = p.B;
     const uint64_t t_start = global_timer_ns();
 
+    // The tensor maps are fetched while the barriers, TMEM and the tile prefix sums
+    // are set up.
+    if (tid == 32 * 2)
+        tma_prefetch_map(&tmk);
+    else if (tid == 32 * 3)
+        tma_prefetch_map(&tmv);
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&k_full[s], 1);
@@ -174,14 +233,11 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
-    if constexpr (HALVES == 1) {
-        // V^T rows 64..127 (the upper half of every V slot) stay zero for the whole
-        // launch; the TMA loads only the lower half.  Likewise Q's upper half.
-        for (int x = tid; x < S * C::BOX_BYTES / 16; x += C::THREADS) {
-            const int slot = x / (C::BOX_BYTES / 16), off = x % (C::BOX_BYTES / 16);
-            reinterpret_cast<uint4 *>(ring + C::V_RING_OFF + (size_t)slot * C::TILE_BYTES + C::BOX_BYTES)[off] =
-                make_uint4(0, 0, 0, 0);
-        }
+    if constexpr (L::NEED_ZERO) {
+        // The block BMM2 reads as V^T rows 64..127 stays zero for the whole launch.
+        // Likewise Q's upper half.
+        for (int x = tid; x < C::BOX_BYTES / 16; x += C::THREADS)
+            reinterpret_cast<uint4 *>(ring + L::ZERO_OFF)[x] = make_uint4(0, 0, 0, 0);
         for (int x = tid; x < 2 * C::QBUF_BYTES / 16; x += C::THREADS)
             reinterpret_cast<uint4 *>(qbuf)[x] = make_uint4(0, 0, 0, 0);
         fence_proxy_async_smem();
@@ -228,10 +284,13 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         start = run_start(c, W, P);
         end = run_start(c + 1, W, P);
     } else {
+        // Segment j = (b, kvh, hc) in that order; its first tile in the global order
+        // (hc, b, kvh, tile).
         const int64_t j = c / p.nsplit, i = c - j * p.nsplit;
         const int b = (int)(j / units);
+        const int64_t u = j - (int64_t)b * units, kv = u / p.hch, hc = u - kv * p.hch;
         const int64_t nbj = prefix[b + 1] - prefix[b];
-        const int64_t seg0 = units * prefix[b] + (j - (int64_t)b * units) * nbj;
+        const int64_t seg0 = hc * p.Hkv * prefix[B] + (int64_t)p.Hkv * prefix[b] + kv * nbj;
         start = seg0 + i * nbj / p.nsplit;
         end = seg0 + (i + 1) * nbj / p.nsplit;
     }
@@ -250,7 +309,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         // ---------------------------------------------------------------- TMA
         const bool is_k = warp == 0;
         const CUtensorMap *map = is_k ? &tmk : &tmv;
-        unsigned char *base = ring + (is_k ? 0 : C::V_RING_OFF);
+        unsigned char *base = ring + (is_k ? 0 : L::V_RING_OFF);
         uint64_t *full = is_k ? k_full : v_full, *emptyb = is_k ? k_empty : v_empty;
         // K/V are read once, except when several 16-head chunks of a KV head (G > 16)
         // stream the same tiles at about the same time: then L2 keeps them for the
@@ -307,10 +366,12 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 }
                 const uint32_t boxes = (uint32_t)(nbox - __popc(badmask));
                 mbar_arrive_expect_tx(&full[s], boxes * (uint32_t)HALVES * (uint32_t)box_rows * 128u);
+                if (p.timeline && is_k && k == 0)
+                    p.timeline[TL_COLS * c + 4] = global_timer_ns();
             }
             __syncwarp();
             if (lane < nbox && !bad) {
-                unsigned char *d = base + (size_t)s * C::TILE_BYTES + (size_t)lane * box_rows * 128;
+                unsigned char *d = base + (size_t)s * L::SLOT_BYTES + (size_t)lane * box_rows * 128;
                 tma_load_2d(d, map, 0, row, &full[s], pol);
                 if constexpr (HALVES == 2)
                     tma_load_2d(d + C::BOX_BYTES, map, 64, row, &full[s], pol);
@@ -335,7 +396,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             const int ntiles = (int)(end - start);
             bool ok = true;
             if (warp == 1) {
-                const uint32_t idesc1 = umma_idesc_bf16(128, NP, 0, 0);
+                const uint32_t idesc1 = F8 ? umma_idesc_e4m3(128, SW, 0, 0) : umma_idesc_bf16(128, NP, 0, 0);
                 TileIter it1;
                 it1.init(start, prefix, B, units, p.hch);
                 int64_t seg1 = -1;
@@ -354,15 +415,19 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                     if (!ok)
                         break;
                     tc_fence_after_sync();
-                    const uint32_t ka = ring_a + (uint32_t)(s * C::TILE_BYTES);
+                    const uint32_t ka = ring_a + (uint32_t)(s * L::SLOT_BYTES);
                     const uint32_t qa = q_a + (uint32_t)(qb * C::QBUF_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
+                    for (int kk = 0; kk < D / KSTEP; ++kk) {
+                        // 32 bytes of every row per instruction: 16 bf16 or 32 E4M3 elements.
                         const uint32_t off = (uint32_t)((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32);
                         const uint32_t qoff = (uint32_t)((kk >> 2) * NP * 128 + (kk & 3) * 32);
-                        umma_bf16(tbase + (uint32_t)(C::S_COL + b * NP),
-                                  umma_smem_desc(ka + off, 16, 1024, SMEM_LAYOUT_SW128),
-                                  umma_smem_desc(qa + qoff, 16, 1024, SMEM_LAYOUT_SW128), idesc1, kk > 0);
+                        const uint64_t ad = umma_smem_desc(ka + off, 16, 1024, SMEM_LAYOUT_SW128);
+                        const uint64_t bd = umma_smem_desc(qa + qoff, 16, 1024, SMEM_LAYOUT_SW128);
+                        if constexpr (F8)
+                            umma_e4m3(tbase + (uint32_t)(C::S_COL + b * SW), ad, bd, idesc1, kk > 0);
+                        else
+                            umma_bf16(tbase + (uint32_t)(C::S_COL + b * SW), ad, bd, idesc1, kk > 0);
                     }
                     umma_commit(&s_full[b]);
                     umma_commit(&k_empty[s]);
@@ -373,7 +438,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 // o_full) when the softmax moves the reference (ctl flag of the tile)
                 // or when a piece ends; the next tile opens the other buffer afresh.
                 // Closes are counted by `u`: use u lives in buffer u & 1.
-                const uint32_t idesc2 = umma_idesc_bf16(128, C::NO, 1, 1);
+                const uint32_t idesc2 = F8 ? umma_idesc_e4m3(128, C::NO, 1, 1) : umma_idesc_bf16(128, C::NO, 1, 1);
                 TileIter itp;
                 itp.init(start, prefix, B, units, p.hch);
                 int64_t segp = itp.seg0;
@@ -403,14 +468,27 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                         segp = itp.seg0;
                     }
                     tc_fence_after_sync();
-                    const uint32_t va = ring_a + (uint32_t)(C::V_RING_OFF + s * C::TILE_BYTES);
+                    const uint32_t va_off = (uint32_t)(L::V_RING_OFF + s * L::SLOT_BYTES);
+                    const uint32_t va = ring_a + va_off;
+                    // V^T rows 64..127: the slot's upper half, or the zero block at D = 64.
+                    const uint32_t vlbo = HALVES == 2 ? (uint32_t)C::BOX_BYTES : (uint32_t)L::ZERO_OFF - va_off;
                     const uint32_t pa = p_a + (uint32_t)(b * C::PBUF_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < T / 16; ++kk) {
-                        umma_bf16(tbase + (uint32_t)(C::O_COL + (u & 1) * C::NO),
-                                  umma_smem_desc(va + (uint32_t)(kk * 2048), C::BOX_BYTES, 1024, SMEM_LAYOUT_SW128),
-                                  umma_smem_desc(pa + (uint32_t)(2 * kk * C::P_LBO), C::P_LBO, 128, SMEM_LAYOUT_NONE),
-                                  idesc2, kk > 0 || !fresh);
+                    for (int kk = 0; kk < T / KSTEP; ++kk) {
+                        if constexpr (F8) {
+                            // 32 tokens per instruction: 4 KB of V rows, four 8-token groups of P.
+                            umma_e4m3(tbase + (uint32_t)(OC + (u & 1) * C::NO),
+                                      umma_smem_desc(va + (uint32_t)(kk * 4096), C::BOX_BYTES, 1024,
+                                                     SMEM_LAYOUT_SW128),
+                                      umma_smem_desc(pa + (uint32_t)(4 * kk * P8_LBO), P8_LBO, 128,
+                                                     SMEM_LAYOUT_NONE),
+                                      idesc2, kk > 0 || !fresh);
+                        } else {
+                            umma_bf16(tbase + (uint32_t)(OC + (u & 1) * C::NO),
+                                      umma_smem_desc(va + (uint32_t)(kk * 2048), vlbo, 1024, SMEM_LAYOUT_SW128),
+                                      umma_smem_desc(pa + (uint32_t)(2 * kk * C::P_LBO), C::P_LBO, 128, SMEM_LAYOUT_NONE),
+                                      idesc2, kk > 0 || !fresh);
+                        }
                     }
                     fresh = false;
                     umma_commit(&v_empty[s]);
@@ -437,6 +515,66 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         const int stid = tid - 64;               // 0..127 among the softmax threads
         const uint32_t tlane = tbase + ((uint32_t)(q4 * 32) << 16);
         const float qscale = p.qscale;
+        // FP8: score scale per head of the current piece (qscale over its Q row's
+        // power-of-two range factor).
+        float qs[F8 ? NV : 1];
+#pragma unroll
+        for (int g = 0; g < (F8 ? NV : 1); ++g)
+            qs[g] = qscale;
+        auto qsc = [&](int g) -> float {
+            if constexpr (F8)
+                return qs[g];
+            else
+                return qscale;
+        };
+        // FP8: the piece's Q rows as two E4M3 terms in the 128-byte-swizzled K-major
+        // layout BMM1 reads, term 1 in rows 0..NP-1 and term 2 in rows NP..2NP-1.
+        // Each row is first scaled by the power of two that brings its largest
+        // magnitude into [2^7, 2^8); red[13 NP + g] receives the inverse.  Thread
+        // stid converts 8 elements of rows stid / 16 and stid / 16 + 8: the 16
+        // threads of a row are 16 consecutive lanes.
+        auto load_q_e4m3 = [&](unsigned char *qd, const TileIter &ti) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int x = stid + 128 * r;
+                const int g = x >> 4, c8 = x & 15;  // row, 8-element chunk of it
+                uint4 w = make_uint4(0, 0, 0, 0);
+                if (ti.hc * NP + g < p.R)
+                    w = __ldg(reinterpret_cast<const uint4 *>(
+                        p.q + (out_row(p, ti.b, ti.kvh, ti.hc * NP + g) * D + c8 * 8)));
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                float v[8];
+                float mx = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    v[2 * j] = __uint_as_float(ww[j] << 16);  // bf16 widening, exact
+                    v[2 * j + 1] = __uint_as_float(ww[j] & 0xffff0000u);
+                    mx = fmaxf(mx, fmaxf(fabsf(v[2 * j]), fabsf(v[2 * j + 1])));
+                }
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1)
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                int sh = 0;
+                if (mx > 0.f)
+                    sh = min(max(7 - (((__float_as_int(mx) >> 23) & 0xff) - 127), -100), 100);
+                const float up = __int_as_float((127 + sh) << 23), down = __int_as_float((127 - sh) << 23);
+                uint32_t t1[2] = {0u, 0u}, t2[2] = {0u, 0u};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint32_t hi, lo;
+                    split_e4m3(v[j] * up, hi, lo);
+                    t1[j >> 2] |= hi << (8 * (j & 3));
+                    t2[j >> 2] |= lo << (8 * (j & 3));
+                }
+                const int c16 = c8 >> 1, sub = (c8 & 1) * 8, g2 = g + NP;
+                *reinterpret_cast<uint2 *>(qd + g * 128 + (((c16 ^ (g & 7)) << 4) + sub)) =
+                    make_uint2(t1[0], t1[1]);
+                *reinterpret_cast<uint2 *>(qd + g2 * 128 + (((c16 ^ (g2 & 7)) << 4) + sub)) =
+                    make_uint2(t2[0], t2[1]);
+                if (c8 == 0)
+                    red[13 * NP + g] = down;
+            }
+        };
         // acc holds the closed O buffers, relative to the current reference m_ref
         // (the open TMEM buffer shares that reference).
         float m_ref[NV], l_t[NV], acc[NV];
@@ -457,12 +595,16 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             if (ok && bounded_wait(&o_full[bc], (uint32_t)((u >> 1) & 1), abort_flag, p.status)) {
                 float olo[NV];
                 tc_fence_after_sync();
-                tmem_load<NV>(tlane + (uint32_t)(C::O_COL + bc * C::NO), o);
-                tmem_load<NV>(tlane + (uint32_t)(C::O_COL + bc * C::NO + NP), olo);
+                tmem_load<NV>(tlane + (uint32_t)(OC + bc * C::NO), o);
+                tmem_load<NV>(tlane + (uint32_t)(OC + bc * C::NO + NP), olo);
                 tc_fence_before_sync();
 #pragma unroll
-                for (int g = 0; g < NV; ++g)
-                    o[g] += olo[g];
+                for (int g = 0; g < NV; ++g) {
+                    if constexpr (F8)
+                        o[g] = fmaf(olo[g], 1.f / 16.f, o[g]);  // the second P term carries x16
+                    else
+                        o[g] += olo[g];
+                }
             } else {
                 ok = false;
                 poisoned = true;
@@ -553,6 +695,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
 
         int len_b = -1;
         int64_t req_len = 0;
+        uint64_t t_scores = 0;
         int k = 0;
         for (int64_t i = start; i < end; ++i, ++k) {
             if (i > start)
@@ -566,6 +709,9 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 // 16-byte chunk cc of a 64-column half at chunk position cc ^ (g & 7)).
                 ++piece;
                 unsigned char *qd = qbuf + ((piece - 1) & 1) * C::QBUF_BYTES;
+                if constexpr (F8) {
+                    load_q_e4m3(qd, it);
+                } else {
 #pragma unroll
                 for (int r = 0; r < HALVES; ++r) {
                     const int x = stid + 128 * r;
@@ -576,8 +722,15 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                             p.q + (out_row(p, it.b, it.kvh, it.hc * NP + g) * D + half * 64 + cc * 8)));
                     *reinterpret_cast<uint4 *>(qd + half * NP * 128 + g * 128 + ((cc ^ (g & 7)) << 4)) = w;
                 }
+                }
                 fence_proxy_async_smem();
                 mbar_arrive(&q_full[(piece - 1) & 1]);
+                if constexpr (F8) {
+                    named_barrier_sync(1, 128);  // the rows' range factors are in red
+#pragma unroll
+                    for (int g = 0; g < NV; ++g)
+                        qs[g] = qscale * red[13 * NP + g];
+                }
                 if (i > start) {
                     flush_fold();
                     epilogue(i);
@@ -601,8 +754,19 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 n = stage_n[s];
                 poisoned |= stage_bad[s] != 0;
                 tc_fence_after_sync();
-                tmem_load<NV>(tlane + (uint32_t)(C::S_COL + b * NP), sc);
+                if constexpr (F8) {
+                    float s2[NV];
+                    tmem_load<NV>(tlane + (uint32_t)(C::S_COL + b * SW), sc);
+                    tmem_load<NV>(tlane + (uint32_t)(C::S_COL + b * SW + NP), s2);
+#pragma unroll
+                    for (int g = 0; g < NV; ++g)
+                        sc[g] = fmaf(s2[g], 1.f / 16.f, sc[g]);  // the second Q term carries x16
+                } else {
+                    tmem_load<NV>(tlane + (uint32_t)(C::S_COL + b * SW), sc);
+                }
                 tc_fence_before_sync();
+                if (k == 0 && stid == 0 && p.timeline)
+                    t_scores = global_timer_ns();
             } else {
                 ok = false;
                 poisoned = true;
@@ -638,7 +802,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             float xmax = -INFINITY;
 #pragma unroll
             for (int g = 0; g < NV; ++g) {
-                x[g] = see[g] ? fmaf(sc[g], qscale, -m_ref[g]) : -INFINITY;
+                x[g] = see[g] ? fmaf(sc[g], qsc(g), -m_ref[g]) : -INFINITY;
                 xmax = fmaxf(xmax, x[g]);
             }
             const bool moved = named_barrier_or(1, 128, !(xmax <= C::LAZY));
@@ -648,7 +812,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 float mx[NV];
 #pragma unroll
                 for (int g = 0; g < NV; ++g)
-                    mx[g] = see[g] ? sc[g] * qscale : -INFINITY;
+                    mx[g] = see[g] ? sc[g] * qsc(g) : -INFINITY;
                 const float wmax = warp_transpose_reduce<NV, true>(mx, lane);
                 float *tred = red + (k & 1) * 4 * NP;
                 if (lane % LPH == 0)
@@ -660,7 +824,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                     const float m_new = tm > m_ref[g] + C::LAZY ? tm : m_ref[g];
                     alpha[g] = m_new == m_ref[g] ? 1.f : fast_exp2(m_ref[g] - m_new);
                     m_ref[g] = m_new;
-                    x[g] = (see[g] && m_new != -INFINITY) ? fmaf(sc[g], qscale, -m_new) : -INFINITY;
+                    x[g] = (see[g] && m_new != -INFINITY) ? fmaf(sc[g], qsc(g), -m_new) : -INFINITY;
                     l_t[g] *= alpha[g];
                     acc[g] *= alpha[g];
                 }
@@ -679,8 +843,34 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             // P = hi + lo, both bf16, as one N = 32 operand (hi heads in columns
             // 0..NP-1, lo heads in NP..2NP-1) in the no-swizzle MN-major layout:
             // token ti's 8-head groups are 16-byte rows of 8x8 core matrices.
-            unsigned char *pd = pbuf + b * C::PBUF_BYTES + (ti >> 3) * C::P_LBO + (ti & 7) * 16;
-            {
+            if constexpr (F8) {
+                // P = t1 + t2 / 16, both E4M3, as one N = 32 operand (term 1 of the
+                // heads in bytes 0..NP-1 of the token's 16-byte row of the first core
+                // matrix, term 2 in the second), no-swizzle MN-major.
+                unsigned char *pd8 = pbuf + b * C::PBUF_BYTES + (ti >> 3) * P8_LBO + (ti & 7) * 16;
+                uint32_t w1[(NV + 3) / 4], w2[(NV + 3) / 4];
+#pragma unroll
+                for (int j = 0; j < (NV + 3) / 4; ++j)
+                    w1[j] = w2[j] = 0u;
+#pragma unroll
+                for (int g = 0; g < NV; ++g) {
+                    uint32_t hi, lo;
+                    split_e4m3(pr[g], hi, lo);
+                    w1[g >> 2] |= hi << (8 * (g & 3));
+                    w2[g >> 2] |= lo << (8 * (g & 3));
+                }
+                if constexpr (NV == 4) {
+                    *reinterpret_cast<uint32_t *>(pd8) = w1[0];
+                    *reinterpret_cast<uint32_t *>(pd8 + 128) = w2[0];
+                } else if constexpr (NV == 8) {
+                    *reinterpret_cast<uint2 *>(pd8) = make_uint2(w1[0], w1[1]);
+                    *reinterpret_cast<uint2 *>(pd8 + 128) = make_uint2(w2[0], w2[1]);
+                } else {
+                    *reinterpret_cast<uint4 *>(pd8) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+                    *reinterpret_cast<uint4 *>(pd8 + 128) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+                }
+            } else {
+                unsigned char *pd = pbuf + b * C::PBUF_BYTES + (ti >> 3) * C::P_LBO + (ti & 7) * 16;
                 constexpr int NW = NV / 2;  // bf16 pairs per term
                 uint32_t whi[NW], wlo[NW];
 #pragma unroll
@@ -708,7 +898,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             // Rows past the valid tokens may hold anything (stale tiles, poison):
             // zero this token's V row so that 0-weight rows add exact zeros.
             if (!valid) {
-                unsigned char *vr = ring + C::V_RING_OFF + (size_t)s * C::TILE_BYTES + ti * 128;
+                unsigned char *vr = ring + L::V_RING_OFF + (size_t)s * L::SLOT_BYTES + ti * 128;
 #pragma unroll
                 for (int h = 0; h < HALVES; ++h)
 #pragma unroll
@@ -731,6 +921,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         }
         flush_fold();
         epilogue(end);
+        const uint64_t t_streamed = p.timeline ? global_timer_ns() : 0;
         // Split segments: publish every partial piece of this run, then merge this
         // CTA's share of each (all owners are resident: cooperative launch).  Every
         // tile has been consumed, so the P buffers and the rings are scratch.
@@ -745,6 +936,12 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                                              reinterpret_cast<float *>(ring), misc + 20, stid, 1,
                                              abort_flag);
         }
+        if (p.timeline && stid == 0) {
+            unsigned long long *rec = p.timeline + TL_COLS * c;
+            rec[5] = t_scores;
+            rec[6] = t_streamed;
+            rec[7] = global_timer_ns();
+        }
     }
 
     // Timeline record and tensor-memory release.
@@ -757,11 +954,14 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     if (p.timeline && tid == 0) {
         unsigned sm;
         asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
-        unsigned long long *rec = p.timeline + 4 * c;
+        unsigned long long *rec = p.timeline + TL_COLS * c;
         rec[0] = t_start;
         rec[1] = global_timer_ns();
         rec[2] = sm;
         rec[3] = (unsigned long long)(end - start);
+        if (start >= end)
+            for (int x = 4; x < TL_COLS; ++x)
+                rec[x] = 0;
     }
 }
 

@@ -29,6 +29,11 @@ constexpr unsigned DEV_TIMEOUT = 4u;
 // Upper bound on any single in-kernel wait; a healthy wait lasts microseconds.
 constexpr uint64_t WAIT_LIMIT_NS = 1500000000ull;
 
+// Per-CTA timeline row (Params::timeline): start ns, end ns, SM id, tiles, then the
+// phases of a tensor-core CTA with work (0 elsewhere): first TMA issue, first
+// scores ready, end of streaming (last piece closed), end of merging.
+constexpr int TL_COLS = 8;
+
 struct Params {
     const uint16_t *q;            // [B, Hq, D] bf16
     const uint16_t *k;            // [num_blocks, Hkv, block_size, D] bf16
@@ -55,7 +60,7 @@ struct Params {
     int bs_shift;
     float qscale;                 // scale * log2(e) (* k_scale for FP8): scores in log2 units
     float vscale;                 // FP8 cache: v_scale, applied to the output (1 for bf16)
-    unsigned long long *timeline; // optional [grid][4]: start ns, end ns, SM id, tiles
+    unsigned long long *timeline; // optional [grid][TL_COLS], see TL_COLS
 };
 
 // floor(t / block_size) for 0 <= t < 2^31 without a divide: with l = ceil(log2 bs)
@@ -71,6 +76,12 @@ __device__ __forceinline__ int page_of(const Params &p, int t)
 // Walks the global tile order one tile at a time.  prefix[b] = sum of n_b'
 // (b' < b) lives in shared memory; units = Hkv * hch segments per request.  Only
 // init() divides; next() is increments and compares.
+// Global tile order: head chunk outermost, then request, KV head, tile, i.e.
+// (hc, b, kvh, j).  With one head chunk this is (b, kvh, j).  With several, the
+// CTAs of the chunks run over the same (b, kvh, j) ranges side by side (exactly
+// when the grid divides by the chunk count), so a K/V tile is read from HBM once
+// and from L2 by the other chunks.  A segment is the nb tiles of one
+// (b, kvh, hc); W = hch * Hkv * prefix[B].
 struct TileIter {
     int b, kvh, hc;
     int j;         // tile index inside the segment
@@ -80,40 +91,47 @@ struct TileIter {
     __device__ __forceinline__ void init(int64_t i, const int *prefix, int B, int64_t units,
                                          int hch)
     {
-        int lo = 0, hi = B;  // units*prefix[lo] <= i < units*prefix[hi]
+        const int64_t hkv = units / hch;
+        const int64_t w1 = hkv * prefix[B];  // tiles per head chunk
+        hc = (int)(i / w1);
+        const int64_t i1 = i - (int64_t)hc * w1;
+        int lo = 0, hi = B;  // hkv*prefix[lo] <= i1 < hkv*prefix[hi]
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (units * prefix[mid] <= i)
+            if (hkv * prefix[mid] <= i1)
                 lo = mid;
             else
                 hi = mid;
         }
         b = lo;
         nb = prefix[lo + 1] - prefix[lo];
-        const int64_t local = i - units * prefix[lo];
-        const int64_t vs = local / nb;
-        j = (int)(local - vs * nb);
-        kvh = (int)(vs / hch);
-        hc = (int)(vs - (int64_t)kvh * hch);
-        seg0 = units * prefix[lo] + vs * nb;
+        const int64_t local = i1 - hkv * prefix[lo];
+        kvh = (int)(local / nb);
+        j = (int)(local - (int64_t)kvh * nb);
+        seg0 = (int64_t)hc * w1 + hkv * prefix[lo] + (int64_t)kvh * nb;
     }
 
     // Advance to the next tile; the caller guarantees one exists.
     __device__ __forceinline__ void next(const int *prefix, int B, int Hkv, int hch)
     {
+        (void)hch;
         if (++j < nb)
             return;
         j = 0;
         seg0 += nb;
-        if (++hc < hch)
-            return;
-        hc = 0;
         if (++kvh < Hkv)
             return;
         kvh = 0;
+        // Next request with tiles; past the last one, the next head chunk's first.
         do {
             ++b;
-        } while (b < B - 1 && prefix[b + 1] == prefix[b]);
+        } while (b < B && prefix[b + 1] == prefix[b]);
+        if (b == B) {
+            ++hc;
+            b = 0;
+            while (prefix[b + 1] == prefix[b])
+                ++b;
+        }
         nb = prefix[b + 1] - prefix[b];
     }
 };

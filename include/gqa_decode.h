@@ -141,12 +141,17 @@ GQA_API int gqa_decode_fixed_split(const void *q, const void *k_cache, const voi
  * gqa_decode (num_splits = 0, the stream-K schedule) or gqa_decode_fixed_split
  * (num_splits >= 1) computes, with the same arguments, workspace and errors, and
  * in addition writes one row per CTA of the decode kernel's grid:
- *   timeline  DEVICE buffer, unsigned 64-bit [timeline_rows][4], 8-byte aligned,
- *             borrowed.  Row c = { start ns, end ns, SM id, tiles }: the GPU's
- *             global nanosecond timer when CTA c began and when it finished
- *             (after any merge it took part in), the SM it ran on, and the
- *             number of tiles (work units) in its run: 128 tokens each on the
- *             tensor-core kernel, the kernel's own tile size on the CUDA cores.
+ *   timeline  DEVICE buffer, unsigned 64-bit [timeline_rows][8], 8-byte aligned,
+ *             borrowed.  Row c = { start ns, end ns, SM id, tiles, first TMA ns,
+ *             first scores ns, streamed ns, merged ns }: the GPU's global
+ *             nanosecond timer when CTA c began and when it finished (after any
+ *             merge it took part in), the SM it ran on, and the number of tiles
+ *             (work units) in its run: 128 tokens each on the tensor-core
+ *             kernel, the kernel's own tile size on the CUDA cores.  For a
+ *             tensor-core CTA with work, the last four are the timer when it
+ *             issued its first K tile, when the first tile's scores were ready,
+ *             when its last piece was closed, and when its merges were done;
+ *             they are 0 for other CTAs and on the CUDA cores.
  *   grid      HOST int or NULL; receives the number of rows written (0 for B = 0).
  * timeline_rows below the grid returns GQA_ERR_WORKSPACE_TOO_SMALL without
  * launching (grid is still set), so a caller may size the buffer from a first

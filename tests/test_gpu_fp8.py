@@ -1,5 +1,6 @@
 """GPU parity of the FP8 E4M3 cache path (gqa_decode_fp8) against the fp64 oracle
-on the same E4M3 bytes and scales."""
+on the same E4M3 bytes and scales: the tensor-core kernel (D = 128, G >= 4) and
+the CUDA-core kernel (the other shapes)."""
 import pytest
 import torch
 
@@ -20,6 +21,8 @@ CASES = [
     (3, 4, 2, 64, [128, 127, 900], 8),
     (2, 16, 4, 256, [777, 2], 16),
     (1, 4, 1, 128, [60000], None),          # one long segment over every CTA
+    (2, 16, 2, 128, [5000, 300], 32),       # G = 8
+    (1, 32, 2, 128, [40000], 64),           # G = 16, long: split segments merged
 ]
 
 

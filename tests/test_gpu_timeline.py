@@ -1,6 +1,7 @@
 """GPU: the per-CTA timeline entry point (gqa_decode_timeline) computes what
 gqa_decode and gqa_decode_fixed_split compute, bit for bit, and records one sane
-row (start ns, end ns, SM id, tiles) per CTA of the decode kernel's grid."""
+row (start ns, end ns, SM id, tiles, then the phase times of a tensor-core CTA)
+per CTA of the decode kernel's grid."""
 import ctypes
 import math
 
@@ -15,14 +16,24 @@ from workloads import make_problem
 pytestmark = pytest.mark.gpu
 
 
-def _rows_ok(tl, tiles=None):
+def _rows_ok(tl, tiles=None, phases=True):
     t = tl.cpu()
-    assert t.dim() == 2 and t.shape[1] == 4 and t.shape[0] >= 1
+    assert t.dim() == 2 and t.shape[1] == gq.TIMELINE_COLS and t.shape[0] >= 1
     assert torch.all(t[:, 0] > 0) and torch.all(t[:, 1] >= t[:, 0])
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     assert torch.all((t[:, 2] >= 0) & (t[:, 2] < sms))
     if tiles is not None:
         assert int(t[:, 3].sum()) == tiles
+    work = t[:, 3] > 0
+    if phases:
+        # start <= first TMA <= first scores <= streamed <= merged <= end, CTAs with work
+        w = t[work]
+        seq = [w[:, 0], w[:, 4], w[:, 5], w[:, 6], w[:, 7], w[:, 1]]
+        for a, b in zip(seq, seq[1:]):
+            assert torch.all(a <= b)
+        assert torch.all(t[~work][:, 4:] == 0)
+    else:
+        assert torch.all(t[:, 4:] == 0)
     return t
 
 
@@ -82,7 +93,7 @@ def test_cuda_core_timeline():
     torch.cuda.synchronize()
     assert ws.status() == 0
     assert torch.equal(out, ref)
-    t = _rows_ok(tl)
+    t = _rows_ok(tl, phases=False)
     assert int(t[:, 3].sum()) > 0
 
 
@@ -92,7 +103,7 @@ def test_timeline_buffer_too_small_launches_nothing():
     ws = gq.Workspace(d.q.device)
     lib = gq.load_library()
     out = torch.full_like(d.q, 7.0)
-    tl = torch.zeros((1, 4), dtype=torch.int64, device="cuda")
+    tl = torch.zeros((1, gq.TIMELINE_COLS), dtype=torch.int64, device="cuda")
     grid = ctypes.c_int(0)
     B, Hq, Hkv, D, bs, mb, nb = gq._shape(d.q, d.k_cache, d.block_table)
     buf = ws.get(gq.workspace_size(B, Hq, Hkv, D, 0))

@@ -45,7 +45,10 @@ def test_bench_kernel_mapping():
                                                    block_size=48)) == "gqa_decode_simt_kernel"
     p = workloads.make_problem("e", 1, 32, 8, 128, [10], seed=1)
     p.meta["kv_elem_bytes"] = 1
-    assert "FP8" in bench.kernel_for(p)
+    assert bench.kernel_for(p) == "gqa_decode_tc_kernel<4> (FP8 E4M3 cache)"
+    p = workloads.make_problem("f", 1, 32, 8, 64, [10], seed=1)
+    p.meta["kv_elem_bytes"] = 1
+    assert bench.kernel_for(p) == "gqa_decode_simt_kernel (FP8 E4M3 cache)"   # D = 64
     # traffic records are keyed to each kernel's own sources
     assert bench.kernel_source_hash("gqa_decode_tc_kernel<4>") != \
         bench.kernel_source_hash("gqa_decode_simt_kernel")
@@ -59,9 +62,9 @@ def test_fixed_split_workspace_grows_with_splits():
 def test_timeline_summary():
     import numpy as np
     # Three CTAs over a 10 us span: busy 10 + 8 + 2 = 20 of 30 us; the idle one has no tiles.
-    tl = np.array([[1000, 11000, 0, 5],
-                   [2000, 10000, 1, 4],
-                   [1000, 3000, 2, 0]])
+    tl = np.array([[1000, 11000, 0, 5, 1500, 3000, 9000, 10500],
+                   [2000, 10000, 1, 4, 2500, 4000, 9500, 9900],
+                   [1000, 3000, 2, 0, 0, 0, 0, 0]])
     s = gq.timeline_summary(tl)
     assert s["ctas"] == 3 and s["ctas_with_work"] == 2 and s["sms"] == 3 and s["tiles"] == 9
     assert abs(s["span_us"] - 10.0) < 1e-12
@@ -69,10 +72,18 @@ def test_timeline_summary():
     assert abs(s["tail_idle"] - 10.0 / 30.0) < 1e-12
     assert s["start_us_max"] == 1.0
     assert s["end_us_min"] == 9.0 and s["end_us_max"] == 10.0   # CTAs with tiles only
+    ph = s["phases_us"]                 # after each CTA's own start, recorded rows only
+    assert ph["first_tma"] == {"median": 0.5, "max": 0.5}
+    assert ph["first_scores"] == {"median": 2.0, "max": 2.0}
+    assert ph["streamed"] == {"median": 7.75, "max": 8.0}
+    assert ph["merged"] == {"median": 8.7, "max": 9.5}
+    assert gq.timeline_summary(np.array([[0, 5, 0, 1] + [0] * 4]))["phases_us"] == {}
     with pytest.raises(ValueError):
-        gq.timeline_summary(np.array([[5, 4, 0, 1]]))             # ends before it starts
+        gq.timeline_summary(np.array([[5, 4, 0, 1] + [0] * 4]))   # ends before it starts
     with pytest.raises(ValueError):
-        gq.timeline_summary(np.zeros((0, 4)))
+        gq.timeline_summary(np.zeros((0, 8)))
+    with pytest.raises(ValueError):
+        gq.timeline_summary(np.zeros((2, 4)))                     # rows of the wrong width
 
 
 def test_cpu_baseline_reports_parity_of_its_sample():
