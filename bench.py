@@ -48,22 +48,12 @@ KERNEL_SOURCES = {
 }
 
 
-def kernel_for(p) -> str:
-    """Which decode kernel the library runs for this problem (mirrors the library's
-    dispatch: tensor cores for D = 64 or 128 (FP8 caches: D = 128) with at least 4
-    query heads per KV head and pages that tile into 128-token boxes, CUDA cores
-    otherwise)."""
-    bs = p.block_size
-    boxes = (not p.paged) or (bs % 128 == 0 if bs >= 128 else (bs >= 8 and 128 % bs == 0))
-    if p.meta.get("kv_elem_bytes") == 1:
-        if p.D == 128 and p.G >= 4 and p.B <= 1024 and boxes:
-            nv = 4 if p.G <= 4 else (8 if p.G <= 8 else 16)
-            return f"gqa_decode_tc_kernel<{nv}> (FP8 E4M3 cache)"
-        return "gqa_decode_simt_kernel (FP8 E4M3 cache)"
-    if p.D in (64, 128) and p.G >= 4 and p.B <= 1024 and boxes:
-        nv = 4 if p.G <= 4 else (8 if p.G <= 8 else 16)
-        return f"gqa_decode_tc_kernel<{nv}>"
-    return "gqa_decode_simt_kernel"
+def plan_for(gq, p, num_splits: int, device: int) -> dict:
+    """What the library launches for this problem and schedule (gqa_decode_plan):
+    the kernel, its template parameters, grid and LeanTiles."""
+    return gq.decode_plan(p.B, p.Hq, p.Hkv, p.D, p.block_size, p.paged, p.num_blocks,
+                          kv_fp8=p.meta.get("kv_elem_bytes") == 1, num_splits=num_splits,
+                          seq_lens_host=p.seq_lens.to(torch.int32), device=device)
 
 
 def parse():
@@ -84,6 +74,10 @@ def parse():
                          "one CTA per SM, FlashDecoding's usual choice)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target duration of the CPU-baseline sample")
+    ap.add_argument("--workloads", default="default",
+                    help="comma-separated workloads timed after the headline in the same run "
+                         "(default: the other configurations and sweep points when the "
+                         "headline is the default llama3_8b at 1 GPU; '' for none)")
     return ap.parse_args()
 
 
@@ -97,7 +91,7 @@ def hbm_peak():
 
 
 def kernel_source_hash(kernel: str) -> str:
-    """Hash of the sources of the named kernel (a kernel_for() name)."""
+    """Hash of the sources of the named kernel (a gqa_decode_plan kernel name)."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES["tc" if "tc_kernel" in kernel else "simt"]:
         with open(os.path.join(ROOT, rel), "rb") as f:
@@ -297,22 +291,129 @@ def run_reference(args, rank: int):
     print(json.dumps(line), flush=True)
 
 
-def step_timeline(gq, d, p, out, ws, stream, flush, splits, schedule):
-    """One more step, untimed and after an L2 flush, through gqa_decode_timeline with
-    the schedule the timed steps ran: per-CTA start/end (%globaltimer) and SM, summed
-    up as span, busy fraction and tail idle."""
-    ns = splits if splits else (1 if schedule.startswith("auto: one CTA") else 0)
-    flush.fill_(0)
-    _, tl = gq.gqa_decode_timeline(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,
-                                   num_splits=ns, out=out, scale=p.scale, workspace=ws,
-                                   stream=stream)
-    torch.cuda.synchronize()
-    if ws.status():
-        raise SystemExit("device status error during the timeline step")
-    summary = gq.timeline_summary(tl)
-    summary["source"] = ("one untimed step through gqa_decode_timeline, same schedule: "
-                         "per-CTA %globaltimer at entry and exit, %smid")
-    return summary
+# Workloads the default run times after the headline, each in the same process and
+# on the same GPU (the other configurations of the metric and the sweep points).
+EXTRA_WORKLOADS = ("long_256k", "varlen_paged", "llama3_8b_fp8", "tiny", "sweep_32_32_128",
+                   "sweep_32_8_128", "sweep_64_4_128", "sweep_64_1_128", "sweep_32_8_64",
+                   "sweep_16_4_256")
+EXTRA_STEPS = 200
+
+
+class Runner:
+    """One workload resident on the GPU and the call that runs one decode step of it
+    (the schedule as the library plans it: gqa_decode_plan)."""
+
+    def __init__(self, gq, p, dev, args, flush):
+        self.gq, self.p, self.dev, self.flush = gq, p, dev, flush
+        self.fp8 = p.meta.get("kv_elem_bytes") == 1
+        self.d = p.to(dev)
+        if self.fp8:  # the cache as FP8 E4M3 bytes with per-tensor scales
+            k8, v8, self.k_scale, self.v_scale = workloads.fp8_caches(p)
+            self.d.k_cache, self.d.v_cache = k8.to(dev), v8.to(dev)
+        self.out = torch.empty_like(self.d.q)
+        self.ws = gq.Workspace(dev)
+        self.stream = torch.cuda.current_stream(dev)
+        self.lens_host = p.seq_lens.to(torch.int32).contiguous()
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        self.mode = "stream-K" if self.fp8 else args.schedule
+        if self.mode == "fixed":
+            segs = p.B * p.Hkv * -(-p.G // 16)
+            self.splits = args.splits if args.splits > 0 else max(1, -(-sms // segs))
+        else:
+            self.splits = -1 if self.mode == "auto" else 0
+        self.plan = plan_for(gq, p, self.splits, dev.index)
+        ns = self.plan["num_splits"]
+        what = ("stream-K" if ns == 0 else "one CTA per (request, KV head)" if ns == 1
+                else f"fixed split x{ns}")
+        self.schedule = (f"auto: {what}" if self.mode == "auto" else what) + \
+            (" (FP8 cache)" if self.fp8 else "")
+
+    def launches_per_step(self) -> int:
+        return 2 if self.plan["merge_launch"] else 1
+
+    def step(self):
+        gq, d, p = self.gq, self.d, self.p
+        kw = dict(out=self.out, scale=p.scale, workspace=self.ws, stream=self.stream)
+        if self.fp8:
+            gq.gqa_decode_fp8(d.q, d.k_cache, d.v_cache, self.k_scale, self.v_scale,
+                              d.block_table, d.seq_lens, **kw)
+        elif self.mode == "fixed":
+            gq.gqa_decode_fixed_split(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,
+                                      self.splits, **kw)
+        elif self.mode == "auto":
+            gq.gqa_decode_auto(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,
+                               self.lens_host, **kw)
+        else:
+            gq.gqa_decode(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens, **kw)
+
+    def warm(self, n: int):
+        for _ in range(max(3, n)):
+            self.flush.fill_(1)
+            self.step()
+        torch.cuda.synchronize(self.dev)
+        if self.ws.status():
+            raise SystemExit(f"{self.p.name}: device status error during warm-up")
+
+    def timed(self, steps: int):
+        """Per-step milliseconds (CUDA events on the launching stream around each
+        step; L2 flushed by a 256 MiB write before each) and the whole region's."""
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        region0 = torch.cuda.Event(enable_timing=True)
+        region1 = torch.cuda.Event(enable_timing=True)
+        region0.record(self.stream)
+        for i in range(steps):
+            self.flush.fill_(i & 0xFF)
+            starts[i].record(self.stream)
+            self.step()
+            ends[i].record(self.stream)
+        region1.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        if self.ws.status():
+            raise SystemExit(f"{self.p.name}: device status error during the timed steps")
+        return [s.elapsed_time(e) for s, e in zip(starts, ends)], region0.elapsed_time(region1)
+
+    def timeline(self):
+        """One more step, untimed and after an L2 flush, through gqa_decode_timeline
+        with the schedule the timed steps ran: per-CTA start/end (%globaltimer) and
+        SM, summed up as span, busy fraction and tail idle, plus the phase times of
+        the tensor-core CTAs."""
+        if self.fp8:
+            return None
+        ns = self.plan["num_splits"]
+        d, p = self.d, self.p
+        self.flush.fill_(0)
+        _, tl = self.gq.gqa_decode_timeline(d.q, d.k_cache, d.v_cache, d.block_table,
+                                            d.seq_lens, num_splits=ns, out=self.out,
+                                            scale=p.scale, workspace=self.ws,
+                                            stream=self.stream)
+        torch.cuda.synchronize(self.dev)
+        if self.ws.status():
+            raise SystemExit(f"{p.name}: device status error during the timeline step")
+        summary = self.gq.timeline_summary(tl)
+        summary["source"] = ("one untimed step through gqa_decode_timeline, same schedule: "
+                             "per-CTA %globaltimer at entry and exit, %smid")
+        return summary
+
+
+def extra_entry(r: Runner, steps: int, warmup: int, peak: float) -> dict:
+    """One workload of the multi-workload block: timed like the headline, fewer steps."""
+    r.warm(warmup)
+    per, _ = r.timed(steps)
+    ms = sum(per) / len(per)
+    gbs = r.p.algorithmic_bytes() / (ms / 1e3) / 1e9
+    tl = r.timeline()
+    e = {"us_per_step": ms * 1e3, "us_per_step_median": statistics.median(per) * 1e3,
+         "GB_per_s": gbs, "frac": gbs / peak, "steps": steps,
+         "algorithmic_bytes": r.p.algorithmic_bytes(), "kernel": r.plan["kernel_name"],
+         "schedule": r.schedule, "grid": r.plan["grid"], "tiles": r.plan["tiles"],
+         "gpu_launches": steps * r.launches_per_step()}
+    if tl:
+        e["tail_idle"] = tl["tail_idle"]
+        e["span_us"] = tl["span_us"]
+        if tl.get("phases_us"):
+            e["phases_us_median"] = {k: v["median"] for k, v in tl["phases_us"].items()}
+    return e
 
 
 def main():
@@ -338,86 +439,30 @@ def main():
                                 device_id=dev)
         pg = dist
 
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     p = workloads.workload(args.workload)
-    fp8 = p.meta.get("kv_elem_bytes") == 1
-    d = p.to(dev)
-    if fp8:  # the cache as FP8 E4M3 bytes with per-tensor scales
-        k8, v8, k_scale, v_scale = workloads.fp8_caches(p)
-        d.k_cache, d.v_cache = k8.to(dev), v8.to(dev)
+    r = Runner(gq, p, dev, args, flush)
+    if r.fp8:
         args.no_e2e = True  # the host-buffer entry point takes bf16 caches
         args.no_cpu_baseline = True  # (bench.py --impl reference times the FP8 oracle)
-    out = torch.empty_like(d.q)
-    ws = gq.Workspace(dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    splits = 0
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    lens_host = p.seq_lens.to(torch.int32).contiguous()
-    if fp8:
-        schedule = "stream-K (FP8 cache)"
-    elif args.schedule == "fixed":
-        segs = p.B * p.Hkv * -(-p.G // 16)
-        splits = args.splits if args.splits > 0 else max(1, -(-sms // segs))
-        schedule = f"fixed-split x{splits}"
-    elif args.schedule == "auto":
-        chosen, _ = gq.select_schedule(lens_host, p.Hq, p.Hkv, p.D, sms, max_splits=1)
-        schedule = "auto: one CTA per (request, KV head)" if chosen else "auto: stream-K"
-    else:
-        schedule = "stream-K"
-
-    def step():
-        if fp8:
-            gq.gqa_decode_fp8(d.q, d.k_cache, d.v_cache, k_scale, v_scale, d.block_table,
-                              d.seq_lens, out=out, scale=p.scale, workspace=ws, stream=stream)
-        elif splits:
-            gq.gqa_decode_fixed_split(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,
-                                      splits, out=out, scale=p.scale, workspace=ws, stream=stream)
-        elif args.schedule == "auto":
-            gq.gqa_decode_auto(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens, lens_host,
-                               out=out, scale=p.scale, workspace=ws, stream=stream)
-        else:
-            gq.gqa_decode(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens, out=out,
-                          scale=p.scale, workspace=ws, stream=stream)
-
-    for _ in range(max(3, args.warmup)):
-        flush.fill_(1)
-        step()
-    torch.cuda.synchronize(dev)
-    if ws.status():
-        raise SystemExit("device status error during warm-up")
+    r.warm(args.warmup)
 
     props = torch.cuda.get_device_properties(dev)
     uuid = getattr(props, "uuid", None)
     sampler = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local_rank))
     sampler.start()
     time.sleep(0.3)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     if pg:
         pg.barrier()
     torch.cuda.synchronize(dev)
     t0 = time.time()
-    region0 = torch.cuda.Event(enable_timing=True)
-    region1 = torch.cuda.Event(enable_timing=True)
-    region0.record(stream)
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        starts[i].record(stream)
-        step()
-        ends[i].record(stream)
-    region1.record(stream)
-    torch.cuda.synchronize(dev)
+    per, region_ms = r.timed(args.steps)
     if pg:
         pg.barrier()
     t1 = time.time()
     sampler.stop()
-    if ws.status():
-        raise SystemExit("device status error during the timed steps")
 
-    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = sum(per) / len(per)
-    region_ms = region0.elapsed_time(region1)
     if pg:
         tt = torch.tensor([ms], device=dev)
         pg.all_reduce(tt, op=pg.ReduceOp.MAX)
@@ -428,10 +473,11 @@ def main():
     peak, peak_kind = hbm_peak()
     achieved = bytes_step / (ms / 1e3) / 1e9
     clocks = sampler.summary(t0, t1)
+    plan = r.plan
 
     line = None
     if rank == 0:
-        traffic = profiled_traffic(p.name, kernel_for(p))
+        traffic = profiled_traffic(p.name, plan["kernel_name"])
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -440,24 +486,44 @@ def main():
             "pct_of_spec_8tbs": 100.0 * achieved / SPEC_HBM_GBS,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 q/K/V; no trained weights)",
-            "config": dict(workload_config(p), schedule=schedule),
+            "config": dict(workload_config(p), schedule=r.schedule),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
-                         "kernel": kernel_for(p),
+                         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)"
+                         if peak_kind == "measured" else
+                         "fallback (MEASURED_PEAKS.json absent: the recipe's 6.65 TB/s)",
+                         "kernel": plan["kernel_name"], "grid": plan["grid"],
+                         "tiles": plan["tiles"],
                          "algorithmic_bytes_per_launch": bytes_step},
-            "gpu_launches": args.steps * (2 if splits > 1 else 1),
+            "gpu_launches": args.steps * r.launches_per_step(),
             "timed_region_ms": region_ms,
             "clocks": clocks,
         }
-    if rank == 0 and not fp8:
-        line["timeline"] = step_timeline(gq, d, p, out, ws, stream, flush, splits, schedule)
-    if splits:  # comparator runs report the kernel numbers only
+        tl = r.timeline()
+        if tl:
+            line["timeline"] = tl
+    if r.mode == "fixed":  # comparator runs report the kernel numbers only
         args.no_e2e = args.no_cpu_baseline = True
     if rank == 0 and not args.no_e2e:
-        line["e2e"] = measure_e2e(gq, p, dev, args, stream)
+        line["e2e"] = measure_e2e(gq, p, dev, args, r.stream)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_oracle_sample(p, args.cpu_seconds, gpu_out=out)
+        line["cpu_baseline"] = cpu_oracle_sample(p, args.cpu_seconds, gpu_out=r.out)
+    extras = [w for w in (args.workloads.split(",") if args.workloads else ()) if w]
+    if args.workloads == "default":
+        extras = list(EXTRA_WORKLOADS) if (world == 1 and args.workload == "llama3_8b"
+                                           and r.mode == "auto") else []
+    if rank == 0 and extras:
+        del r
+        block = {}
+        for name in extras:
+            rr = Runner(gq, workloads.workload(name), dev, args, flush)
+            block[name] = extra_entry(rr, min(args.steps, EXTRA_STEPS), args.warmup, peak)
+            del rr
+            torch.cuda.empty_cache()
+        line["workloads"] = block
+        line["workloads_note"] = ("other configurations timed in the same run, same method "
+                                  "(L2 flushed before each step, CUDA events), "
+                                  f"min(steps, {EXTRA_STEPS}) steps each; frac of the same peak")
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg:

@@ -34,9 +34,23 @@ EXPORTED = ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states", "gqa
             "gqa_status", "gqa_decode_host_buffer_bytes", "gqa_decode_host", "gqa_error_string",
             "gqa_decode_noalloc", "gqa_decode_fixed_split_workspace_size",
             "gqa_decode_fixed_split", "gqa_select_schedule", "gqa_decode_auto",
-            "gqa_decode_multi", "gqa_decode_fp8", "gqa_decode_timeline")
+            "gqa_decode_multi", "gqa_decode_fp8", "gqa_decode_timeline", "gqa_decode_plan")
 GQA_ERR_SCRATCH_LIMIT = 6
 TIMELINE_COLS = 8  # values per CTA row of gqa_decode_timeline
+KERNEL_TENSOR_CORE = 1
+KERNEL_CUDA_CORE = 2
+
+
+class _Plan(ctypes.Structure):
+    """gqa_plan of include/gqa_decode.h."""
+    _fields_ = [("kernel", ctypes.c_int), ("heads_per_pass", ctypes.c_int),
+                ("head_chunks", ctypes.c_int), ("num_splits", ctypes.c_int),
+                ("grid", ctypes.c_int), ("threads_per_cta", ctypes.c_int),
+                ("cooperative", ctypes.c_int), ("merge_launch", ctypes.c_int),
+                ("tile_tokens", ctypes.c_int), ("ring_stages", ctypes.c_int),
+                ("box_rows", ctypes.c_int), ("tiles", ctypes.c_longlong),
+                ("smem_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t),
+                ("kernel_name", ctypes.c_char * 64)]
 
 _lib = None
 
@@ -73,13 +87,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_decode_fp8.argtypes = [P, P, P, F, F, P, P, P, I, I, I, I, I, F, I, I, P, SZ, P]
     lib.gqa_decode_timeline.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, I,
                                         ctypes.POINTER(I), P, SZ, P]
+    lib.gqa_decode_plan.argtypes = [I, I, I, I, I, I, I, I, I, I, P, I, ctypes.POINTER(_Plan)]
+    lib.gqa_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P]
     lib.gqa_error_string.argtypes = [I]
     lib.gqa_error_string.restype = ctypes.c_char_p
     for name in ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states",
                  "gqa_merge_states", "gqa_status", "gqa_decode_host",
                  "gqa_decode_fixed_split_workspace_size", "gqa_decode_fixed_split",
                  "gqa_select_schedule", "gqa_decode_auto", "gqa_decode_multi",
-                 "gqa_decode_fp8"):
+                 "gqa_decode_fp8", "gqa_decode_plan", "gqa_decode_noalloc",
+                 "gqa_decode_timeline"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -401,6 +418,34 @@ def gqa_decode_multi(q, k_cache, v_cache, block_table, seq_lens, out=None, scale
     return out
 
 
+def decode_plan(B: int, Hq: int, Hkv: int, D: int, block_size: int, paged: bool,
+                num_blocks: int = 0, qlen: int = 1, kv_fp8: bool = False, num_splits: int = 0,
+                seq_lens_host=None, device: int | None = None) -> dict:
+    """What a call would launch (the C ABI's gqa_decode_plan): kernel, template
+    parameters, schedule, grid, LeanTiles.  num_splits: -1 = gqa_decode_auto's choice
+    (needs seq_lens_host and a device), 0 = stream-K, n = fixed split.  device < 0
+    skips the device query (grid -1 for stream-K)."""
+    lib = load_library()
+    if device is None:
+        device = torch.cuda.current_device()
+    lens = None
+    if seq_lens_host is not None:
+        lens = (seq_lens_host.detach().to("cpu", torch.int32).contiguous()
+                if torch.is_tensor(seq_lens_host)
+                else torch.tensor(list(seq_lens_host), dtype=torch.int32))
+        if lens.numel() != B:
+            raise ValueError("seq_lens_host must hold B lengths")
+    pl = _Plan()
+    _check("gqa_decode_plan",
+           lib.gqa_decode_plan(B, Hq, Hkv, D, block_size, int(bool(paged)), num_blocks, qlen,
+                               int(bool(kv_fp8)), num_splits,
+                               None if lens is None else ctypes.c_void_p(lens.data_ptr()),
+                               int(device), ctypes.byref(pl)))
+    out = {name: getattr(pl, name) for name, _ in _Plan._fields_}
+    out["kernel_name"] = pl.kernel_name.decode()
+    return out
+
+
 def select_schedule(seq_lens, Hq: int, Hkv: int, D: int, num_sms: int, max_splits: int = 64):
     """Host-side schedule choice: (num_splits, est_us) with num_splits = 0 for the
     stream-K gqa_decode, n > 0 for gqa_decode_fixed_split with n chunks; est_us =
@@ -502,18 +547,25 @@ def gqa_decode_noalloc(q, k_cache, v_cache, block_table, seq_lens, out=None, sca
     """gqa_decode for callers that cannot allocate device memory: the library uses
     its own fixed 8 MiB device scratch instead of a workspace.  Calls on one device
     share that scratch, so they must not overlap on the GPU.  (`out` is allocated
-    here only when the caller passes none.)"""
+    here only when the caller passes none.)  Tensors are checked as gqa_decode
+    checks them, before anything is launched."""
     lib = load_library()
-    fn = lib.gqa_decode_noalloc
-    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-    fn.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P]
-    fn.restype = I
     B, Hq, Hkv, D, bs, mb, nb = _shape(q, k_cache, block_table)
+    dev = q.device
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _require(t, n, torch.bfloat16, dev)
+    _require(seq_lens, "seq_lens", torch.int32, dev)
+    if block_table is not None:
+        _require(block_table, "block_table", torch.int32, dev)
     if out is None:
         out = torch.empty_like(q)
+    _require(out, "out", torch.bfloat16, dev)
+    if tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out must have q's shape")
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
-    with torch.cuda.device(q.device):
-        rc = fn(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
-                _ptr(out), B, Hq, Hkv, D, bs, scale, mb, nb, _stream_ptr(stream))
+    with torch.cuda.device(dev):
+        rc = lib.gqa_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                    _ptr(seq_lens), _ptr(out), B, Hq, Hkv, D, bs, scale, mb, nb,
+                                    _stream_ptr(stream))
     _check("gqa_decode_noalloc", rc)
     return out

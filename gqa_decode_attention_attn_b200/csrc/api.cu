@@ -4,6 +4,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <queue>
@@ -64,6 +65,8 @@ struct Variant {
     size_t smem_max;                  // shared memory at the largest batch
     size_t (*smem)(int B);
     int slot_floats;
+    int tile_tokens;                  // tokens per LeanTile
+    int stages;                       // ring stages
 };
 
 template <int D, int GC, bool ST, bool F8>
@@ -71,7 +74,7 @@ Variant make_variant()
 {
     using C = SimtCfg<D, GC, F8>;
     return Variant{simt_fn<D, GC, ST, F8>(), C::THREADS, C::smem_bytes(GQA_MAX_BATCH), &C::smem_bytes,
-                   C::SLOT_FLOATS};
+                   C::SLOT_FLOATS, C::T, C::STAGES};
 }
 
 template <bool ST, bool F8>
@@ -231,9 +234,9 @@ bool tc_head_dim(int D)
 // ---- tensor-core path: applicability and tensor maps -------------------------
 
 // Tokens per TMA box along the cache rows: one box per page, 128 for big pages.
-int tc_box_rows(const int32_t *block_table, int block_size)
+int tc_box_rows(bool paged, int block_size)
 {
-    if (!block_table)
+    if (!paged)
         return 128;
     if (block_size >= 128)
         return block_size % 128 == 0 ? 128 : 0;
@@ -241,14 +244,14 @@ int tc_box_rows(const int32_t *block_table, int block_size)
 }
 
 // R = query rows per KV head (query tokens x G).
-bool tc_applicable(bool states, int B, int Hq, int Hkv, int D, int block_size,
-                   const int32_t *block_table, int num_blocks, int R)
+bool tc_applicable(bool states, int B, int Hkv, int D, int block_size, bool paged,
+                   int num_blocks, int R)
 {
     if (states || !tc_head_dim(D) || R < TC_MIN_G || B > TcCfg::MAX_BATCH)
         return false;
-    if (tc_box_rows(block_table, block_size) == 0)
+    if (tc_box_rows(paged, block_size) == 0)
         return false;
-    const int64_t blocks = block_table ? num_blocks : B;
+    const int64_t blocks = paged ? num_blocks : B;
     const int64_t rows = blocks * Hkv * (int64_t)block_size;
     return rows > 0 && rows < (int64_t(1) << 31);
 }
@@ -332,6 +335,89 @@ int check_shape(int B, int Hq, int Hkv, int D, int block_size, const int32_t *bl
     return GQA_OK;
 }
 
+// Everything a call's launch depends on, decided on the host from the shape
+// alone: which kernel, how many query heads one pass carries, the grid, shared
+// memory and the workspace layout.  run_decode launches from it and
+// gqa_decode_plan reports it, so the two cannot disagree.
+struct Plan {
+    bool use_tc = false;   // tensor-core kernel (else the CUDA-core kernel)
+    bool mq = false;       // several query tokens per request
+    bool fp8 = false;
+    Variant v{};           // CUDA-core kernel variant
+    int G = 0, R = 0;      // query heads per KV head; query rows per KV head
+    int nv = 0;            // heads one pass carries (tensor cores: 4, 8, 16; CUDA cores: GC)
+    int hch = 0;           // passes (head chunks) per KV head
+    int nsplit = 0;        // 0: stream-K; n > 0: fixed split into n chunks
+    int ctas = 0;          // persistent grid; -1 when no device was given
+    int64_t items = 0;     // fixed split: CTAs of the decode kernel
+    int64_t grid = 0;      // CTAs of the decode kernel
+    int threads = 0;
+    int tile_tokens = 0;
+    int stages = 0;
+    size_t smem = 0;       // dynamic shared memory per CTA
+    int box_rows = 0;      // tensor cores: tokens per TMA box
+    WorkspaceLayout w{};
+};
+
+// dev < 0: no device query (the grid and the workspace are left at -1 / 0).
+int make_plan(bool states, int B, int Hq, int Hkv, int D, int block_size, bool paged,
+              int num_blocks, int qlen, bool fp8, int nsplit, int dev, Plan &pl)
+{
+    pl = Plan{};
+    if (qlen < 1 || qlen > GQA_MAX_QLEN)
+        return GQA_ERR_INVALID_ARG;
+    pl.G = Hq / Hkv;
+    pl.R = qlen * pl.G;
+    pl.mq = qlen > 1;
+    pl.fp8 = fp8;
+    // FP8 caches run on the tensor cores at D = 128 (one query token), else on the
+    // CUDA-core kernel.
+    pl.use_tc = (!fp8 || (D == 128 && qlen == 1)) &&
+                tc_applicable(states, B, Hkv, D, block_size, paged, num_blocks, pl.R);
+    if (!pl.use_tc && !pick_variant(D, pl.G, states, pl.v, fp8))
+        return GQA_ERR_UNSUPPORTED;
+    if (!pl.use_tc && qlen > 1)  // several query tokens run on the tensor-core kernel only
+        return GQA_ERR_UNSUPPORTED;
+    if (nsplit > 0 && !pl.use_tc)
+        return GQA_ERR_UNSUPPORTED;
+    if (pl.use_tc) {
+        pl.hch = (pl.R + TcCfg::NP - 1) / TcCfg::NP;
+        pl.nv = pl.R <= 4 ? 4 : (pl.R <= 8 ? 8 : 16);
+        pl.threads = TcCfg::THREADS;
+        pl.tile_tokens = TcCfg::T;
+        pl.stages = fp8 ? TcGeom<128, true>::STAGES
+                        : (D == 64 ? TcGeom<64>::STAGES : TcGeom<128>::STAGES);
+        pl.smem = tc_smem_bytes(D, B, fp8);
+        pl.box_rows = tc_box_rows(paged, block_size);
+    } else {
+        const int gc = head_chunk(pl.G);
+        pl.hch = (pl.G + gc - 1) / gc;
+        pl.nv = gc;
+        pl.threads = pl.v.threads;
+        pl.tile_tokens = pl.v.tile_tokens;
+        pl.stages = pl.v.stages;
+        pl.smem = pl.v.smem(B);
+    }
+    pl.nsplit = nsplit > 0 ? nsplit : 0;
+    pl.items = nsplit > 0 ? (int64_t)B * Hkv * pl.hch * nsplit : 0;
+    if (pl.items > (int64_t)1 << 30)
+        return GQA_ERR_INVALID_ARG;
+    if (dev < 0) {
+        pl.ctas = -1;
+        pl.grid = nsplit > 0 ? pl.items : -1;
+        return GQA_OK;
+    }
+    int rc = pl.use_tc ? tc_ctas(pl.R, dev, pl.ctas, pl.mq, D, fp8) : persistent_ctas(pl.v, dev, pl.ctas);
+    if (rc)
+        return rc;
+    // One chunk per segment (nsplit = 1) always finishes its segment: no slots.
+    pl.w = nsplit > 1    ? layout_for((int)((pl.items + 1) / 2), TcCfg::SLOT_FLOATS)
+           : nsplit == 1 ? layout_for(0, TcCfg::SLOT_FLOATS)
+                         : layout_for(pl.ctas, pl.use_tc ? TcCfg::SLOT_FLOATS : pl.v.slot_floats);
+    pl.grid = nsplit > 0 ? pl.items : pl.ctas;
+    return GQA_OK;
+}
+
 // nsplit = 0: the stream-K schedule; nsplit > 0: the fixed-split comparator
 // (tensor-core shapes only), a grid of one CTA per (segment, chunk) followed by
 // merge_split_kernel.
@@ -359,39 +445,25 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         return GQA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || (out && !aligned16(out)))
         return GQA_ERR_MISALIGNED;
-    const int G = Hq / Hkv;
-    if (qlen < 1 || qlen > GQA_MAX_QLEN)
-        return GQA_ERR_INVALID_ARG;
-    const int R = qlen * G;  // query rows per KV head
-    // FP8 caches run on the tensor cores at D = 128 (one query token), else on the
-    // CUDA-core kernel.
-    const bool use_tc = (!fp8 || (D == 128 && qlen == 1)) &&
-                        tc_applicable(states, B, Hq, Hkv, D, block_size, block_table, num_blocks, R);
-    Variant v;
-    if (!use_tc && !pick_variant(D, G, states, v, fp8))
-        return GQA_ERR_UNSUPPORTED;
-    if (!use_tc && qlen > 1)  // several query tokens run on the tensor-core kernel only
-        return GQA_ERR_UNSUPPORTED;
+    // Shape errors first (no device query), then the plan for the current device.
+    Plan pl;
+    if ((rc = make_plan(states, B, Hq, Hkv, D, block_size, block_table != nullptr, num_blocks, qlen,
+                        fp8, nsplit, -1, pl)))
+        return rc;
     int dev = 0;
     if ((rc = current_device(dev)))
         return rc;
-    int ctas = 0;
-    if ((rc = use_tc ? tc_ctas(R, dev, ctas, qlen > 1, D, fp8) : persistent_ctas(v, dev, ctas)))
+    if ((rc = make_plan(states, B, Hq, Hkv, D, block_size, block_table != nullptr, num_blocks, qlen,
+                        fp8, nsplit, dev, pl)))
         return rc;
-    if (nsplit > 0 && !use_tc)
-        return GQA_ERR_UNSUPPORTED;
-    const int hch_tc = (R + TcCfg::NP - 1) / TcCfg::NP;
-    const int64_t items = nsplit > 0 ? (int64_t)B * Hkv * hch_tc * nsplit : 0;
-    if (items > (int64_t)1 << 30)
-        return GQA_ERR_INVALID_ARG;
-    // One chunk per segment (nsplit = 1) always finishes its segment: no slots.
-    const WorkspaceLayout w = nsplit > 1    ? layout_for((int)((items + 1) / 2), TcCfg::SLOT_FLOATS)
-                              : nsplit == 1 ? layout_for(0, TcCfg::SLOT_FLOATS)
-                                            : layout_for(ctas, use_tc ? TcCfg::SLOT_FLOATS : v.slot_floats);
+    const bool use_tc = pl.use_tc;
+    const int G = pl.G, R = pl.R, ctas = pl.ctas;
+    const int64_t items = pl.items;
+    const WorkspaceLayout w = pl.w;
     if (workspace_bytes < w.total)
         return GQA_ERR_WORKSPACE_TOO_SMALL;
     // The decode kernel's grid: one timeline row (TL_COLS values) per CTA.
-    const int64_t grid = nsplit > 0 ? items : ctas;
+    const int64_t grid = pl.grid;
     if (grid_out)
         *grid_out = (int)grid;
     if (timeline && timeline_rows < grid)
@@ -423,7 +495,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     p.block_size = block_size;
     p.max_blocks = block_table ? max_blocks : 1;
     p.num_blocks = block_table ? num_blocks : B;
-    p.hch = use_tc ? hch_tc : (G + head_chunk(G) - 1) / head_chunk(G);
+    p.hch = pl.hch;
     p.nsplit = nsplit > 0 ? nsplit : 0;
     p.capacity = block_table ? (int64_t)max_blocks * block_size : (int64_t)block_size;
     p.qscale = scale * LOG2E * (fp8 ? k_scale : 1.0f);
@@ -440,7 +512,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     }
 
     if (use_tc) {
-        const int box_rows = tc_box_rows(block_table, block_size);
+        const int box_rows = pl.box_rows;
         const int64_t rows = (block_table ? (int64_t)num_blocks : (int64_t)B) * Hkv * block_size;
         CUtensorMap tmk, tmv;
         if (!encode_kv_map(&tmk, k_cache, rows, box_rows, D, fp8) ||
@@ -449,11 +521,10 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         if (nsplit > 0) {
             // Fixed split: as many CTAs as chunks, in waves; no CTA waits for another.
             const cudaStream_t st = static_cast<cudaStream_t>(stream);
-            tc_kernel_for(R, qlen > 1, D, fp8)<<<(unsigned)items, TcCfg::THREADS, tc_smem_bytes(D, B, fp8), st>>>(
+            tc_kernel_for(R, qlen > 1, D, fp8)<<<(unsigned)items, TcCfg::THREADS, pl.smem, st>>>(
                 p, tmk, tmv, box_rows);
             if (B > 0 && nsplit > 1) {
-                const int nv = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
-                const int64_t threads = (int64_t)B * Hkv * hch_tc * nv * D;
+                const int64_t threads = (int64_t)B * Hkv * pl.hch * pl.nv * D;
                 tc_merge_for(R, D)<<<(unsigned)((threads + 127) / 128), 128, 0, st>>>(p);
             }
             return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
@@ -464,7 +535,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)ctas);
         cfg.blockDim = dim3(TcCfg::THREADS);
-        cfg.dynamicSmemBytes = tc_smem_bytes(D, B, fp8);
+        cfg.dynamicSmemBytes = pl.smem;
         cfg.stream = static_cast<cudaStream_t>(stream);
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeCooperative;
@@ -474,7 +545,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         if (cudaLaunchKernelEx(&cfg, tc_kernel_for(R, qlen > 1, D, fp8), p, tmk, tmv, box_rows) != cudaSuccess)
             return GQA_ERR_CUDA;
     } else {
-        v.fn<<<ctas, v.threads, v.smem(B), static_cast<cudaStream_t>(stream)>>>(p);
+        pl.v.fn<<<ctas, pl.threads, pl.smem, static_cast<cudaStream_t>(stream)>>>(p);
     }
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
@@ -575,6 +646,22 @@ int select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int 
         est_us[0] = (float)sk;
         est_us[1] = tc ? (float)best : -1.0f;
     }
+    return GQA_OK;
+}
+
+// gqa_decode_auto's choice between stream-K (0) and one CTA per (request, KV
+// head) (1).  The second runs on the tensor-core kernel only, so a shape that
+// kernel does not take (a page size its TMA boxes cannot tile, too many rows
+// for a tensor map, a small group) stays on stream-K.
+static int auto_splits(int B, int Hq, int Hkv, int D, int block_size, bool paged, int num_blocks,
+                       const int32_t *seq_lens_host, int sms, int &ns)
+{
+    ns = 0;
+    int rc = select_schedule(B, Hq, Hkv, D, seq_lens_host, sms, 1, &ns, nullptr);
+    if (rc)
+        return rc;
+    if (ns && !tc_applicable(false, B, Hkv, D, block_size, paged, num_blocks, Hq / Hkv))
+        ns = 0;
     return GQA_OK;
 }
 
@@ -686,11 +773,83 @@ int gqa_decode_auto(const void *q, const void *k_cache, const void *v_cache,
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return GQA_ERR_CUDA;
     int ns = 0;
-    if ((rc = select_schedule(B, Hq, Hkv, D, seq_lens_host, sms, 1, &ns, nullptr)))
+    if ((rc = auto_splits(B, Hq, Hkv, D, block_size, block_table != nullptr, num_blocks,
+                          seq_lens_host, sms, ns)))
         return rc;
     return run_decode(false, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, out,
                       nullptr, nullptr, nullptr, B, Hq, Hkv, D, block_size, scale,
                       max_blocks_per_seq, num_blocks, workspace, workspace_bytes, stream, ns);
+}
+
+int gqa_decode_plan(int B, int Hq, int Hkv, int D, int block_size, int paged, int num_blocks,
+                    int qlen, int kv_fp8, int num_splits, const int32_t *seq_lens_host, int device,
+                    gqa_plan *plan)
+{
+    if (!plan || num_splits < -1)
+        return GQA_ERR_INVALID_ARG;
+    std::memset(plan, 0, sizeof *plan);
+    int rc = check_shape(B, Hq, Hkv, D, block_size, paged ? &B : nullptr, 1,
+                         paged ? num_blocks : 0, 1.0f);
+    if (rc)
+        return rc;
+    if (paged && num_blocks < 0)
+        return GQA_ERR_INVALID_ARG;
+    if (B > 0 && num_splits == -1 && (!seq_lens_host || device < 0))
+        return GQA_ERR_INVALID_ARG;
+    if (seq_lens_host)
+        for (int b = 0; b < B; ++b)
+            if (seq_lens_host[b] < 0)
+                return GQA_ERR_INVALID_ARG;
+    if (kv_fp8 && (qlen != 1))
+        return GQA_ERR_UNSUPPORTED;
+    int ns = num_splits;
+    if (ns == -1 && B > 0) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+            return GQA_ERR_CUDA;
+        if ((rc = auto_splits(B, Hq, Hkv, D, block_size, paged != 0, num_blocks, seq_lens_host, sms,
+                              ns)))
+            return rc;
+    }
+    ns = ns < 0 ? 0 : ns;
+    plan->num_splits = ns;
+    plan->tiles = -1;
+    plan->grid = -1;
+    if (B == 0) {  // nothing is launched
+        plan->grid = 0;
+        plan->tiles = 0;
+        return GQA_OK;
+    }
+    Plan pl;
+    if ((rc = make_plan(false, B, Hq, Hkv, D, block_size, paged != 0, num_blocks, qlen,
+                        kv_fp8 != 0, ns, device, pl)))
+        return rc;
+    plan->kernel = pl.use_tc ? GQA_KERNEL_TENSOR_CORE : GQA_KERNEL_CUDA_CORE;
+    plan->heads_per_pass = pl.nv;
+    plan->head_chunks = pl.hch;
+    plan->grid = (int)pl.grid;
+    plan->threads_per_cta = pl.threads;
+    plan->cooperative = pl.use_tc && ns == 0;
+    plan->merge_launch = ns > 1;
+    plan->tile_tokens = pl.tile_tokens;
+    plan->ring_stages = pl.stages;
+    plan->box_rows = pl.box_rows;
+    plan->smem_bytes = pl.smem;
+    plan->workspace_bytes = device >= 0 ? pl.w.total : 0;
+    if (seq_lens_host) {
+        long long tiles = 0;
+        for (int b = 0; b < B; ++b)
+            tiles += ((long long)seq_lens_host[b] + pl.tile_tokens - 1) / pl.tile_tokens;
+        plan->tiles = tiles * Hkv * pl.hch;
+    }
+    if (pl.use_tc)
+        std::snprintf(plan->kernel_name, sizeof plan->kernel_name,
+                      "gqa_decode_tc_kernel<NV=%d,MQ=%d,D=%d,F8=%d>", pl.nv, pl.mq ? 1 : 0, D,
+                      kv_fp8 ? 1 : 0);
+    else
+        std::snprintf(plan->kernel_name, sizeof plan->kernel_name,
+                      "gqa_decode_simt_kernel<D=%d,GC=%d,ST=0,F8=%d>", D, pl.nv, kv_fp8 ? 1 : 0);
+    return GQA_OK;
 }
 
 int gqa_decode_multi(const void *q, const void *k_cache, const void *v_cache,

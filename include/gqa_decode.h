@@ -197,6 +197,50 @@ GQA_API int gqa_decode_auto(const void *q, const void *k_cache, const void *v_ca
                             void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * What a call would launch, reported without launching anything: the kernel
+ * and its template parameters, the schedule, the grid and the LeanTile count
+ * (the work units of LeanAttention decode tiles digest, section
+ * "Hardware-sized work units").  The library's own launch path decides from the
+ * same host-side plan, so the report is what runs.
+ *   paged          1: a paged pool of num_blocks blocks (block_table non-NULL);
+ *                  0: a contiguous cache (block_size = per-request capacity)
+ *   qlen           query tokens per request (1: gqa_decode; > 1: gqa_decode_multi)
+ *   kv_fp8         1: an FP8 E4M3 cache (gqa_decode_fp8; qlen must be 1)
+ *   num_splits     -1: the choice gqa_decode_auto makes (needs seq_lens_host and
+ *                  a device); 0: gqa_decode (stream-K); n > 0: gqa_decode_fixed_split
+ *   seq_lens_host  HOST int32 [B] or NULL; with it, plan->tiles is filled in
+ *   device         CUDA device for the grid and workspace size; < 0: no device
+ *                  query (grid = -1 for stream-K, workspace_bytes = 0)
+ *   plan           HOST, written on GQA_OK
+ * Errors: those gqa_decode would return for the shape (GQA_ERR_UNSUPPORTED for a
+ * schedule or format the shape cannot run), GQA_ERR_INVALID_ARG for a NULL plan,
+ * num_splits < -1, a negative length, or num_splits = -1 without lengths or a
+ * device.  B = 0 gives kernel = 0 (nothing is launched).
+ */
+#define GQA_KERNEL_TENSOR_CORE 1  /* gqa_decode_tc_kernel: tcgen05 MMAs, TMA tiles */
+#define GQA_KERNEL_CUDA_CORE 2    /* gqa_decode_simt_kernel: packed FMAs on CUDA cores */
+typedef struct gqa_plan {
+    int kernel;              /* GQA_KERNEL_*, 0 when nothing is launched */
+    int heads_per_pass;      /* query rows one pass carries (tensor cores: 4, 8, 16) */
+    int head_chunks;         /* passes per KV head */
+    int num_splits;          /* 0: stream-K; n > 0: fixed split into n chunks */
+    int grid;                /* CTAs of the decode kernel (-1: no device given) */
+    int threads_per_cta;
+    int cooperative;         /* 1: cooperative launch (every CTA resident) */
+    int merge_launch;        /* 1: a second kernel merges the fixed-split chunks */
+    int tile_tokens;         /* tokens per LeanTile */
+    int ring_stages;         /* shared-memory ring slots per K (and per V) stream */
+    int box_rows;            /* tensor cores: tokens per TMA box (0 on CUDA cores) */
+    long long tiles;         /* LeanTiles of the step (-1 without seq_lens_host) */
+    size_t smem_bytes;       /* dynamic shared memory per CTA */
+    size_t workspace_bytes;  /* workspace the call needs on `device` */
+    char kernel_name[64];    /* e.g. "gqa_decode_tc_kernel<NV=4,MQ=0,D=128,F8=0>" */
+} gqa_plan;
+GQA_API int gqa_decode_plan(int B, int Hq, int Hkv, int D, int block_size, int paged,
+                            int num_blocks, int qlen, int kv_fp8, int num_splits,
+                            const int32_t *seq_lens_host, int device, gqa_plan *plan);
+
+/*
  * Several query tokens per request: the verification pass of speculative
  * decoding, where the large model scores the qlen drafted positions in one pass
  * (Inference optimization: KV cache, MQA/GQA, batching..., section 5

@@ -1,5 +1,5 @@
-"""CPU checks of host-side helpers: FP8 cache preparation, the bench's kernel
-mapping and traffic-record keying, workspace sizes."""
+"""CPU checks of host-side helpers: FP8 cache preparation, the dispatch report
+(gqa_decode_plan) and traffic-record keying, workspace sizes."""
 import os
 import sys
 
@@ -31,27 +31,54 @@ def test_fp8_caches_range_scale_and_poison():
     assert torch.all(err <= p.k_cache.float()[fin].abs() * 2 ** -4 + ks * 2 ** -9)
 
 
-def test_bench_kernel_mapping():
+def _plan(B, Hq, Hkv, D, bs=None, paged=False, nb=0, **kw):
+    return gq.decode_plan(B, Hq, Hkv, D, bs if bs is not None else 4096, paged, nb, device=-1,
+                          **kw)
+
+
+def test_plan_reports_the_dispatch():
+    """gqa_decode_plan (no device query) reports the kernel the launch path takes."""
+    tc, cc = gq.KERNEL_TENSOR_CORE, gq.KERNEL_CUDA_CORE
+    p = _plan(16, 32, 8, 128, seq_lens_host=[8192] * 16)
+    assert p["kernel"] == tc and p["heads_per_pass"] == 4 and p["head_chunks"] == 1
+    assert p["kernel_name"] == "gqa_decode_tc_kernel<NV=4,MQ=0,D=128,F8=0>"
+    assert p["cooperative"] == 1 and p["tile_tokens"] == 128 and p["tiles"] == 16 * 8 * 64
+    assert _plan(1, 32, 32, 128)["kernel"] == cc                      # G = 1
+    d64 = _plan(1, 32, 8, 64)
+    assert d64["kernel"] == tc and d64["ring_stages"] == 5            # D = 64, deep ring
+    assert _plan(1, 32, 8, 256)["kernel"] == cc                       # D = 256
+    assert _plan(1, 32, 8, 128, bs=48, paged=True, nb=10)["kernel"] == cc  # page size
+    assert _plan(1, 32, 8, 128, bs=64, paged=True, nb=10)["box_rows"] == 64
+    f8 = _plan(1, 32, 8, 128, kv_fp8=True)
+    assert f8["kernel"] == tc and f8["kernel_name"].endswith("F8=1>")
+    assert _plan(1, 32, 8, 64, kv_fp8=True)["kernel"] == cc           # FP8 at D = 64
+    mqa = _plan(8, 64, 1, 128, seq_lens_host=[100] * 8)
+    assert mqa["heads_per_pass"] == 16 and mqa["head_chunks"] == 4 and mqa["tiles"] == 8 * 4
+    assert _plan(2, 32, 8, 128, qlen=4)["kernel_name"].startswith("gqa_decode_tc_kernel<NV=16,MQ=1")
+    fx = _plan(2, 32, 8, 128, num_splits=4)
+    assert fx["num_splits"] == 4 and fx["grid"] == 2 * 8 * 4 and fx["merge_launch"] == 1
+    assert _plan(0, 32, 8, 128)["kernel"] == 0                        # nothing launched
+    # a traffic record is keyed to the sources of the kernel the plan names
     import bench
-    assert bench.kernel_for(workloads.make_problem("a", 1, 32, 8, 128, [10], seed=1)).startswith(
-        "gqa_decode_tc_kernel")
-    assert bench.kernel_for(workloads.make_problem("b", 1, 32, 32, 128, [10], seed=1)) == \
-        "gqa_decode_simt_kernel"                     # G = 1
-    assert bench.kernel_for(workloads.make_problem("c", 1, 32, 8, 64, [10], seed=1)).startswith(
-        "gqa_decode_tc_kernel")                      # D = 64
-    assert bench.kernel_for(workloads.make_problem("c", 1, 32, 8, 256, [10], seed=1)) == \
-        "gqa_decode_simt_kernel"                     # D = 256
-    assert bench.kernel_for(workloads.make_problem("d", 1, 32, 8, 128, [10], seed=1,
-                                                   block_size=48)) == "gqa_decode_simt_kernel"
-    p = workloads.make_problem("e", 1, 32, 8, 128, [10], seed=1)
-    p.meta["kv_elem_bytes"] = 1
-    assert bench.kernel_for(p) == "gqa_decode_tc_kernel<4> (FP8 E4M3 cache)"
-    p = workloads.make_problem("f", 1, 32, 8, 64, [10], seed=1)
-    p.meta["kv_elem_bytes"] = 1
-    assert bench.kernel_for(p) == "gqa_decode_simt_kernel (FP8 E4M3 cache)"   # D = 64
-    # traffic records are keyed to each kernel's own sources
-    assert bench.kernel_source_hash("gqa_decode_tc_kernel<4>") != \
-        bench.kernel_source_hash("gqa_decode_simt_kernel")
+    assert bench.kernel_source_hash(p["kernel_name"]) != \
+        bench.kernel_source_hash(_plan(1, 32, 32, 128)["kernel_name"])
+
+
+def test_plan_errors():
+    with pytest.raises(gq.GqaError) as e:
+        _plan(2, 32, 8, 256, num_splits=2)        # fixed split needs the tensor-core kernel
+    assert e.value.code == 2
+    with pytest.raises(gq.GqaError) as e:
+        _plan(2, 32, 8, 128, num_splits=-1)       # auto needs lengths and a device
+    assert e.value.code == 1
+    with pytest.raises(gq.GqaError) as e:
+        _plan(2, 32, 8, 128, qlen=2, kv_fp8=True)
+    assert e.value.code == 2
+    with pytest.raises(gq.GqaError) as e:
+        _plan(2, 30, 8, 128)                      # Hq % Hkv != 0
+    assert e.value.code == 1
+    with pytest.raises(gq.GqaError):
+        _plan(1, 32, 8, 128, seq_lens_host=[-1])
 
 
 def test_fixed_split_workspace_grows_with_splits():
