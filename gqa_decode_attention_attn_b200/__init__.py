@@ -34,7 +34,8 @@ EXPORTED = ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states", "gqa
             "gqa_status", "gqa_decode_host_buffer_bytes", "gqa_decode_host", "gqa_error_string",
             "gqa_decode_noalloc", "gqa_decode_fixed_split_workspace_size",
             "gqa_decode_fixed_split", "gqa_select_schedule", "gqa_decode_auto",
-            "gqa_decode_multi", "gqa_decode_fp8", "gqa_decode_timeline", "gqa_decode_plan")
+            "gqa_decode_multi", "gqa_decode_fp8", "gqa_decode_timeline", "gqa_decode_plan",
+            "gqa_set_wait_limit")
 GQA_ERR_SCRATCH_LIMIT = 6
 TIMELINE_COLS = 8  # values per CTA row of gqa_decode_timeline
 KERNEL_TENSOR_CORE = 1
@@ -89,6 +90,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                         ctypes.POINTER(I), P, SZ, P]
     lib.gqa_decode_plan.argtypes = [I, I, I, I, I, I, I, I, I, I, P, I, ctypes.POINTER(_Plan)]
     lib.gqa_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P]
+    lib.gqa_set_wait_limit.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong)]
     lib.gqa_error_string.argtypes = [I]
     lib.gqa_error_string.restype = ctypes.c_char_p
     for name in ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states",
@@ -96,10 +98,18 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                  "gqa_decode_fixed_split_workspace_size", "gqa_decode_fixed_split",
                  "gqa_select_schedule", "gqa_decode_auto", "gqa_decode_multi",
                  "gqa_decode_fp8", "gqa_decode_plan", "gqa_decode_noalloc",
-                 "gqa_decode_timeline"):
+                 "gqa_decode_timeline", "gqa_set_wait_limit"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
+
+
+def set_wait_limit(ns: int) -> int:
+    """Limit of each in-kernel wait for progress, for launches from now on (0: the
+    default 1.5 s); returns the previous limit in ns (gqa_set_wait_limit)."""
+    prev = ctypes.c_ulonglong(0)
+    _check("gqa_set_wait_limit", load_library().gqa_set_wait_limit(int(ns), ctypes.byref(prev)))
+    return prev.value
 
 
 def error_string(code: int) -> str:

@@ -10,6 +10,7 @@
 #include <queue>
 #include <vector>
 #include <algorithm>
+#include <atomic>
 
 #include "decode_simt.cuh"
 #include "decode_tc.cuh"
@@ -40,6 +41,10 @@ constexpr double SCHED_MERGE_US = 3.0;
 constexpr double SCHED_SPLIT_MERGE_US = 5.0;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Limit of each in-kernel wait for progress, for launches from now on
+// (gqa_set_wait_limit).
+std::atomic<unsigned long long> g_wait_ns{WAIT_LIMIT_NS};
 
 // Query heads per chunk for the CUDA-core kernel: the next power of two >= G,
 // capped at 8 (larger groups run as several chunks).
@@ -501,6 +506,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
     p.qscale = scale * LOG2E * (fp8 ? k_scale : 1.0f);
     p.vscale = fp8 ? v_scale : 1.0f;
     p.timeline = timeline;
+    p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
     // Magic number for t / block_size (t < 2^31): see page_of().
     {
         int l = 0;
@@ -991,6 +997,16 @@ int gqa_decode_host(const void *q, const void *k_cache, const void *v_cache,
     if (cudaMemcpyAsync(out, dbuf + h.out, qbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return GQA_ERR_CUDA;
     return cudaStreamSynchronize(s) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+int gqa_set_wait_limit(unsigned long long ns, unsigned long long *previous)
+{
+    if (ns != 0 && (ns < 1000ull || ns > 10000000000ull))
+        return GQA_ERR_INVALID_ARG;
+    const unsigned long long old = g_wait_ns.exchange(ns ? ns : WAIT_LIMIT_NS);
+    if (previous)
+        *previous = old;
+    return GQA_OK;
 }
 
 const char *gqa_error_string(int code)

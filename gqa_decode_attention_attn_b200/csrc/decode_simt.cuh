@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(SimtCfg<D, GC, F8>::THREADS, 1)
                 it.next(prefix, B, p.Hkv, p.hch);
             const int s = k % C::STAGES;
             const uint32_t ph = (uint32_t)((k / C::STAGES) & 1);
-            if (k >= C::STAGES && !bounded_wait(&empty[s], ph ^ 1u, abort_flag, p.status))
+            if (k >= C::STAGES && !bounded_wait(&empty[s], ph ^ 1u, abort_flag, p))
                 break;
             if (it.b != cur_b) {
                 cur_b = it.b;
@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(SimtCfg<D, GC, F8>::THREADS, 1)
 
         const int s = k % C::STAGES;
         const uint32_t ph = (uint32_t)((k / C::STAGES) & 1);
-        const bool ready = bounded_wait(&full[s], ph, abort_flag, p.status);
+        const bool ready = bounded_wait(&full[s], ph, abort_flag, p);
         if (!ready) {
             poisoned = true;
         } else {

@@ -116,6 +116,16 @@ __device__ __forceinline__ void split_e4m3(float x, uint32_t &hi, uint32_t &lo)
     lo = to_e4m3((x - e4m3_value(hi)) * 16.f);
 }
 
+// x as three E4M3 terms, x ~ t1 + t2 / 16 + t3 / 256 (about 12 significant bits;
+// each term carries the remainder of the ones before it, scaled by 16).
+__device__ __forceinline__ void split3_e4m3(float x, uint32_t &t1, uint32_t &t2, uint32_t &t3)
+{
+    t1 = to_e4m3(x);
+    const float r1 = (x - e4m3_value(t1)) * 16.f;
+    t2 = to_e4m3(r1);
+    t3 = to_e4m3((r1 - e4m3_value(t2)) * 16.f);
+}
+
 // Max or sum of NV per-lane values across the 32 lanes of a warp, transposed so
 // that lane l ends with the result for index l / (32 / NV) (NV <= 32).
 template <int NV, bool MAX>
@@ -152,9 +162,12 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[NV], int lane)
 // 64..127 read from a block of zeros (written once, never loaded), so the O rows
 // 64..127 are zero and are not read back.
 // F8: the cache holds FP8 E4M3 (D = 128): the MMAs run kind::f8f6f4 (K = 32) on
-// the cache bytes as loaded; Q and P enter as two E4M3 terms each, t1 + t2 / 16,
-// side by side in N = 32 (one term per 16 columns), and the softmax and the fold
-// add the two column blocks back.  Scores are scaled by p.qscale (which holds the
+// the cache bytes as loaded.  Q enters as two E4M3 terms, t1 + t2 / 16 (exact for
+// bf16 q after the row's power-of-two scaling), side by side in N = 32 (one term
+// per 16 columns); P as three, t1 + t2 / 16 + t3 / 256, in N = 48: two terms
+// leave the weights of the keys that dominate a row 8 significant bits, whose
+// error alone can move a bf16 output by one unit.  The softmax and the fold add
+// the column blocks back.  Scores are scaled by p.qscale (which holds the
 // K scale) and by the power of two that brought each Q row into E4M3's range.
 template <int NV, bool MQ, int DH = 128, bool F8 = false>
 __global__ void __launch_bounds__(TcCfg::THREADS, 1)
@@ -170,8 +183,11 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     constexpr int KSTEP = F8 ? 32 : 16;             // MMA K per instruction
     // FP8 P: per 8-token group, two 128-byte core matrices along N (16 E4M3 heads
     // per 16-byte row: term 1, then term 2).
-    constexpr int P8_LBO = (C::NO / 16) * 128;
-    static_assert(OC + 2 * C::NO <= C::TMEM_COLS, "tensor memory columns");
+    constexpr int NO = F8 ? 3 * NP : C::NO;         // BMM2 columns: the P terms side by side
+    constexpr int P8_LBO = 3 * 128;                 // FP8 P: three core matrices per 8 tokens
+    constexpr int TMEM_COLS = F8 ? 256 : C::TMEM_COLS;
+    static_assert(OC + 2 * NO <= TMEM_COLS, "tensor memory columns");
+    static_assert(!F8 || (T / 8) * P8_LBO <= C::PBUF_BYTES, "FP8 P buffer");
     static_assert(D == 64 || D == 128, "head dimension");
     constexpr int SLOT = slot_floats(NV, D);
     constexpr int LPH = 32 / NV;  // lanes per head after a transposed warp reduction
@@ -230,7 +246,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
     }
     if constexpr (L::NEED_ZERO) {
@@ -335,7 +351,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 it.next(prefix, B, p.Hkv, p.hch);
             const int s = k % S;
             const uint32_t ph = (uint32_t)((k / S) & 1);
-            if (k >= S && !bounded_wait(&emptyb[s], ph ^ 1u, abort_flag, p.status))
+            if (k >= S && !bounded_wait(&emptyb[s], ph ^ 1u, abort_flag, p))
                 break;
             if (it.b != cur_b) {
                 cur_b = it.b;
@@ -409,9 +425,9 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                         ++piece1;
                     }
                     const int s = k % S, b = k & 1, qb = (piece1 - 1) & 1;
-                    ok = bounded_wait(&k_full[s], (uint32_t)((k / S) & 1), abort_flag, p.status) &&
-                         (k < 2 || bounded_wait(&s_free[b], (uint32_t)(((k - 2) >> 1) & 1), abort_flag, p.status)) &&
-                         bounded_wait(&q_full[qb], (uint32_t)(((piece1 - 1) >> 1) & 1), abort_flag, p.status);
+                    ok = bounded_wait(&k_full[s], (uint32_t)((k / S) & 1), abort_flag, p) &&
+                         (k < 2 || bounded_wait(&s_free[b], (uint32_t)(((k - 2) >> 1) & 1), abort_flag, p)) &&
+                         bounded_wait(&q_full[qb], (uint32_t)(((piece1 - 1) >> 1) & 1), abort_flag, p);
                     if (!ok)
                         break;
                     tc_fence_after_sync();
@@ -438,7 +454,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 // o_full) when the softmax moves the reference (ctl flag of the tile)
                 // or when a piece ends; the next tile opens the other buffer afresh.
                 // Closes are counted by `u`: use u lives in buffer u & 1.
-                const uint32_t idesc2 = F8 ? umma_idesc_e4m3(128, C::NO, 1, 1) : umma_idesc_bf16(128, C::NO, 1, 1);
+                const uint32_t idesc2 = F8 ? umma_idesc_e4m3(128, NO, 1, 1) : umma_idesc_bf16(128, NO, 1, 1);
                 TileIter itp;
                 itp.init(start, prefix, B, units, p.hch);
                 int64_t segp = itp.seg0;
@@ -446,7 +462,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 bool fresh = true;
                 for (int k = 0; k < ntiles && ok; ++k) {
                     const int s = k % S, b = k & 1;
-                    if (!bounded_wait(&p_full[b], (uint32_t)((k >> 1) & 1), abort_flag, p.status)) {
+                    if (!bounded_wait(&p_full[b], (uint32_t)((k >> 1) & 1), abort_flag, p)) {
                         ok = false;
                         break;
                     }
@@ -456,8 +472,8 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                         fresh = true;
                     }
                     ok = (!fresh || u < 2 ||
-                          bounded_wait(&o_free[u & 1], (uint32_t)(((u - 2) >> 1) & 1), abort_flag, p.status)) &&
-                         bounded_wait(&v_full[s], (uint32_t)((k / S) & 1), abort_flag, p.status);
+                          bounded_wait(&o_free[u & 1], (uint32_t)(((u - 2) >> 1) & 1), abort_flag, p)) &&
+                         bounded_wait(&v_full[s], (uint32_t)((k / S) & 1), abort_flag, p);
                     if (!ok)
                         break;
                     // Does the piece end with tile k?  (itp runs one tile ahead.)
@@ -477,14 +493,14 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                     for (int kk = 0; kk < T / KSTEP; ++kk) {
                         if constexpr (F8) {
                             // 32 tokens per instruction: 4 KB of V rows, four 8-token groups of P.
-                            umma_e4m3(tbase + (uint32_t)(OC + (u & 1) * C::NO),
+                            umma_e4m3(tbase + (uint32_t)(OC + (u & 1) * NO),
                                       umma_smem_desc(va + (uint32_t)(kk * 4096), C::BOX_BYTES, 1024,
                                                      SMEM_LAYOUT_SW128),
                                       umma_smem_desc(pa + (uint32_t)(4 * kk * P8_LBO), P8_LBO, 128,
                                                      SMEM_LAYOUT_NONE),
                                       idesc2, kk > 0 || !fresh);
                         } else {
-                            umma_bf16(tbase + (uint32_t)(OC + (u & 1) * C::NO),
+                            umma_bf16(tbase + (uint32_t)(OC + (u & 1) * NO),
                                       umma_smem_desc(va + (uint32_t)(kk * 2048), vlbo, 1024, SMEM_LAYOUT_SW128),
                                       umma_smem_desc(pa + (uint32_t)(2 * kk * C::P_LBO), C::P_LBO, 128, SMEM_LAYOUT_NONE),
                                       idesc2, kk > 0 || !fresh);
@@ -592,17 +608,23 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         auto fold = [&](const float (&w)[NV]) {
             const int bc = u & 1;
             float o[NV];
-            if (ok && bounded_wait(&o_full[bc], (uint32_t)((u >> 1) & 1), abort_flag, p.status)) {
+            if (ok && bounded_wait(&o_full[bc], (uint32_t)((u >> 1) & 1), abort_flag, p)) {
                 float olo[NV];
                 tc_fence_after_sync();
-                tmem_load<NV>(tlane + (uint32_t)(OC + bc * C::NO), o);
-                tmem_load<NV>(tlane + (uint32_t)(OC + bc * C::NO + NP), olo);
-                tc_fence_before_sync();
+                tmem_load<NV>(tlane + (uint32_t)(OC + bc * NO), o);
+                tmem_load<NV>(tlane + (uint32_t)(OC + bc * NO + NP), olo);
+                if constexpr (F8) {
+                    // P terms 2 and 3 carry x16 and x256.
+                    float o3[NV];
+                    tmem_load<NV>(tlane + (uint32_t)(OC + bc * NO + 2 * NP), o3);
 #pragma unroll
-                for (int g = 0; g < NV; ++g) {
-                    if constexpr (F8)
-                        o[g] = fmaf(olo[g], 1.f / 16.f, o[g]);  // the second P term carries x16
-                    else
+                    for (int g = 0; g < NV; ++g)
+                        o[g] = fmaf(fmaf(o3[g], 1.f / 16.f, olo[g]), 1.f / 16.f, o[g]);
+                }
+                tc_fence_before_sync();
+                if constexpr (!F8) {
+#pragma unroll
+                    for (int g = 0; g < NV; ++g)
                         o[g] += olo[g];
                 }
             } else {
@@ -749,8 +771,8 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             const int s = k % S, b = k & 1;
             float sc[NV];
             int n = 0;
-            if (ok && bounded_wait(&v_full[s], (uint32_t)((k / S) & 1), abort_flag, p.status) &&
-                bounded_wait(&s_full[b], (uint32_t)((k >> 1) & 1), abort_flag, p.status)) {
+            if (ok && bounded_wait(&v_full[s], (uint32_t)((k / S) & 1), abort_flag, p) &&
+                bounded_wait(&s_full[b], (uint32_t)((k >> 1) & 1), abort_flag, p)) {
                 n = stage_n[s];
                 poisoned |= stage_bad[s] != 0;
                 tc_fence_after_sync();
@@ -830,7 +852,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 }
             }
             // This P buffer was last read by BMM2 two tiles ago.
-            if (k >= 2 && ok && !bounded_wait(&p_free[b], (uint32_t)(((k - 2) >> 1) & 1), abort_flag, p.status)) {
+            if (k >= 2 && ok && !bounded_wait(&p_free[b], (uint32_t)(((k - 2) >> 1) & 1), abort_flag, p)) {
                 ok = false;
                 poisoned = true;
             }
@@ -844,30 +866,34 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             // 0..NP-1, lo heads in NP..2NP-1) in the no-swizzle MN-major layout:
             // token ti's 8-head groups are 16-byte rows of 8x8 core matrices.
             if constexpr (F8) {
-                // P = t1 + t2 / 16, both E4M3, as one N = 32 operand (term 1 of the
-                // heads in bytes 0..NP-1 of the token's 16-byte row of the first core
-                // matrix, term 2 in the second), no-swizzle MN-major.
+                // P = t1 + t2 / 16 + t3 / 256, all E4M3, as one N = 48 operand (term
+                // i of the heads in bytes 0..NP-1 of the token's 16-byte row of core
+                // matrix i), no-swizzle MN-major.
                 unsigned char *pd8 = pbuf + b * C::PBUF_BYTES + (ti >> 3) * P8_LBO + (ti & 7) * 16;
-                uint32_t w1[(NV + 3) / 4], w2[(NV + 3) / 4];
+                uint32_t w1[(NV + 3) / 4], w2[(NV + 3) / 4], w3[(NV + 3) / 4];
 #pragma unroll
                 for (int j = 0; j < (NV + 3) / 4; ++j)
-                    w1[j] = w2[j] = 0u;
+                    w1[j] = w2[j] = w3[j] = 0u;
 #pragma unroll
                 for (int g = 0; g < NV; ++g) {
-                    uint32_t hi, lo;
-                    split_e4m3(pr[g], hi, lo);
-                    w1[g >> 2] |= hi << (8 * (g & 3));
-                    w2[g >> 2] |= lo << (8 * (g & 3));
+                    uint32_t t1, t2, t3;
+                    split3_e4m3(pr[g], t1, t2, t3);
+                    w1[g >> 2] |= t1 << (8 * (g & 3));
+                    w2[g >> 2] |= t2 << (8 * (g & 3));
+                    w3[g >> 2] |= t3 << (8 * (g & 3));
                 }
                 if constexpr (NV == 4) {
                     *reinterpret_cast<uint32_t *>(pd8) = w1[0];
                     *reinterpret_cast<uint32_t *>(pd8 + 128) = w2[0];
+                    *reinterpret_cast<uint32_t *>(pd8 + 256) = w3[0];
                 } else if constexpr (NV == 8) {
                     *reinterpret_cast<uint2 *>(pd8) = make_uint2(w1[0], w1[1]);
                     *reinterpret_cast<uint2 *>(pd8 + 128) = make_uint2(w2[0], w2[1]);
+                    *reinterpret_cast<uint2 *>(pd8 + 256) = make_uint2(w3[0], w3[1]);
                 } else {
                     *reinterpret_cast<uint4 *>(pd8) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
                     *reinterpret_cast<uint4 *>(pd8 + 128) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+                    *reinterpret_cast<uint4 *>(pd8 + 256) = make_uint4(w3[0], w3[1], w3[2], w3[3]);
                 }
             } else {
                 unsigned char *pd = pbuf + b * C::PBUF_BYTES + (ti >> 3) * C::P_LBO + (ti & 7) * 16;
@@ -949,7 +975,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after_sync();
-        tmem_dealloc(tbase, C::TMEM_COLS);
+        tmem_dealloc(tbase, TMEM_COLS);
     }
     if (p.timeline && tid == 0) {
         unsigned sm;

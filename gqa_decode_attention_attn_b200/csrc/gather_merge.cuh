@@ -16,7 +16,7 @@
 //
 // counters[vseg]: bits 0..15 count published pieces, bits 16..31 count finished
 // slices; the owner that finishes the last slice resets the word to zero.  Waits
-// are bounded (WAIT_LIMIT_NS): on expiry the kernel's status gets DEV_TIMEOUT and
+// are bounded (Params::wait_ns): on expiry the kernel's status gets DEV_TIMEOUT and
 // the slice is written as NaN.
 #pragma once
 
@@ -73,7 +73,7 @@ __device__ __forceinline__ void merge_segment_gather(const Params &p, int64_t c,
         bool ok = true;
         const uint64_t t0 = global_timer_ns();
         while ((ld_acquire(&p.counters[vseg]) & 0xFFFF) < no) {
-            if (*abort_flag || global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+            if (*abort_flag || global_timer_ns() - t0 > p.wait_ns) {
                 ok = false;
                 break;
             }

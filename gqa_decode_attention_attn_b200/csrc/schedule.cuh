@@ -26,7 +26,10 @@ constexpr unsigned DEV_BAD_BLOCK = 1u;
 constexpr unsigned DEV_BAD_LENGTH = 2u;
 constexpr unsigned DEV_TIMEOUT = 4u;
 
-// Upper bound on any single in-kernel wait; a healthy wait lasts microseconds.
+// Default upper bound on any single in-kernel wait for progress (a pipeline stage,
+// another CTA's partial state); a healthy wait lasts microseconds.  A launch may
+// carry a shorter one (Params::wait_ns).  The waits at exit for the CTA's own
+// copies and tensor-core work in flight always use this default.
 constexpr uint64_t WAIT_LIMIT_NS = 1500000000ull;
 
 // Per-CTA timeline row (Params::timeline): start ns, end ns, SM id, tiles, then the
@@ -61,6 +64,7 @@ struct Params {
     float qscale;                 // scale * log2(e) (* k_scale for FP8): scores in log2 units
     float vscale;                 // FP8 cache: v_scale, applied to the output (1 for bf16)
     unsigned long long *timeline; // optional [grid][TL_COLS], see TL_COLS
+    uint64_t wait_ns;             // limit of each wait for progress (see WAIT_LIMIT_NS)
 };
 
 // floor(t / block_size) for 0 <= t < 2^31 without a divide: with l = ceil(log2 bs)
@@ -207,9 +211,10 @@ __device__ __forceinline__ int64_t out_row(const Params &p, int b, int kvh, int 
     return ((int64_t)b * p.qlen + i) * p.Hq + (int64_t)kvh * p.G + h;
 }
 
-// Bounded wait on an mbarrier phase.  On timeout: status bit, CTA abort flag.
+// Bounded wait on an mbarrier phase (at most p.wait_ns).  On timeout: status bit,
+// CTA abort flag.
 __device__ __forceinline__ bool bounded_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                             unsigned *status)
+                                             const Params &p)
 {
     if (mbar_try_wait(bar, parity))
         return true;
@@ -219,8 +224,8 @@ __device__ __forceinline__ bool bounded_wait(uint64_t *bar, uint32_t parity, vol
     while (!mbar_try_wait(bar, parity)) {
         if (*abort_flag)
             return false;
-        if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
-            atomicOr(status, DEV_TIMEOUT);
+        if (global_timer_ns() - t0 > p.wait_ns) {
+            atomicOr(p.status, DEV_TIMEOUT);
             *abort_flag = 1;
             return false;
         }

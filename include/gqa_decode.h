@@ -266,9 +266,14 @@ GQA_API int gqa_decode_multi(const void *q, const void *k_cache, const void *v_c
  * long-context inference, list of techniques): k_cache and v_cache hold one byte
  * per element in the bf16 caches' layouts; element values are e4m3(byte) * k_scale
  * and e4m3(byte) * v_scale (one scale per tensor, > 0).  q and out stay bf16.  A
- * decode step reads half the bytes.  Runs on the CUDA-core kernel, the E4M3 bytes
- * widened exactly in registers (k_scale folded into q, v_scale applied to the
- * output).  Workspace: gqa_decode_workspace_size.  Errors as gqa_decode.
+ * decode step reads half the bytes.  At D = 128 with at least 4 query heads per
+ * KV head (and the tensor-core kernel's page sizes, B <= 1024) it runs on the
+ * tensor cores: kind::f8f6f4 MMAs read the cache bytes as loaded; q enters as
+ * two E4M3 terms (t1 + t2 / 16, each q row first scaled by a power of two) and
+ * the softmax weights as three (t1 + t2 / 16 + t3 / 256); accumulation in fp32.  Other shapes run on the
+ * CUDA-core kernel, the E4M3 bytes widened exactly in registers.  k_scale is
+ * folded into the scores, v_scale applied to the output.  Workspace:
+ * gqa_decode_workspace_size.  Errors as gqa_decode.
  */
 GQA_API int gqa_decode_fp8(const void *q, const void *k_cache, const void *v_cache, float k_scale,
                            float v_scale, const int32_t *block_table, const int32_t *seq_lens,
@@ -357,6 +362,22 @@ GQA_API int gqa_decode_noalloc(const void *q, const void *k_cache, const void *v
                                const int32_t *block_table, const int32_t *seq_lens, void *out,
                                int B, int Hq, int Hkv, int D, int block_size, float scale,
                                int max_blocks_per_seq, int num_blocks, void *stream);
+
+/*
+ * The longest any wait inside the decode kernels for progress may last -- a
+ * pipeline stage, or the partial states of the other CTAs sharing a split
+ * (request, KV head) -- before the kernel gives up on it: it then sets
+ * GQA_DEV_TIMEOUT, stops streaming, writes NaN to the rows it could not finish
+ * and returns (the LeanAttention decode tiles digest's split pieces are merged by
+ * CTAs that wait for one another; a wait that cannot end must not hang the GPU).
+ * Healthy waits last microseconds; the default limit is 1.5 s.  The setting is
+ * process-wide and applies to calls launched after this returns.  ns = 0
+ * restores the default; otherwise 1e3 <= ns <= 1e10, else GQA_ERR_INVALID_ARG.
+ * *previous (HOST, may be NULL) receives the limit in force before.  The waits at
+ * exit for the kernel's own copies and tensor-core work in flight keep the
+ * default limit whatever is set here, so no CTA leaves with work outstanding.
+ */
+GQA_API int gqa_set_wait_limit(unsigned long long ns, unsigned long long *previous);
 
 /* Human-readable text for a GQA_ERR_* code. */
 GQA_API const char *gqa_error_string(int code);

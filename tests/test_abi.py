@@ -83,3 +83,14 @@ def test_timeline_argument_checks(lib):
     assert rc(rows=-1) == 1
     assert rc(B=-1) == 1                # the shape checks of gqa_decode
     assert rc(B=0) == 0 and grid.value == 0   # empty batch: nothing launched, no rows
+
+
+def test_wait_limit_arguments(lib):
+    """gqa_set_wait_limit: 0 restores the 1.5 s default, 1 us .. 10 s accepted."""
+    with pytest.raises(gq.GqaError):
+        gq.set_wait_limit(10)            # below 1 us
+    with pytest.raises(gq.GqaError):
+        gq.set_wait_limit(10 ** 11)      # above 10 s
+    assert gq.set_wait_limit(5_000_000) == 1_500_000_000
+    assert gq.set_wait_limit(0) == 5_000_000
+    assert gq.set_wait_limit(0) == 1_500_000_000

@@ -137,27 +137,54 @@ def test_single_key_returns_value_row():
 FULL = ["tiny", "llama3_8b", "long_256k"] + [f"sweep_{a}_{b}_{c}" for a, b, c in workloads.SWEEP]
 
 
+def run_auto(p, out=None, workspace=None):
+    """The bench's path: gqa_decode_auto with the host copy of the lengths."""
+    d = p.to("cuda")
+    return gq.gqa_decode_auto(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,
+                              p.seq_lens.to(torch.int32).contiguous(), out=out, scale=p.scale,
+                              workspace=workspace)
+
+
 @pytest.mark.parametrize("name", FULL)
 def test_workload_full_parity(name):
+    """Every output of the full-size workload, through gqa_decode (stream-K) and
+    gqa_decode_auto (the schedule the bench times), under the plain bar."""
     p = workloads.workload(name)
+    r = ref(p)
     out = run(p)
     torch.cuda.synchronize()
-    parity(out, ref(p), name)
+    parity(out, r, name)
+    out = run_auto(p)
+    torch.cuda.synchronize()
+    parity(out, r, name + " (auto)")
 
 
-def test_varlen_paged_sampled_rows():
-    """Full-size variable-length paged batch: every output is finite (poisoned slots and
-    unused table entries never read); sampled requests (shortest, longest, random)
-    match the oracle row by row."""
+def test_varlen_paged_full():
+    """Full-size variable-length paged batch: all 64 requests element by element
+    (poisoned tail slots and unused table entries are never read), through both
+    schedules."""
     p = workloads.workload("varlen_paged")
-    out = run(p)
-    torch.cuda.synchronize()
-    assert torch.isfinite(out.float()).all()
-    lens = p.seq_lens.tolist()
-    pick = sorted({int(np.argmin(lens)), int(np.argmax(lens)), 7, 31, 50})
-    for b in pick:
-        r = ref(p, rows=(b * p.Hq, (b + 1) * p.Hq))
-        parity(out[b], r, f"varlen request {b} (L={lens[b]})")
+    r = ref(p)
+    for fn, what in ((run, "stream-K"), (run_auto, "auto")):
+        out = fn(p)
+        torch.cuda.synchronize()
+        parity(out, r, f"varlen_paged ({what})")
+
+
+def test_auto_on_pages_the_tensor_cores_do_not_take():
+    """gqa_decode_auto on page sizes the tensor-core kernel cannot tile (3, 100 tokens)
+    with G = 4: the same result as gqa_decode, against the oracle."""
+    for bs, lens in ((3, [50, 2000]), (100, [4000, 17])):
+        p = make_problem("autopage", 2, 32, 8, 128, lens, seed=11 + bs, block_size=bs,
+                         spare_blocks=2)
+        r = ref(p)
+        parity(run_auto(p), r, f"auto, {bs}-token pages")
+        parity(run(p), r, f"decode, {bs}-token pages")
+        dec = gq.HostDecoder(p.B, p.Hq, p.Hkv, p.D, p.block_size, p.max_blocks, p.num_blocks,
+                             True)
+        out = torch.empty_like(p.q)
+        dec(p.q, p.k_cache, p.v_cache, p.block_table, p.seq_lens, out, scale=p.scale)
+        parity(out, r, f"host buffers, {bs}-token pages")
 
 
 # --------------------------------------------------------------------- invariants
@@ -185,6 +212,53 @@ def test_deterministic_repeat():
     outs = [gq.gqa_decode(d.q, d.k_cache, d.v_cache, None, d.seq_lens).clone() for _ in range(3)]
     for o in outs[1:]:
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["long_256k", "one_segment_200k", "varlen_small"])
+def test_split_segments_bitwise_repeat(name):
+    """Segments split over many CTAs are merged in a fixed order, so repeated calls
+    give bit-identical outputs whatever the CTAs' timing (other work and an L2
+    flush run between the calls to perturb it)."""
+    if name == "long_256k":
+        p = workloads.workload(name)
+    elif name == "one_segment_200k":
+        p = make_problem(name, 1, 16, 1, 128, [200000], seed=21, block_size=64)
+    else:
+        p = make_problem(name, 6, 32, 8, 128, [40000, 1, 9000, 700, 25000, 3], seed=22,
+                         block_size=16)
+    d = p.to("cuda")
+    junk = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    outs = []
+    for i in range(4):
+        junk.fill_(i)
+        if i % 2:
+            torch.cuda._sleep(1000 * (i + 1))
+        outs.append(gq.gqa_decode(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,
+                                  scale=p.scale).clone())
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+
+
+def test_plan_matches_what_runs():
+    """gqa_decode_plan's grid is the grid the timeline entry point records, for the
+    stream-K and the one-CTA-per-segment schedule."""
+    for name in ("long_256k", "tiny"):
+        p = workloads.workload(name)
+        d = p.to("cuda")
+        lens = p.seq_lens.to(torch.int32)
+        auto = gq.decode_plan(p.B, p.Hq, p.Hkv, p.D, p.block_size, p.paged, p.num_blocks,
+                              num_splits=-1, seq_lens_host=lens)
+        for ns in (0, 1):
+            plan = gq.decode_plan(p.B, p.Hq, p.Hkv, p.D, p.block_size, p.paged, p.num_blocks,
+                                  num_splits=ns, seq_lens_host=lens)
+            _, tl = gq.gqa_decode_timeline(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,
+                                           num_splits=ns, scale=p.scale)
+            torch.cuda.synchronize()
+            assert tl.shape[0] == plan["grid"] > 0
+            assert int(tl[:, 3].sum()) == plan["tiles"]
+            assert plan["workspace_bytes"] > 0 and plan["smem_bytes"] > 0
+        assert auto["num_splits"] == (0 if name == "long_256k" else 1)
 
 
 def test_contiguous_equals_paged():

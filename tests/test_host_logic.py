@@ -127,3 +127,20 @@ def test_cpu_baseline_reports_parity_of_its_sample():
     wrong[1, 3, 7] += 1.0                               # one wrong element is seen
     assert bench.cpu_oracle_sample(p, 0.2, gpu_out=wrong)["parity_of_sample"]["max_abs"] > 0.9
     assert "parity_of_sample" not in bench.cpu_oracle_sample(p, 0.05)
+
+
+def test_bf16_scaled_bound_is_the_binade_half_ulp():
+    """The stress-case tolerance: half a bf16 ulp of |ref|'s binade plus slack, and
+    exactly MAX_ABS below |ref| = 4; every correctly rounded value meets it."""
+    import numpy as np
+    from gpu_util import MAX_ABS, bf16_scaled_bound, half_ulp_bf16
+    assert half_ulp_bf16(np.array([1.0, 1.99, 2.0, 4.0, 4.5, 7.99]))[[0, 1, 2, 3, 4, 5]].tolist() == \
+        [2 ** -8, 2 ** -8, 2 ** -7, 2 ** -6, 2 ** -6, 2 ** -6]
+    below = np.linspace(-3.999, 3.999, 10001)
+    assert np.all(bf16_scaled_bound(below) == MAX_ABS)
+    assert bf16_scaled_bound(np.array([4.5]))[0] < 2 ** -6 + 2e-3
+    x = torch.randn(200000, dtype=torch.float64) * 8
+    rounded = x.to(torch.bfloat16).double()
+    assert np.all((rounded - x).abs().numpy() <= bf16_scaled_bound(x.numpy()))
+    # a one-ulp miss above 4 is caught
+    assert not np.all(2 * half_ulp_bf16(np.array([4.5])) <= bf16_scaled_bound(np.array([4.5])))

@@ -70,3 +70,41 @@ def test_noalloc_rejects_shapes_beyond_its_limits():
             4097, 4, 1, 128, p.block_size, p.scale, 0, 0, None)
     assert rc == 2 and "unsupported" in gq.error_string(rc)
     assert "8 MiB" in gq.error_string(gq.GQA_ERR_SCRATCH_LIMIT)
+
+
+def test_noalloc_scratch_covers_every_shape_within_the_maxima():
+    """The header's claim: every shape within GQA_MAX_BATCH and GQA_MAX_QHEADS needs
+    no more scratch than the fixed 8 MiB (gqa_decode_workspace_size is what the
+    entry point compares against), at the extreme batch and head counts."""
+    gq, _ = _noalloc_fn()
+    limit = 8 << 20
+    for D in (64, 128, 256):
+        for Hq, Hkv in ((256, 1), (256, 256), (256, 64), (4, 1)):
+            need = gq.workspace_size(4096, Hq, Hkv, D)
+            assert need <= limit, (D, Hq, Hkv, need)
+
+
+def test_noalloc_python_wrapper_checks_and_matches():
+    """The Python wrapper checks its tensors before anything is launched (a CPU
+    length array or a float32 output would otherwise reach the kernel as a bad
+    pointer) and otherwise returns gqa_decode's result."""
+    gq, _ = _noalloc_fn()
+    p = make_problem("wrap", 2, 32, 8, 128, [5000, 77], seed=80, block_size=16, spare_blocks=2)
+    d = p.to("cuda")
+    with pytest.raises(ValueError):
+        gq.gqa_decode_noalloc(d.q, d.k_cache, d.v_cache, d.block_table, p.seq_lens)
+    with pytest.raises(ValueError):
+        gq.gqa_decode_noalloc(d.q, d.k_cache, d.v_cache, p.block_table, d.seq_lens)
+    with pytest.raises(TypeError):
+        gq.gqa_decode_noalloc(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,
+                              out=torch.empty(d.q.shape, dtype=torch.float32, device="cuda"))
+    with pytest.raises(ValueError):
+        gq.gqa_decode_noalloc(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,
+                              out=torch.empty(2, 128, 32, dtype=torch.bfloat16,
+                                              device="cuda").transpose(1, 2))
+    expect = gq.gqa_decode(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens, scale=p.scale)
+    for _ in range(2):
+        got = gq.gqa_decode_noalloc(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,
+                                    scale=p.scale)
+        torch.cuda.synchronize()
+        parity(got, as_f64(expect), "python wrapper")
