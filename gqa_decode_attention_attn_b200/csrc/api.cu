@@ -647,7 +647,8 @@ int select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int 
             }
         }
     }
-    *num_splits = (tc && best < sk) ? best_s : 0;
+    // On a tie the fixed split wins: it needs neither a cooperative launch nor merges.
+    *num_splits = (tc && best <= sk) ? best_s : 0;
     if (est_us) {
         est_us[0] = (float)sk;
         est_us[1] = tc ? (float)best : -1.0f;

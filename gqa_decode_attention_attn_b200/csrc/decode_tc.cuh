@@ -302,13 +302,13 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     } else {
         // Segment j = (b, kvh, hc) in that order; its first tile in the global order
         // (hc, b, kvh, tile).
-        const int64_t j = c / p.nsplit, i = c - j * p.nsplit;
-        const int b = (int)(j / units);
-        const int64_t u = j - (int64_t)b * units, kv = u / p.hch, hc = u - kv * p.hch;
+        const int64_t j = div_nonneg(c, p.nsplit), i = c - j * p.nsplit;
+        const int b = (int)div_nonneg(j, units);
+        const int64_t u = j - (int64_t)b * units, kv = div_nonneg(u, p.hch), hc = u - kv * p.hch;
         const int64_t nbj = prefix[b + 1] - prefix[b];
         const int64_t seg0 = hc * p.Hkv * prefix[B] + (int64_t)p.Hkv * prefix[b] + kv * nbj;
-        start = seg0 + i * nbj / p.nsplit;
-        end = seg0 + (i + 1) * nbj / p.nsplit;
+        start = seg0 + div_nonneg(i * nbj, p.nsplit);
+        end = seg0 + div_nonneg((i + 1) * nbj, p.nsplit);
     }
     const int G = p.G;
 

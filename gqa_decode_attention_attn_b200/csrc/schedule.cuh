@@ -77,6 +77,16 @@ __device__ __forceinline__ int page_of(const Params &p, int t)
     return (int)((__umulhi(p.bs_magic, u) + u) >> p.bs_shift);
 }
 
+// Quotient of non-negative x by positive y, in 32 bits when both fit (the
+// 64-bit division is several times longer, and the prologue and the merge tail
+// call these on their critical paths).
+__device__ __forceinline__ int64_t div_nonneg(int64_t x, int64_t y)
+{
+    if ((((uint64_t)x | (uint64_t)y) >> 32) == 0)
+        return (int64_t)((uint32_t)x / (uint32_t)y);
+    return x / y;
+}
+
 // Walks the global tile order one tile at a time.  prefix[b] = sum of n_b'
 // (b' < b) lives in shared memory; units = Hkv * hch segments per request.  Only
 // init() divides; next() is increments and compares.
@@ -95,9 +105,9 @@ struct TileIter {
     __device__ __forceinline__ void init(int64_t i, const int *prefix, int B, int64_t units,
                                          int hch)
     {
-        const int64_t hkv = units / hch;
+        const int64_t hkv = div_nonneg(units, hch);
         const int64_t w1 = hkv * prefix[B];  // tiles per head chunk
-        hc = (int)(i / w1);
+        hc = (int)div_nonneg(i, w1);
         const int64_t i1 = i - (int64_t)hc * w1;
         int lo = 0, hi = B;  // hkv*prefix[lo] <= i1 < hkv*prefix[hi]
         while (hi - lo > 1) {
@@ -110,7 +120,7 @@ struct TileIter {
         b = lo;
         nb = prefix[lo + 1] - prefix[lo];
         const int64_t local = i1 - hkv * prefix[lo];
-        kvh = (int)(local / nb);
+        kvh = (int)div_nonneg(local, nb);
         j = (int)(local - (int64_t)kvh * nb);
         seg0 = (int64_t)hc * w1 + hkv * prefix[lo] + (int64_t)kvh * nb;
     }
@@ -164,16 +174,6 @@ struct RunWalker {
         }
     }
 };
-
-// Quotient of non-negative x by positive y, in 32 bits when both fit (the
-// 64-bit division is several times longer, and the merge tail calls these on
-// its critical path).
-__device__ __forceinline__ int64_t div_nonneg(int64_t x, int64_t y)
-{
-    if ((((uint64_t)x | (uint64_t)y) >> 32) == 0)
-        return (int64_t)((uint32_t)x / (uint32_t)y);
-    return x / y;
-}
 
 // First tile of CTA c, and the CTA whose run holds tile i.
 __device__ __forceinline__ int64_t run_start(int64_t c, int64_t W, int64_t P)
