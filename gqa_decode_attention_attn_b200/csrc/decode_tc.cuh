@@ -673,7 +673,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
 #pragma unroll
                 for (int g = 0; g < NV; ++g)
                     if (g < rows && ti < D)
-                        write_result<false>(p, out_row(p, cur.b, cur.kvh, r0 + g), ti, D, acc[g], m_ref[g],
+                        write_result<false>(p, MQ ? out_row(p, cur.b, cur.kvh, r0 + g) : out_row_q1(p, cur.b, cur.kvh, r0 + g), ti, D, acc[g], m_ref[g],
                                             lsum[g], pois);
             } else {
 #pragma unroll
@@ -719,10 +719,13 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         int64_t req_len = 0;
         uint64_t t_scores = 0;
         int k = 0;
-        for (int64_t i = start; i < end; ++i, ++k) {
-            if (i > start)
+        // One pass past the last tile (i == end) closes the last piece, so that the
+        // piece epilogue is written out once.
+        for (int64_t i = start;; ++i, ++k) {
+            const bool past = i == end;
+            if (i > start && !past)
                 it.next(prefix, B, p.Hkv, p.hch);
-            const bool first_tile = i == start || it.seg0 != cur.seg0;
+            const bool first_tile = !past && (i == start || it.seg0 != cur.seg0);
             if (first_tile) {
                 // Q of the new (request, KV head, head chunk) goes out first: the MMA
                 // warp issues this tile's BMM1 before the previous tile's BMM2, and
@@ -753,10 +756,14 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                     for (int g = 0; g < NV; ++g)
                         qs[g] = qscale * red[13 * NP + g];
                 }
+            }
+            if (first_tile || past) {
                 if (i > start) {
                     flush_fold();
                     epilogue(i);
                 }
+                if (past)
+                    break;
                 cur = it;
                 piece_first = i;
                 poisoned = false;
@@ -945,8 +952,6 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 fold_pend = true;
             }
         }
-        flush_fold();
-        epilogue(end);
         const uint64_t t_streamed = p.timeline ? global_timer_ns() : 0;
         // Split segments: publish every partial piece of this run, then merge this
         // CTA's share of each (all owners are resident: cooperative launch).  Every
@@ -957,7 +962,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             publish_piece(p, pending[x].vseg, stid, 1, 128);
         for (int x = 0; x < npending; ++x) {
             const PendingPiece &pp = pending[x];
-            merge_segment_gather<NV, D, 128>(p, c, pp.seg0, pp.nb, pp.first, pp.vseg, W, P, pp.rows,
+            merge_segment_gather<NV, D, 128, MQ>(p, c, pp.seg0, pp.nb, pp.first, pp.vseg, W, P, pp.rows,
                                              pp.b, pp.kvh, pp.r0, reinterpret_cast<int *>(pbuf),
                                              reinterpret_cast<float *>(ring), misc + 20, stid, 1,
                                              abort_flag);

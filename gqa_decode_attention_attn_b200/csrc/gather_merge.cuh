@@ -50,7 +50,7 @@ __device__ __forceinline__ void publish_piece(const Params &p, int64_t vseg, int
 // query rows r0 .. r0 + rows - 1 of (request b, KV head kvh), written to
 // out_row(p, b, kvh, r).  list: >= no ints of shared memory; buf: shared floats
 // for the gathered slices (see the bound in the kernel).
-template <int NV, int D, int NT>
+template <int NV, int D, int NT, bool MQ>
 __device__ __forceinline__ void merge_segment_gather(const Params &p, int64_t c, int64_t seg0,
                                                      int nb, int64_t piece_first, int64_t vseg,
                                                      int64_t W, int64_t P, int rows, int b, int kvh,
@@ -185,11 +185,11 @@ __device__ __forceinline__ void merge_segment_gather(const Params &p, int64_t c,
             if (sub != 0 || x >= Ec)
                 continue;
             if (!ok) {
-                write_result<false>(p, out_row(p, b, kvh, r0 + g), e - g * D, D, 0.f, 0.f, 0.f, true);
+                write_result<false>(p, MQ ? out_row(p, b, kvh, r0 + g) : out_row_q1(p, b, kvh, r0 + g), e - g * D, D, 0.f, 0.f, 0.f, true);
                 continue;
             }
             const float ls = hl_s[h];
-            write_result<false>(p, out_row(p, b, kvh, r0 + g), e - g * D, D, a, hm_s[h], ls, ls != ls);
+            write_result<false>(p, MQ ? out_row(p, b, kvh, r0 + g) : out_row_q1(p, b, kvh, r0 + g), e - g * D, D, a, hm_s[h], ls, ls != ls);
         }
     }
     named_barrier_sync(bar_id, NT);  // list and buf are reused by the next segment

@@ -211,6 +211,12 @@ __device__ __forceinline__ int64_t out_row(const Params &p, int b, int kvh, int 
     return ((int64_t)b * p.qlen + i) * p.Hq + (int64_t)kvh * p.G + h;
 }
 
+// out_row for one query token per request (qlen = 1): no division.
+__device__ __forceinline__ int64_t out_row_q1(const Params &p, int b, int kvh, int r)
+{
+    return (int64_t)b * p.Hq + (int64_t)kvh * p.G + r;
+}
+
 // Bounded wait on an mbarrier phase (at most p.wait_ns).  On timeout: status bit,
 // CTA abort flag.
 __device__ __forceinline__ bool bounded_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
@@ -245,7 +251,8 @@ __device__ __forceinline__ void write_result(const Params &p, int64_t row, int d
             p.st_l[row] = poisoned ? __int_as_float(0x7fc00000) : ls;
         }
     } else {
-        float o = poisoned ? __int_as_float(0x7fc00000) : (ls > 0.f ? p.vscale * a / ls : 0.f);
+        // (fast reciprocal division: well inside the bf16 output's precision)
+        float o = poisoned ? __int_as_float(0x7fc00000) : (ls > 0.f ? __fdividef(p.vscale * a, ls) : 0.f);
         __nv_bfloat16 h = __float2bfloat16_rn(o);
         p.out[row * D + d] = *reinterpret_cast<uint16_t *>(&h);
     }
