@@ -407,7 +407,8 @@ def extra_entry(r: Runner, steps: int, warmup: int, peak: float) -> dict:
          "GB_per_s": gbs, "frac": gbs / peak, "steps": steps,
          "algorithmic_bytes": r.p.algorithmic_bytes(), "kernel": r.plan["kernel_name"],
          "schedule": r.schedule, "grid": r.plan["grid"], "tiles": r.plan["tiles"],
-         "gpu_launches": steps * r.launches_per_step()}
+         "gpu_launches": steps * r.launches_per_step(),
+         "traffic": profiled_traffic(r.p.name, r.plan["kernel_name"])}
     if tl:
         e["tail_idle"] = tl["tail_idle"]
         e["span_us"] = tl["span_us"]
