@@ -1029,9 +1029,9 @@ const char *gqa_error_string(int code)
 // ---------------------------------------------------------------------------
 // gqa_decode_noalloc: gqa_decode for callers that cannot allocate device memory.
 //
-// Some callers may not call cudaMalloc at all: code running inside a CUDA-graph
-// capture or another runtime's memory pool, plug-ins whose host owns every
-// allocation, or latency-critical paths that forbid allocator calls.  They still
+// Some callers may not call cudaMalloc at all: code running under another
+// runtime's memory pool, plug-ins whose host owns every allocation, or
+// latency-critical paths that forbid allocator calls.  They still
 // own q, the caches and out, but cannot hand us a workspace.  For them the
 // scratch gqa_decode needs (status word, ticket counters, partial-state slots)
 // lives in one fixed array in this library's device image.  Every GPU that loads
