@@ -373,6 +373,32 @@ class Runner:
             raise SystemExit(f"{self.p.name}: device status error during the timed steps")
         return [s.elapsed_time(e) for s, e in zip(starts, ends)], region0.elapsed_time(region1)
 
+    def floor(self, steps: int):
+        """The streaming floor of this step: gqa_stream_floor over the same number of
+        K and V bytes, read from the workload's own cache buffers, on every SM, timed
+        like the step (L2 flushed before each, CUDA events).  Mean and median us."""
+        gq, d, p = self.gq, self.d, self.p
+        tile = gq.FLOOR_TILE_BYTES
+        kv = (p.algorithmic_bytes() - 4 * p.B * p.Hq * p.D) // 2  # bytes of K (= of V)
+        nbytes = max(tile, kv // tile * tile)
+        sms = torch.cuda.get_device_properties(self.dev).multi_processor_count
+        run = lambda: gq.stream_floor(d.k_cache, d.v_cache, nbytes, sms, self.ws, self.stream)
+        for _ in range(3):
+            self.flush.fill_(1)
+            run()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for i, (a, b) in enumerate(ev):
+            self.flush.fill_(i & 0xFF)
+            a.record(self.stream)
+            run()
+            b.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        if self.ws.status():
+            raise SystemExit(f"{p.name}: device status error in the streaming floor")
+        us = [a.elapsed_time(b) * 1e3 for a, b in ev]
+        return sum(us) / len(us), statistics.median(us), 2 * nbytes, sms
+
     def timeline(self):
         """One more step, untimed and after an L2 flush, through gqa_decode_timeline
         with the schedule the timed steps ran: per-CTA start/end (%globaltimer) and
@@ -403,12 +429,14 @@ def extra_entry(r: Runner, steps: int, warmup: int, peak: float) -> dict:
     ms = sum(per) / len(per)
     gbs = r.p.algorithmic_bytes() / (ms / 1e3) / 1e9
     tl = r.timeline()
+    floor_us, _, _, _ = r.floor(steps)
     e = {"us_per_step": ms * 1e3, "us_per_step_median": statistics.median(per) * 1e3,
          "GB_per_s": gbs, "frac": gbs / peak, "steps": steps,
          "algorithmic_bytes": r.p.algorithmic_bytes(), "kernel": r.plan["kernel_name"],
          "schedule": r.schedule, "grid": r.plan["grid"], "tiles": r.plan["tiles"],
          "gpu_launches": steps * r.launches_per_step(),
-         "traffic": profiled_traffic(r.p.name, r.plan["kernel_name"])}
+         "traffic": profiled_traffic(r.p.name, r.plan["kernel_name"]),
+         "floor_us": floor_us, "floor_frac": floor_us / (ms * 1e3)}
     if tl:
         e["tail_idle"] = tl["tail_idle"]
         e["span_us"] = tl["span_us"]
@@ -503,6 +531,14 @@ def main():
         tl = r.timeline()
         if tl:
             line["timeline"] = tl
+        f_mean, f_med, f_bytes, f_ctas = r.floor(args.steps)
+        line["stream_floor"] = {
+            "us_per_step": f_mean, "us_per_step_median": f_med, "kv_bytes": f_bytes,
+            "ctas": f_ctas, "GB_per_s": f_bytes / (f_mean / 1e6) / 1e9,
+            "floor_frac": f_mean / (ms * 1e3),
+            "what": ("gqa_stream_floor: the same K and V bytes through the decode kernel's "
+                     "TMA boxes and rings with no arithmetic, timed like the step; "
+                     "floor_frac = floor time / step time")}
     if r.mode == "fixed":  # comparator runs report the kernel numbers only
         args.no_e2e = args.no_cpu_baseline = True
     if rank == 0 and not args.no_e2e:

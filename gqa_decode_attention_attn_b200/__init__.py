@@ -35,7 +35,7 @@ EXPORTED = ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states", "gqa
             "gqa_decode_noalloc", "gqa_decode_fixed_split_workspace_size",
             "gqa_decode_fixed_split", "gqa_select_schedule", "gqa_decode_auto",
             "gqa_decode_multi", "gqa_decode_fp8", "gqa_decode_timeline", "gqa_decode_plan",
-            "gqa_set_wait_limit")
+            "gqa_set_wait_limit", "gqa_stream_floor")
 GQA_ERR_SCRATCH_LIMIT = 6
 TIMELINE_COLS = 8  # values per CTA row of gqa_decode_timeline
 KERNEL_TENSOR_CORE = 1
@@ -91,6 +91,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_decode_plan.argtypes = [I, I, I, I, I, I, I, I, I, I, P, I, ctypes.POINTER(_Plan)]
     lib.gqa_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P]
     lib.gqa_set_wait_limit.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong)]
+    lib.gqa_stream_floor.argtypes = [P, P, ctypes.c_longlong, I, P, SZ, P]
     lib.gqa_error_string.argtypes = [I]
     lib.gqa_error_string.restype = ctypes.c_char_p
     for name in ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states",
@@ -98,7 +99,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                  "gqa_decode_fixed_split_workspace_size", "gqa_decode_fixed_split",
                  "gqa_select_schedule", "gqa_decode_auto", "gqa_decode_multi",
                  "gqa_decode_fp8", "gqa_decode_plan", "gqa_decode_noalloc",
-                 "gqa_decode_timeline", "gqa_set_wait_limit"):
+                 "gqa_decode_timeline", "gqa_set_wait_limit", "gqa_stream_floor"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -110,6 +111,32 @@ def set_wait_limit(ns: int) -> int:
     prev = ctypes.c_ulonglong(0)
     _check("gqa_set_wait_limit", load_library().gqa_set_wait_limit(int(ns), ctypes.byref(prev)))
     return prev.value
+
+
+FLOOR_TILE_BYTES = 128 * 256  # one 128-row tile of 256-byte rows (gqa_stream_floor)
+
+
+def stream_floor(k: torch.Tensor, v: torch.Tensor, nbytes: int, ctas: int,
+                 workspace: Optional[Workspace] = None, stream=None) -> None:
+    """Stream the first `nbytes` bytes of k and of v (a multiple of FLOOR_TILE_BYTES)
+    through the decode kernels' TMA rings with no arithmetic, over `ctas` CTAs: the
+    measurement reference of gqa_stream_floor.  Asynchronous; a wait that ran out
+    shows in workspace.status()."""
+    lib = load_library()
+    dev = k.device
+    for t, n in ((k, "k"), (v, "v")):
+        if t.device != dev or dev.type != "cuda":
+            raise ValueError(f"{n} must be a CUDA tensor on {dev}")
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+        if nbytes > t.numel() * t.element_size():
+            raise ValueError(f"{n} holds fewer than {nbytes} bytes")
+    if nbytes <= 0 or nbytes % FLOOR_TILE_BYTES:
+        raise ValueError(f"nbytes must be a positive multiple of {FLOOR_TILE_BYTES}")
+    ws = workspace or default_workspace(dev)
+    buf = ws.get(256)
+    _check("gqa_stream_floor", lib.gqa_stream_floor(_ptr(k), _ptr(v), nbytes // 256, int(ctas),
+                                                    _ptr(buf), buf.numel(), _stream_ptr(stream)))
 
 
 def error_string(code: int) -> str:

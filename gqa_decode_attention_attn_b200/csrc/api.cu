@@ -16,6 +16,7 @@
 #include "decode_tc.cuh"
 #include "gqa_decode.h"
 #include "merge_states.cuh"
+#include "stream_floor.cuh"
 
 namespace gqa {
 namespace {
@@ -998,6 +999,34 @@ int gqa_decode_host(const void *q, const void *k_cache, const void *v_cache,
     if (cudaMemcpyAsync(out, dbuf + h.out, qbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return GQA_ERR_CUDA;
     return cudaStreamSynchronize(s) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+int gqa_stream_floor(const void *k, const void *v, long long rows, int ctas, void *workspace,
+                     size_t workspace_bytes, void *stream)
+{
+    using C = FloorCfg;
+    if (!k || !v || !workspace || rows < C::T || rows % C::T != 0 || rows > (1ll << 31) - C::T ||
+        ctas < 1)
+        return GQA_ERR_INVALID_ARG;
+    if (workspace_bytes < STATUS_BYTES)
+        return GQA_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(workspace))
+        return GQA_ERR_MISALIGNED;
+    int dev = 0, max_ctas = 0;
+    if (current_device(dev) != GQA_OK)
+        return GQA_ERR_CUDA;
+    const int rc = persistent_ctas_fn(reinterpret_cast<const void *>(stream_floor_kernel), C::THREADS,
+                                      C::SMEM, dev, max_ctas);
+    if (rc != GQA_OK)
+        return rc;
+    if (ctas > max_ctas)
+        return GQA_ERR_INVALID_ARG;
+    CUtensorMap tmk, tmv;
+    if (!encode_kv_map(&tmk, k, rows, C::T, 128) || !encode_kv_map(&tmv, v, rows, C::T, 128))
+        return GQA_ERR_CUDA;
+    stream_floor_kernel<<<ctas, C::THREADS, C::SMEM, static_cast<cudaStream_t>(stream)>>>(
+        tmk, tmv, rows / C::T, static_cast<unsigned *>(workspace), g_wait_ns.load());
+    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
 int gqa_set_wait_limit(unsigned long long ns, unsigned long long *previous)

@@ -379,6 +379,26 @@ GQA_API int gqa_decode_noalloc(const void *q, const void *k_cache, const void *v
  */
 GQA_API int gqa_set_wait_limit(unsigned long long ns, unsigned long long *previous);
 
+/*
+ * Measurement reference, not part of the attention path: streams k and v, each
+ * a contiguous bf16 array of `rows` rows of 128 columns (256 bytes per row;
+ * rows a positive multiple of 128, below 2^31), through the decode kernels'
+ * TMA boxes and three-slot rings of 32 KB with no arithmetic, over `ctas`
+ * CTAs (1 .. resident CTAs of the device), CTA c taking 128-row tiles
+ * [c W / ctas, (c+1) W / ctas) of the W = rows / 128 as the stream-K decode
+ * schedule does.  A decode step is bound by reading its K and V from HBM
+ * (Attention co-design for long-context inference, section "Difference between
+ * prefill and decode", Equation 1 and Figure 2), so this kernel, timed like a
+ * step over the step's K and V bytes, gives the floor that streaming alone
+ * reaches under that timing.  The bytes are read, never interpreted.
+ * k, v, workspace: DEVICE, 16-byte aligned; workspace as for gqa_decode (at
+ * least its status word): a bounded wait that runs out sets GQA_DEV_TIMEOUT
+ * there.  Returns GQA_OK, GQA_ERR_INVALID_ARG, GQA_ERR_WORKSPACE_TOO_SMALL,
+ * GQA_ERR_MISALIGNED or GQA_ERR_CUDA; asynchronous.
+ */
+GQA_API int gqa_stream_floor(const void *k, const void *v, long long rows, int ctas,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
 /* Human-readable text for a GQA_ERR_* code. */
 GQA_API const char *gqa_error_string(int code);
 

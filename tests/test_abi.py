@@ -94,3 +94,21 @@ def test_wait_limit_arguments(lib):
     assert gq.set_wait_limit(5_000_000) == 1_500_000_000
     assert gq.set_wait_limit(0) == 5_000_000
     assert gq.set_wait_limit(0) == 1_500_000_000
+
+
+def test_stream_floor_argument_checks(lib):
+    """gqa_stream_floor rejects bad arguments on the host, before any CUDA call."""
+    P = ctypes.c_void_p
+
+    def rc(k=16, v=16, rows=256, ctas=4, ws=16, ws_bytes=256):
+        return lib.gqa_stream_floor(None if k is None else P(k), None if v is None else P(v),
+                                    rows, ctas, None if ws is None else P(ws), ws_bytes, None)
+
+    assert rc(k=None) == 1
+    assert rc(ws=None) == 1
+    assert rc(rows=0) == 1
+    assert rc(rows=200) == 1            # not a whole number of 128-row tiles
+    assert rc(rows=1 << 31) == 1        # row coordinates are 32-bit
+    assert rc(ctas=0) == 1
+    assert rc(ws_bytes=8) == 3          # no room for the status word
+    assert rc(v=24) == 4                # not 16-byte aligned
