@@ -45,6 +45,8 @@ KERNEL_SOURCES = {
     "tc": [_CSRC + f for f in ("decode_tc.cuh", "gather_merge.cuh", "schedule.cuh", "tc.cuh",
                                "ptx.cuh")],
     "simt": [_CSRC + f for f in ("decode_simt.cuh", "schedule.cuh", "ptx.cuh")],
+    "wide": [_CSRC + f for f in ("decode_tc_wide.cuh", "decode_tc.cuh", "gather_merge.cuh",
+                                 "schedule.cuh", "tc.cuh", "ptx.cuh")],
 }
 
 
@@ -93,7 +95,8 @@ def hbm_peak():
 def kernel_source_hash(kernel: str) -> str:
     """Hash of the sources of the named kernel (a gqa_decode_plan kernel name)."""
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES["tc" if "tc_kernel" in kernel else "simt"]:
+    kind = "wide" if "tc_wide_kernel" in kernel else "tc" if "tc_kernel" in kernel else "simt"
+    for rel in KERNEL_SOURCES[kind]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

@@ -582,7 +582,7 @@ class HostDecoder:
 def gqa_decode_noalloc(q, k_cache, v_cache, block_table, seq_lens, out=None, scale=None,
                        stream=None):
     """gqa_decode for callers that cannot allocate device memory: the library uses
-    its own fixed 8 MiB device scratch instead of a workspace.  Calls on one device
+    its own fixed 16 MiB device scratch instead of a workspace.  Calls on one device
     share that scratch, so they must not overlap on the GPU.  (`out` is allocated
     here only when the caller passes none.)  Tensors are checked as gqa_decode
     checks them, before anything is launched."""

@@ -14,6 +14,7 @@
 
 #include "decode_simt.cuh"
 #include "decode_tc.cuh"
+#include "decode_tc_wide.cuh"
 #include "gqa_decode.h"
 #include "merge_states.cuh"
 #include "stream_floor.cuh"
@@ -231,6 +232,20 @@ int tc_ctas(int G, int dev, int &ctas, bool mq = false, int D = 128, bool fp8 = 
                               TcCfg::THREADS, tc_smem_bytes(D, TcCfg::MAX_BATCH, fp8), dev, ctas);
 }
 
+// The wide tensor-core kernel (64 heads per pass) takes bf16 caches at D = 128
+// with one query token and more than 16 query heads per KV head; the fixed split
+// into several chunks (merge_split_kernel) stays on the 16-head kernel.
+bool tc_wide(int R, int D, bool mq, bool fp8, int nsplit)
+{
+    return !mq && !fp8 && D == 128 && R > TcCfg::NP && nsplit <= 1;
+}
+
+int tc_wide_ctas(int dev, int &ctas)
+{
+    return persistent_ctas_fn(reinterpret_cast<const void *>(gqa_decode_tc_wide_kernel), TcWide::THREADS,
+                              TcWide::smem_bytes(TcCfg::MAX_BATCH), dev, ctas);
+}
+
 // Head dimensions the tensor-core kernel is built for.
 bool tc_head_dim(int D)
 {
@@ -349,9 +364,10 @@ struct Plan {
     bool use_tc = false;   // tensor-core kernel (else the CUDA-core kernel)
     bool mq = false;       // several query tokens per request
     bool fp8 = false;
+    bool wide = false;     // the 64-heads-per-pass tensor-core kernel
     Variant v{};           // CUDA-core kernel variant
     int G = 0, R = 0;      // query heads per KV head; query rows per KV head
-    int nv = 0;            // heads one pass carries (tensor cores: 4, 8, 16; CUDA cores: GC)
+    int nv = 0;            // heads one pass carries (tensor cores: 4, 8, 16, 64; CUDA cores: GC)
     int hch = 0;           // passes (head chunks) per KV head
     int nsplit = 0;        // 0: stream-K; n > 0: fixed split into n chunks
     int ctas = 0;          // persistent grid; -1 when no device was given
@@ -386,7 +402,16 @@ int make_plan(bool states, int B, int Hq, int Hkv, int D, int block_size, bool p
         return GQA_ERR_UNSUPPORTED;
     if (nsplit > 0 && !pl.use_tc)
         return GQA_ERR_UNSUPPORTED;
-    if (pl.use_tc) {
+    pl.wide = pl.use_tc && tc_wide(pl.R, D, pl.mq, fp8, nsplit);
+    if (pl.wide) {
+        pl.hch = (pl.R + TcWide::NP - 1) / TcWide::NP;
+        pl.nv = TcWide::NP;
+        pl.threads = TcWide::THREADS;
+        pl.tile_tokens = TcWide::T;
+        pl.stages = TcWide::SV;
+        pl.smem = TcWide::smem_bytes(B);
+        pl.box_rows = tc_box_rows(paged, block_size);
+    } else if (pl.use_tc) {
         pl.hch = (pl.R + TcCfg::NP - 1) / TcCfg::NP;
         pl.nv = pl.R <= 4 ? 4 : (pl.R <= 8 ? 8 : 16);
         pl.threads = TcCfg::THREADS;
@@ -413,13 +438,16 @@ int make_plan(bool states, int B, int Hq, int Hkv, int D, int block_size, bool p
         pl.grid = nsplit > 0 ? pl.items : -1;
         return GQA_OK;
     }
-    int rc = pl.use_tc ? tc_ctas(pl.R, dev, pl.ctas, pl.mq, D, fp8) : persistent_ctas(pl.v, dev, pl.ctas);
+    int rc = pl.wide     ? tc_wide_ctas(dev, pl.ctas)
+             : pl.use_tc ? tc_ctas(pl.R, dev, pl.ctas, pl.mq, D, fp8)
+                         : persistent_ctas(pl.v, dev, pl.ctas);
     if (rc)
         return rc;
     // One chunk per segment (nsplit = 1) always finishes its segment: no slots.
-    pl.w = nsplit > 1    ? layout_for((int)((pl.items + 1) / 2), TcCfg::SLOT_FLOATS)
-           : nsplit == 1 ? layout_for(0, TcCfg::SLOT_FLOATS)
-                         : layout_for(pl.ctas, pl.use_tc ? TcCfg::SLOT_FLOATS : pl.v.slot_floats);
+    const int tc_slot = pl.wide ? TcWide::SLOT_FLOATS : TcCfg::SLOT_FLOATS;
+    pl.w = nsplit > 1    ? layout_for((int)((pl.items + 1) / 2), tc_slot)
+           : nsplit == 1 ? layout_for(0, tc_slot)
+                         : layout_for(pl.ctas, pl.use_tc ? tc_slot : pl.v.slot_floats);
     pl.grid = nsplit > 0 ? pl.items : pl.ctas;
     return GQA_OK;
 }
@@ -528,8 +556,8 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         if (nsplit > 0) {
             // Fixed split: as many CTAs as chunks, in waves; no CTA waits for another.
             const cudaStream_t st = static_cast<cudaStream_t>(stream);
-            tc_kernel_for(R, qlen > 1, D, fp8)<<<(unsigned)items, TcCfg::THREADS, pl.smem, st>>>(
-                p, tmk, tmv, box_rows);
+            const TcKernelFn fn = pl.wide ? gqa_decode_tc_wide_kernel : tc_kernel_for(R, qlen > 1, D, fp8);
+            fn<<<(unsigned)items, pl.threads, pl.smem, st>>>(p, tmk, tmv, box_rows);
             if (B > 0 && nsplit > 1) {
                 const int64_t threads = (int64_t)B * Hkv * pl.hch * pl.nv * D;
                 tc_merge_for(R, D)<<<(unsigned)((threads + 127) / 128), 128, 0, st>>>(p);
@@ -541,7 +569,7 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         // rather than run otherwise).
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)ctas);
-        cfg.blockDim = dim3(TcCfg::THREADS);
+        cfg.blockDim = dim3(pl.threads);
         cfg.dynamicSmemBytes = pl.smem;
         cfg.stream = static_cast<cudaStream_t>(stream);
         cudaLaunchAttribute attr[1];
@@ -549,7 +577,8 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, tc_kernel_for(R, qlen > 1, D, fp8), p, tmk, tmv, box_rows) != cudaSuccess)
+        const TcKernelFn fn = pl.wide ? gqa_decode_tc_wide_kernel : tc_kernel_for(R, qlen > 1, D, fp8);
+        if (cudaLaunchKernelEx(&cfg, fn, p, tmk, tmv, box_rows) != cudaSuccess)
             return GQA_ERR_CUDA;
     } else {
         pl.v.fn<<<ctas, pl.threads, pl.smem, static_cast<cudaStream_t>(stream)>>>(p);
@@ -577,8 +606,13 @@ int select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int 
             return GQA_ERR_INVALID_ARG;
     const int G = Hq / Hkv;
     const bool tc = tc_head_dim(D) && G >= TC_MIN_G && B <= TcCfg::MAX_BATCH;
-    const int64_t units = (int64_t)Hkv * (tc ? (G + TcCfg::NP - 1) / TcCfg::NP
-                                             : (G + head_chunk(G) - 1) / head_chunk(G));
+    // Segments per request: head passes per KV head.  Stream-K and one chunk per
+    // segment take the wide kernel's 64-head passes where it applies; a split into
+    // several chunks runs 16-head passes.
+    const int64_t units16 = (int64_t)Hkv * (tc ? (G + TcCfg::NP - 1) / TcCfg::NP
+                                               : (G + head_chunk(G) - 1) / head_chunk(G));
+    const int64_t units = tc && tc_wide(G, D, false, false, 0)
+                              ? (int64_t)Hkv * ((G + TcWide::NP - 1) / TcWide::NP) : units16;
     // Microseconds per 128-token K+V tile for a CTA while `active` CTAs stream.
     const double tile_bytes = 4.0 * TcCfg::T * D;
     auto tile_us = [&](int64_t active) {
@@ -616,11 +650,12 @@ int select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int 
     int best_s = 1;
     if (tc) {
         for (int sp = 1; sp <= max_splits; sp *= 2) {
-            if ((int64_t)B * units * sp > ((int64_t)1 << 21))
+            const int64_t un = sp == 1 ? units : units16;
+            if ((int64_t)B * un * sp > ((int64_t)1 << 21))
                 break;  // keep the host-side estimate cheap
             int64_t items = 0;
             for (int b = 0; b < B; ++b)
-                items += units * std::min<int64_t>(nb[b], sp);
+                items += un * std::min<int64_t>(nb[b], sp);
             const double tu = tile_us(std::min(P, items));
             std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
             for (int64_t i = 0; i < P; ++i)
@@ -628,7 +663,7 @@ int select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int 
             double makespan = 0.0;
             bool any_split = false;
             for (int b = 0; b < B; ++b)
-                for (int64_t u = 0; u < units; ++u) {
+                for (int64_t u = 0; u < un; ++u) {
                     int nonempty = 0;
                     for (int i = 0; i < sp; ++i) {
                         const int64_t len = (int64_t)(i + 1) * nb[b] / sp - (int64_t)i * nb[b] / sp;
@@ -698,6 +733,13 @@ int gqa_decode_workspace_size(int B, int Hq, int Hkv, int D, int device, size_t 
         if ((rc = tc_ctas(TC_MIN_G, device, ctas)))
             return rc;
         const size_t t = layout_for(ctas, TcCfg::SLOT_FLOATS).total;
+        best = t > best ? t : best;
+    }
+    if (tc_wide(Hq / Hkv, D, false, false, 0)) {  // 64 heads per pass: larger slots
+        int ctas = 0;
+        if ((rc = tc_wide_ctas(device, ctas)))
+            return rc;
+        const size_t t = layout_for(ctas, TcWide::SLOT_FLOATS).total;
         best = t > best ? t : best;
     }
     *bytes = best;
@@ -850,7 +892,10 @@ int gqa_decode_plan(int B, int Hq, int Hkv, int D, int block_size, int paged, in
             tiles += ((long long)seq_lens_host[b] + pl.tile_tokens - 1) / pl.tile_tokens;
         plan->tiles = tiles * Hkv * pl.hch;
     }
-    if (pl.use_tc)
+    if (pl.wide)
+        std::snprintf(plan->kernel_name, sizeof plan->kernel_name, "gqa_decode_tc_wide_kernel<NV=%d,D=%d>",
+                      pl.nv, D);
+    else if (pl.use_tc)
         std::snprintf(plan->kernel_name, sizeof plan->kernel_name,
                       "gqa_decode_tc_kernel<NV=%d,MQ=%d,D=%d,F8=%d>", pl.nv, pl.mq ? 1 : 0, D,
                       kv_fp8 ? 1 : 0);
@@ -1048,7 +1093,7 @@ const char *gqa_error_string(int code)
     case GQA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
     case GQA_ERR_MISALIGNED: return "bf16 tensor not 16-byte aligned";
     case GQA_ERR_CUDA: return "CUDA runtime error";
-    case GQA_ERR_SCRATCH_LIMIT: return "shape needs more scratch than gqa_decode_noalloc's fixed 8 MiB";
+    case GQA_ERR_SCRATCH_LIMIT: return "shape needs more scratch than gqa_decode_noalloc's fixed 16 MiB";
     default: return "unknown error";
     }
 }
@@ -1068,7 +1113,7 @@ const char *gqa_error_string(int code)
 // ---------------------------------------------------------------------------
 namespace {
 
-constexpr size_t NOALLOC_SCRATCH_BYTES = 8u << 20;  // 8 MiB per device
+constexpr size_t NOALLOC_SCRATCH_BYTES = 16u << 20;  // 16 MiB per device
 
 // Device-side scratch shared by every gqa_decode_noalloc call on a device.  In
 // host code this name is only a handle; its device address comes from

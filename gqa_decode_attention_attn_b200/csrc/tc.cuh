@@ -101,10 +101,9 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
                  : "memory");
 }
 
-// 16 consecutive 32-bit columns of this thread's TMEM lane (32x32b shape), and
-// the wait for them, in one statement so no use can be scheduled before the wait.
 // N consecutive 32-bit columns of this warp's 32 TMEM lanes (one lane per
-// thread), N = 4, 8 or 16, waiting for the load to complete.
+// thread, 32x32b shape), N = 4, 8, 16 or 32, and the wait for them, in one
+// statement so that no use can be scheduled before the wait.
 template <int N>
 __device__ __forceinline__ void tmem_load(uint32_t taddr, float (&v)[N]);
 
@@ -152,6 +151,43 @@ __device__ __forceinline__ void tmem_load<4>(uint32_t taddr, float (&v)[4])
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         v[i] = __uint_as_float(r[i]);
+}
+
+template <>
+__device__ __forceinline__ void tmem_load<32>(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+                 "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+                   "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]),
+                   "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+                   "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+                   "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr)
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
+// 16 consecutive 32-bit columns of this warp's 32 TMEM lanes from registers (one
+// lane per thread), waiting until the store has completed.
+__device__ __forceinline__ void tmem_store16(uint32_t taddr, const float (&v)[16])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+                 "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};\n\t"
+                 "tcgen05.wait::st.sync.aligned;"
+                 ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
+                   "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
+                   "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+                   "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+                   "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+                   "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+                 : "memory");
 }
 
 // Generic-proxy shared-memory writes become visible to the async proxy (TMA,

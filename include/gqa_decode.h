@@ -343,9 +343,9 @@ GQA_API int gqa_decode_host(const void *q, const void *k_cache, const void *v_ca
  * allocator calls are forbidden -- and so cannot pass the workspace gqa_decode
  * wants.  Arguments, layouts and results are those of gqa_decode.
  *
- * Scratch: one fixed 8 MiB array inside the library's device image, held by
+ * Scratch: one fixed 16 MiB array inside the library's device image, held by
  * every GPU that loads the library until the process exits.  A shape whose
- * scratch need (gqa_decode_workspace_size) exceeds 8 MiB is rejected with
+ * scratch need (gqa_decode_workspace_size) exceeds 16 MiB is rejected with
  * GQA_ERR_SCRATCH_LIMIT; B above GQA_MAX_BATCH or Hq above GQA_MAX_QHEADS with
  * GQA_ERR_UNSUPPORTED.  On B200 every shape within those maxima fits.
  *

@@ -73,6 +73,12 @@ SMALL = [
     (1, 4, 1, 128, [100000], None),
     (1, 16, 1, 128, [200000], 64),
     (1, 2, 1, 64, [150000], 16),
+    # the 64-heads-per-pass tensor-core kernel (G > 16 at D = 128)
+    (3, 48, 1, 128, [129, 1, 4000], 16),                # G = 48: padded 64-head pass
+    (2, 128, 1, 128, [3000, 257], 32),                  # G = 128: two 64-head passes
+    (4, 64, 2, 128, [5000, 1, 0, 777], None),           # contiguous, an empty request
+    (1, 64, 1, 128, [150000], 64),                      # one long segment over every CTA
+    (2, 32, 1, 128, [130, 9000], 8),                    # G = 32, 8-token pages
     # tensor-core path at D = 64
     (2, 32, 4, 64, [3001, 77], 32),                     # G = 8
     (2, 16, 2, 64, [1000, 999], None),                  # contiguous
@@ -102,6 +108,8 @@ OUTLIER = [
     (6, 8, 1, 128, [2000, 1, 4097, 640, 130, 9000], 32, 16.0),
     (1, 16, 1, 128, [100000], None, 24.0),
     (4, 16, 4, 64, [5000, 3000, 1, 700], 16, 16.0),
+    (4, 64, 1, 128, [6000, 3000, 1, 900], 16, 16.0),    # 64-head passes
+    (1, 64, 1, 128, [100000], 64, 24.0),                # 64-head passes, split segment
 ]
 
 
@@ -214,7 +222,7 @@ def test_deterministic_repeat():
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
 
 
-@pytest.mark.parametrize("name", ["long_256k", "one_segment_200k", "varlen_small"])
+@pytest.mark.parametrize("name", ["long_256k", "one_segment_200k", "varlen_small", "mqa_200k"])
 def test_split_segments_bitwise_repeat(name):
     """Segments split over many CTAs are merged in a fixed order, so repeated calls
     give bit-identical outputs whatever the CTAs' timing (other work and an L2
@@ -223,6 +231,8 @@ def test_split_segments_bitwise_repeat(name):
         p = workloads.workload(name)
     elif name == "one_segment_200k":
         p = make_problem(name, 1, 16, 1, 128, [200000], seed=21, block_size=64)
+    elif name == "mqa_200k":   # the 64-heads-per-pass kernel
+        p = make_problem(name, 2, 64, 1, 128, [200000, 31000], seed=23, block_size=64)
     else:
         p = make_problem(name, 6, 32, 8, 128, [40000, 1, 9000, 700, 25000, 3], seed=22,
                          block_size=16)
@@ -243,7 +253,7 @@ def test_split_segments_bitwise_repeat(name):
 def test_plan_matches_what_runs():
     """gqa_decode_plan's grid is the grid the timeline entry point records, for the
     stream-K and the one-CTA-per-segment schedule."""
-    for name in ("long_256k", "tiny"):
+    for name in ("long_256k", "tiny", "sweep_64_1_128"):
         p = workloads.workload(name)
         d = p.to("cuda")
         lens = p.seq_lens.to(torch.int32)
@@ -258,7 +268,7 @@ def test_plan_matches_what_runs():
             assert tl.shape[0] == plan["grid"] > 0
             assert int(tl[:, 3].sum()) == plan["tiles"]
             assert plan["workspace_bytes"] > 0 and plan["smem_bytes"] > 0
-        assert auto["num_splits"] == (0 if name == "long_256k" else 1)
+        assert auto["num_splits"] == (1 if name == "tiny" else 0)
 
 
 def test_contiguous_equals_paged():
@@ -341,9 +351,10 @@ def test_merge_states_against_oracle():
 
 # --------------------------------------------------------------------- errors, no faults
 
-def test_bad_block_id_sets_status_and_nan_rows():
+@pytest.mark.parametrize("Hq", [4, 64])
+def test_bad_block_id_sets_status_and_nan_rows(Hq):
     lens = [100, 90]
-    p = make_problem("badblk", 2, 4, 1, 128, lens, seed=12, block_size=16)
+    p = make_problem("badblk", 2, Hq, 1, 128, lens, seed=12, block_size=16)
     p.block_table[1, 2] = p.num_blocks + 1000          # out of the pool: must not be read
     ws = gq.Workspace("cuda")
     out = run(p, workspace=ws)
@@ -351,7 +362,7 @@ def test_bad_block_id_sets_status_and_nan_rows():
     assert st & gq.DEV_BAD_BLOCK
     o = out.cpu().float()
     assert torch.isnan(o[1]).all()
-    r = ref(make_problem("badblk", 2, 4, 1, 128, lens, seed=12, block_size=16))
+    r = ref(make_problem("badblk", 2, Hq, 1, 128, lens, seed=12, block_size=16))
     parity(out[0], r[0], "unaffected request")
     assert ws.status() == 0                             # cleared by the read
 

@@ -52,8 +52,16 @@ def test_plan_reports_the_dispatch():
     f8 = _plan(1, 32, 8, 128, kv_fp8=True)
     assert f8["kernel"] == tc and f8["kernel_name"].endswith("F8=1>")
     assert _plan(1, 32, 8, 64, kv_fp8=True)["kernel"] == cc           # FP8 at D = 64
-    mqa = _plan(8, 64, 1, 128, seq_lens_host=[100] * 8)
-    assert mqa["heads_per_pass"] == 16 and mqa["head_chunks"] == 4 and mqa["tiles"] == 8 * 4
+    mqa = _plan(8, 64, 1, 128, seq_lens_host=[100] * 8)   # G = 64: one 64-head pass per tile
+    assert mqa["heads_per_pass"] == 64 and mqa["head_chunks"] == 1 and mqa["tiles"] == 8
+    assert mqa["kernel_name"] == "gqa_decode_tc_wide_kernel<NV=64,D=128>" and mqa["ring_stages"] == 3
+    assert _plan(2, 128, 1, 128)["head_chunks"] == 2                  # G = 128: two passes of 64
+    assert _plan(2, 32, 1, 128)["heads_per_pass"] == 64               # G = 32 on the wide kernel
+    assert _plan(2, 32, 2, 128)["heads_per_pass"] == 16               # G = 16 stays at 16
+    assert _plan(2, 64, 1, 64)["heads_per_pass"] == 16                # D = 64: 16-head passes
+    wfx = _plan(2, 64, 1, 128, num_splits=4)                          # fixed split: 16-head kernel
+    assert wfx["heads_per_pass"] == 16 and wfx["grid"] == 2 * 4 * 4
+    assert _plan(2, 64, 1, 128, num_splits=1)["heads_per_pass"] == 64
     assert _plan(2, 32, 8, 128, qlen=4)["kernel_name"].startswith("gqa_decode_tc_kernel<NV=16,MQ=1")
     fx = _plan(2, 32, 8, 128, num_splits=4)
     assert fx["num_splits"] == 4 and fx["grid"] == 2 * 8 * 4 and fx["merge_launch"] == 1

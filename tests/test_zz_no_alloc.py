@@ -69,15 +69,15 @@ def test_noalloc_rejects_shapes_beyond_its_limits():
     rc = fn(ptr(p.q), ptr(p.k_cache), ptr(p.v_cache), None, ptr(p.seq_lens), ptr(out),
             4097, 4, 1, 128, p.block_size, p.scale, 0, 0, None)
     assert rc == 2 and "unsupported" in gq.error_string(rc)
-    assert "8 MiB" in gq.error_string(gq.GQA_ERR_SCRATCH_LIMIT)
+    assert "16 MiB" in gq.error_string(gq.GQA_ERR_SCRATCH_LIMIT)
 
 
 def test_noalloc_scratch_covers_every_shape_within_the_maxima():
     """The header's claim: every shape within GQA_MAX_BATCH and GQA_MAX_QHEADS needs
-    no more scratch than the fixed 8 MiB (gqa_decode_workspace_size is what the
+    no more scratch than the fixed 16 MiB (gqa_decode_workspace_size is what the
     entry point compares against), at the extreme batch and head counts."""
     gq, _ = _noalloc_fn()
-    limit = 8 << 20
+    limit = 16 << 20
     for D in (64, 128, 256):
         for Hq, Hkv in ((256, 1), (256, 256), (256, 64), (4, 1)):
             need = gq.workspace_size(4096, Hq, Hkv, D)
