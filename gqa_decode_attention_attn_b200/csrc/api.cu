@@ -200,6 +200,8 @@ TcKernelFn tc_kernel_for(int G, bool mq = false, int D = 128, bool fp8 = false)
     }
     if (D == 64)
         return mq ? tc_kernel_nv<true, 64>(G) : tc_kernel_nv<false, 64>(G);
+    if (D == 256)  // one query token (the plan keeps several on the CUDA-core kernel's check)
+        return tc_kernel_nv<false, 256>(G);
     return mq ? tc_kernel_nv<true, 128>(G) : tc_kernel_nv<false, 128>(G);
 }
 
@@ -216,14 +218,20 @@ MergeFn tc_merge_nv(int G)
 
 MergeFn tc_merge_for(int G, int D = 128)
 {
-    return D == 64 ? tc_merge_nv<64>(G) : tc_merge_nv<128>(G);
+    return D == 64 ? tc_merge_nv<64>(G) : D == 256 ? tc_merge_nv<256>(G) : tc_merge_nv<128>(G);
 }
 
 size_t tc_smem_bytes(int D, int B, bool fp8 = false)
 {
     if (fp8)
         return TcGeom<128, true>::smem_bytes(B);
-    return D == 64 ? TcGeom<64>::smem_bytes(B) : TcGeom<128>::smem_bytes(B);
+    return D == 64 ? TcGeom<64>::smem_bytes(B) : D == 256 ? TcGeom<256>::smem_bytes(B) : TcGeom<128>::smem_bytes(B);
+}
+
+// Floats of one partial-state slot of the 16-head tensor-core kernel at head dimension D.
+int tc_slot_floats(int D)
+{
+    return D == 256 ? slot_floats(TcCfg::NP, 256) : TcCfg::SLOT_FLOATS;
 }
 
 int tc_ctas(int G, int dev, int &ctas, bool mq = false, int D = 128, bool fp8 = false)
@@ -246,10 +254,10 @@ int tc_wide_ctas(int dev, int &ctas)
                               TcWide::smem_bytes(TcCfg::MAX_BATCH), dev, ctas);
 }
 
-// Head dimensions the tensor-core kernel is built for.
+// Head dimensions the tensor-core kernel is built for (256: one query token, bf16).
 bool tc_head_dim(int D)
 {
-    return D == 64 || D == 128;
+    return D == 64 || D == 128 || D == 256;
 }
 
 // ---- tensor-core path: applicability and tensor maps -------------------------
@@ -394,7 +402,7 @@ int make_plan(bool states, int B, int Hq, int Hkv, int D, int block_size, bool p
     pl.fp8 = fp8;
     // FP8 caches run on the tensor cores at D = 128 (one query token), else on the
     // CUDA-core kernel.
-    pl.use_tc = (!fp8 || (D == 128 && qlen == 1)) &&
+    pl.use_tc = (!fp8 || (D == 128 && qlen == 1)) && (D != 256 || qlen == 1) &&
                 tc_applicable(states, B, Hkv, D, block_size, paged, num_blocks, pl.R);
     if (!pl.use_tc && !pick_variant(D, pl.G, states, pl.v, fp8))
         return GQA_ERR_UNSUPPORTED;
@@ -417,7 +425,7 @@ int make_plan(bool states, int B, int Hq, int Hkv, int D, int block_size, bool p
         pl.threads = TcCfg::THREADS;
         pl.tile_tokens = TcCfg::T;
         pl.stages = fp8 ? TcGeom<128, true>::STAGES
-                        : (D == 64 ? TcGeom<64>::STAGES : TcGeom<128>::STAGES);
+                        : (D == 64 ? TcGeom<64>::STAGES : D == 256 ? TcGeom<256>::STAGES : TcGeom<128>::STAGES);
         pl.smem = tc_smem_bytes(D, B, fp8);
         pl.box_rows = tc_box_rows(paged, block_size);
     } else {
@@ -444,7 +452,7 @@ int make_plan(bool states, int B, int Hq, int Hkv, int D, int block_size, bool p
     if (rc)
         return rc;
     // One chunk per segment (nsplit = 1) always finishes its segment: no slots.
-    const int tc_slot = pl.wide ? TcWide::SLOT_FLOATS : TcCfg::SLOT_FLOATS;
+    const int tc_slot = pl.wide ? TcWide::SLOT_FLOATS : tc_slot_floats(D);
     pl.w = nsplit > 1    ? layout_for((int)((pl.items + 1) / 2), tc_slot)
            : nsplit == 1 ? layout_for(0, tc_slot)
                          : layout_for(pl.ctas, pl.use_tc ? tc_slot : pl.v.slot_floats);
@@ -732,7 +740,7 @@ int gqa_decode_workspace_size(int B, int Hq, int Hkv, int D, int device, size_t 
         int ctas = 0;
         if ((rc = tc_ctas(TC_MIN_G, device, ctas)))
             return rc;
-        const size_t t = layout_for(ctas, TcCfg::SLOT_FLOATS).total;
+        const size_t t = layout_for(ctas, tc_slot_floats(D)).total;
         best = t > best ? t : best;
     }
     if (tc_wide(Hq / Hkv, D, false, false, 0)) {  // 64 heads per pass: larger slots
@@ -769,7 +777,7 @@ int gqa_decode_fixed_split_workspace_size(int B, int Hq, int Hkv, int D, int num
     const int64_t items = (int64_t)B * Hkv * ((G + TcCfg::NP - 1) / TcCfg::NP) * num_splits;
     if (items > (int64_t)1 << 30)
         return GQA_ERR_INVALID_ARG;
-    *bytes = layout_for(num_splits > 1 ? (int)((items + 1) / 2) : 0, TcCfg::SLOT_FLOATS).total;
+    *bytes = layout_for(num_splits > 1 ? (int)((items + 1) / 2) : 0, tc_slot_floats(D)).total;
     return GQA_OK;
 }
 

@@ -66,18 +66,24 @@ static_assert(TcCfg::O_COL + 2 * TcCfg::NO <= TcCfg::TMEM_COLS, "tensor memory c
 // flight).  At bf16 D = 64 BMM2 still runs M = 128 over V^T; its rows 64..127
 // come from one 16 KB block of zeros shared by every V slot (the operand's
 // leading-byte offset points there).  At 8 bits one box row spans all 128 rows
-// of V^T.
+// of V^T.  At bf16 D = 256 a tile's two 128-column halves are two consecutive
+// slots of the 32 KB rings (SUB = 2): BMM1 accumulates S over both, BMM2 writes
+// each half's O rows to its own TMEM columns; Q (8 KB) has one buffer, so that the
+// rings keep three slots.
 template <int D, bool F8 = false>
 struct TcGeom {
     static_assert(!F8 || D == 128, "FP8 tiles are built for D = 128");
-    static constexpr int BOXES = (F8 ? D : 2 * D) / 128;   // 128-byte boxes per token row
+    static constexpr int SUB = D == 256 ? 2 : 1;           // ring slots per tile
+    static constexpr int BOXES = (F8 ? D : 2 * D / SUB) / 128;  // 128-byte boxes per token row of a slot
     static constexpr bool NEED_ZERO = !F8 && D == 64;
     static constexpr int STAGES = BOXES == 1 ? 5 : 3;      // slots per ring (K ring, V ring)
     static constexpr int SLOT_BYTES = BOXES * TcCfg::BOX_BYTES;
+    static constexpr int QBUFS = D == 256 ? 1 : 2;         // Q buffers
+    static constexpr int QBUF = (D == 256 ? 2 : 1) * TcCfg::QBUF_BYTES;
     static constexpr size_t V_RING_OFF = (size_t)STAGES * SLOT_BYTES;
     static constexpr size_t ZERO_OFF = 2 * V_RING_OFF;                 // NEED_ZERO only
     static constexpr size_t Q_OFF = ZERO_OFF + (NEED_ZERO ? TcCfg::BOX_BYTES : 0);
-    static constexpr size_t P_OFF = Q_OFF + 2 * TcCfg::QBUF_BYTES;
+    static constexpr size_t P_OFF = Q_OFF + QBUFS * QBUF;
     static constexpr size_t BAR_OFF = P_OFF + 2 * TcCfg::PBUF_BYTES;
     static constexpr int NBAR = 4 * STAGES + 16;
     static constexpr size_t MISC_OFF = BAR_OFF + NBAR * 8;
@@ -177,7 +183,10 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     using C = TcCfg;
     using L = TcGeom<DH, F8>;
     constexpr int S = L::STAGES, NP = C::NP, D = DH, T = C::T;
-    constexpr int HALVES = L::BOXES;  // 128-byte boxes loaded per token row
+    constexpr int HALVES = L::BOXES;  // 128-byte boxes loaded per token row of a slot
+    constexpr int SUB = L::SUB;       // ring slots per tile (2 at D = 256)
+    constexpr int QH = D / 64;        // 64-column halves of a bf16 Q row
+    constexpr int QBUFS = L::QBUFS;
     constexpr int SW = F8 ? 2 * NP : NP;            // S columns per buffer
     constexpr int OC = F8 ? 4 * NP : C::O_COL;      // first O column
     constexpr int KSTEP = F8 ? 32 : 16;             // MMA K per instruction
@@ -185,10 +194,10 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     // per 16-byte row: term 1, then term 2).
     constexpr int NO = F8 ? 3 * NP : C::NO;         // BMM2 columns: the P terms side by side
     constexpr int P8_LBO = 3 * 128;                 // FP8 P: three core matrices per 8 tokens
-    constexpr int TMEM_COLS = F8 ? 256 : C::TMEM_COLS;
-    static_assert(OC + 2 * NO <= TMEM_COLS, "tensor memory columns");
+    constexpr int TMEM_COLS = (F8 || SUB == 2) ? 256 : C::TMEM_COLS;
+    static_assert(OC + 2 * NO * SUB <= TMEM_COLS, "tensor memory columns");
     static_assert(!F8 || (T / 8) * P8_LBO <= C::PBUF_BYTES, "FP8 P buffer");
-    static_assert(D == 64 || D == 128, "head dimension");
+    static_assert(D == 64 || D == 128 || (D == 256 && !MQ && !F8), "head dimension");
     constexpr int SLOT = slot_floats(NV, D);
     constexpr int LPH = 32 / NV;  // lanes per head after a transposed warp reduction
     static_assert(NV == 4 || NV == 8 || NV == 16, "softmax head count");
@@ -254,7 +263,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         // Likewise Q's upper half.
         for (int x = tid; x < C::BOX_BYTES / 16; x += C::THREADS)
             reinterpret_cast<uint4 *>(ring + L::ZERO_OFF)[x] = make_uint4(0, 0, 0, 0);
-        for (int x = tid; x < 2 * C::QBUF_BYTES / 16; x += C::THREADS)
+        for (int x = tid; x < QBUFS * L::QBUF / 16; x += C::THREADS)
             reinterpret_cast<uint4 *>(qbuf)[x] = make_uint4(0, 0, 0, 0);
         fence_proxy_async_smem();
     }
@@ -345,56 +354,112 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 return -1;
             return (int)((blk * p.Hkv + ti.kvh) * p.block_size + (t - pg * p.block_size));
         };
-        int cur_b = -1, len = 0, k = 0;
-        for (int64_t i = start; i < end; ++i, ++k) {
-            if (i > start)
-                it.next(prefix, B, p.Hkv, p.hch);
-            const int s = k % S;
-            const uint32_t ph = (uint32_t)((k / S) & 1);
-            if (k >= S && !bounded_wait(&emptyb[s], ph ^ 1u, abort_flag, p))
-                break;
-            if (it.b != cur_b) {
-                cur_b = it.b;
-                int64_t b0, l0;
-                request_range<false>(p, cur_b, b0, l0);
-                len = (int)l0;
-            }
-            const int tok0 = it.j * T;
-            const int n = min(T, len - tok0);
-            const int nbox = (n + box_rows - 1) / box_rows;
-            bool bad = false;
-            int row = 0;
-            if (lane < nbox) {
-                row = box_row(it, tok0);
-                bad = row < 0;
-                row = bad ? 0 : row;
-            }
-            const unsigned badmask = __ballot_sync(0xffffffffu, bad);
-            if (lane == 0) {
-                // Tile metadata travels with the V slot: a V slot is recycled only
-                // after every softmax thread has posted this tile's P, while a K
-                // slot may be refilled before a slow softmax thread looks at it.
-                if (!is_k) {
-                    stage_n[s] = n;
-                    stage_bad[s] = badmask != 0;
-                    if (badmask)
-                        atomicOr(p.status, DEV_BAD_BLOCK);
+        int cur_b = -1, len = 0, ks = 0;  // ks: ring slots filled (SUB per tile)
+        if constexpr (SUB == 1) {
+            for (int64_t i = start; i < end; ++i, ++ks) {
+                if (i > start)
+                    it.next(prefix, B, p.Hkv, p.hch);
+                const int s = ks % S;
+                const uint32_t ph = (uint32_t)((ks / S) & 1);
+                if (ks >= S && !bounded_wait(&emptyb[s], ph ^ 1u, abort_flag, p))
+                    break;
+                if (it.b != cur_b) {
+                    cur_b = it.b;
+                    int64_t b0, l0;
+                    request_range<false>(p, cur_b, b0, l0);
+                    len = (int)l0;
                 }
-                const uint32_t boxes = (uint32_t)(nbox - __popc(badmask));
-                mbar_arrive_expect_tx(&full[s], boxes * (uint32_t)HALVES * (uint32_t)box_rows * 128u);
-                if (p.timeline && is_k && k == 0)
-                    p.timeline[TL_COLS * c + 4] = global_timer_ns();
+                const int tok0 = it.j * T;
+                const int n = min(T, len - tok0);
+                const int nbox = (n + box_rows - 1) / box_rows;
+                bool bad = false;
+                int row = 0;
+                if (lane < nbox) {
+                    row = box_row(it, tok0);
+                    bad = row < 0;
+                    row = bad ? 0 : row;
+                }
+                const unsigned badmask = __ballot_sync(0xffffffffu, bad);
+                if (lane == 0) {
+                    // Tile metadata travels with the V slot: a V slot is recycled only
+                    // after every softmax thread has posted this tile's P, while a K
+                    // slot may be refilled before a slow softmax thread looks at it.
+                    if (!is_k) {
+                        stage_n[s] = n;
+                        stage_bad[s] = badmask != 0;
+                        if (badmask)
+                            atomicOr(p.status, DEV_BAD_BLOCK);
+                    }
+                    const uint32_t boxes = (uint32_t)(nbox - __popc(badmask));
+                    mbar_arrive_expect_tx(&full[s], boxes * (uint32_t)HALVES * (uint32_t)box_rows * 128u);
+                    if (p.timeline && is_k && ks == 0)
+                        p.timeline[TL_COLS * c + 4] = global_timer_ns();
+                }
+                __syncwarp();
+                if (lane < nbox && !bad) {
+                    unsigned char *d = base + (size_t)s * L::SLOT_BYTES + (size_t)lane * box_rows * 128;
+                    tma_load_2d(d, map, 0, row, &full[s], pol);
+                    if constexpr (HALVES == 2)
+                        tma_load_2d(d + C::BOX_BYTES, map, 64, row, &full[s], pol);
+                }
             }
-            __syncwarp();
-            if (lane < nbox && !bad) {
-                unsigned char *d = base + (size_t)s * L::SLOT_BYTES + (size_t)lane * box_rows * 128;
-                tma_load_2d(d, map, 0, row, &full[s], pol);
-                if constexpr (HALVES == 2)
-                    tma_load_2d(d + C::BOX_BYTES, map, 64, row, &full[s], pol);
+        } else {
+            // D = 256: the tile's two column halves go to two consecutive slots.
+            bool stop = false;
+            for (int64_t i = start; i < end && !stop; ++i) {
+                if (i > start)
+                    it.next(prefix, B, p.Hkv, p.hch);
+                int n = 0, nbox = 0, row = 0;
+                bool bad = false;
+                unsigned badmask = 0;
+#pragma unroll
+                for (int sub = 0; sub < SUB; ++sub, ++ks) {
+                    const int s = ks % S;
+                    const uint32_t ph = (uint32_t)((ks / S) & 1);
+                    if (ks >= S && !bounded_wait(&emptyb[s], ph ^ 1u, abort_flag, p)) {
+                        stop = true;
+                        break;
+                    }
+                    if (sub == 0) {
+                        if (it.b != cur_b) {
+                            cur_b = it.b;
+                            int64_t b0, l0;
+                            request_range<false>(p, cur_b, b0, l0);
+                            len = (int)l0;
+                        }
+                        const int tok0 = it.j * T;
+                        n = min(T, len - tok0);
+                        nbox = (n + box_rows - 1) / box_rows;
+                        if (lane < nbox) {
+                            row = box_row(it, tok0);
+                            bad = row < 0;
+                            row = bad ? 0 : row;
+                        }
+                        badmask = __ballot_sync(0xffffffffu, bad);
+                    }
+                    if (lane == 0) {
+                        if (!is_k) {
+                            stage_n[s] = n;
+                            stage_bad[s] = badmask != 0;
+                            if (badmask)
+                                atomicOr(p.status, DEV_BAD_BLOCK);
+                        }
+                        const uint32_t boxes = (uint32_t)(nbox - __popc(badmask));
+                        mbar_arrive_expect_tx(&full[s], boxes * (uint32_t)HALVES * (uint32_t)box_rows * 128u);
+                        if (p.timeline && is_k && ks == 0)
+                            p.timeline[TL_COLS * c + 4] = global_timer_ns();
+                    }
+                    __syncwarp();
+                    if (lane < nbox && !bad) {
+                        unsigned char *d = base + (size_t)s * L::SLOT_BYTES + (size_t)lane * box_rows * 128;
+                        tma_load_2d(d, map, sub * 128, row, &full[s], pol);
+                        tma_load_2d(d + C::BOX_BYTES, map, sub * 128 + 64, row, &full[s], pol);
+                    }
+                }
             }
         }
         if (lane == 0) {
-            for (int kk = max(0, k - S); kk < k; ++kk) {
+            for (int kk = max(0, ks - S); kk < ks; ++kk) {
                 const uint64_t t0 = global_timer_ns();
                 while (!mbar_try_wait(&full[kk % S], (uint32_t)((kk / S) & 1)) &&
                        global_timer_ns() - t0 < WAIT_LIMIT_NS) {
@@ -424,29 +489,36 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                         seg1 = it1.seg0;
                         ++piece1;
                     }
-                    const int s = k % S, b = k & 1, qb = (piece1 - 1) & 1;
-                    ok = bounded_wait(&k_full[s], (uint32_t)((k / S) & 1), abort_flag, p) &&
-                         (k < 2 || bounded_wait(&s_free[b], (uint32_t)(((k - 2) >> 1) & 1), abort_flag, p)) &&
-                         bounded_wait(&q_full[qb], (uint32_t)(((piece1 - 1) >> 1) & 1), abort_flag, p);
-                    if (!ok)
-                        break;
-                    tc_fence_after_sync();
-                    const uint32_t ka = ring_a + (uint32_t)(s * L::SLOT_BYTES);
-                    const uint32_t qa = q_a + (uint32_t)(qb * C::QBUF_BYTES);
+                    const int b = k & 1, qb = QBUFS == 2 ? (piece1 - 1) & 1 : 0;
+                    const uint32_t qpar = (uint32_t)((QBUFS == 2 ? (piece1 - 1) >> 1 : piece1 - 1) & 1);
+                    const uint32_t qa = q_a + (uint32_t)(qb * L::QBUF);
 #pragma unroll
-                    for (int kk = 0; kk < D / KSTEP; ++kk) {
-                        // 32 bytes of every row per instruction: 16 bf16 or 32 E4M3 elements.
-                        const uint32_t off = (uint32_t)((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32);
-                        const uint32_t qoff = (uint32_t)((kk >> 2) * NP * 128 + (kk & 3) * 32);
-                        const uint64_t ad = umma_smem_desc(ka + off, 16, 1024, SMEM_LAYOUT_SW128);
-                        const uint64_t bd = umma_smem_desc(qa + qoff, 16, 1024, SMEM_LAYOUT_SW128);
-                        if constexpr (F8)
-                            umma_e4m3(tbase + (uint32_t)(C::S_COL + b * SW), ad, bd, idesc1, kk > 0);
-                        else
-                            umma_bf16(tbase + (uint32_t)(C::S_COL + b * SW), ad, bd, idesc1, kk > 0);
+                    for (int sub = 0; sub < SUB && ok; ++sub) {
+                        const int ks = k * SUB + sub, s = ks % S;
+                        ok = bounded_wait(&k_full[s], (uint32_t)((ks / S) & 1), abort_flag, p) &&
+                             (sub > 0 || k < 2 ||
+                              bounded_wait(&s_free[b], (uint32_t)(((k - 2) >> 1) & 1), abort_flag, p)) &&
+                             (sub > 0 || bounded_wait(&q_full[qb], qpar, abort_flag, p));
+                        if (!ok)
+                            break;
+                        tc_fence_after_sync();
+                        const uint32_t ka = ring_a + (uint32_t)(s * L::SLOT_BYTES);
+#pragma unroll
+                        for (int kk = 0; kk < D / SUB / KSTEP; ++kk) {
+                            // 32 bytes of every row per instruction: 16 bf16 or 32 E4M3 elements.
+                            const uint32_t off = (uint32_t)((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32);
+                            const uint32_t qoff = (uint32_t)((2 * sub + (kk >> 2)) * NP * 128 + (kk & 3) * 32);
+                            const uint64_t ad = umma_smem_desc(ka + off, 16, 1024, SMEM_LAYOUT_SW128);
+                            const uint64_t bd = umma_smem_desc(qa + qoff, 16, 1024, SMEM_LAYOUT_SW128);
+                            if constexpr (F8)
+                                umma_e4m3(tbase + (uint32_t)(C::S_COL + b * SW), ad, bd, idesc1, kk > 0);
+                            else
+                                umma_bf16(tbase + (uint32_t)(C::S_COL + b * SW), ad, bd, idesc1, sub > 0 || kk > 0);
+                        }
+                        if (sub == SUB - 1)
+                            umma_commit(&s_full[b]);
+                        umma_commit(&k_empty[s]);
                     }
-                    umma_commit(&s_full[b]);
-                    umma_commit(&k_empty[s]);
                 }
             } else {
                 // O accumulates in one TMEM buffer across tiles while the softmax
@@ -461,7 +533,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 int u = 0;
                 bool fresh = true;
                 for (int k = 0; k < ntiles && ok; ++k) {
-                    const int s = k % S, b = k & 1;
+                    const int b = k & 1;
                     if (!bounded_wait(&p_full[b], (uint32_t)((k >> 1) & 1), abort_flag, p)) {
                         ok = false;
                         break;
@@ -471,9 +543,8 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                         ++u;
                         fresh = true;
                     }
-                    ok = (!fresh || u < 2 ||
-                          bounded_wait(&o_free[u & 1], (uint32_t)(((u - 2) >> 1) & 1), abort_flag, p)) &&
-                         bounded_wait(&v_full[s], (uint32_t)((k / S) & 1), abort_flag, p);
+                    ok = !fresh || u < 2 ||
+                         bounded_wait(&o_free[u & 1], (uint32_t)(((u - 2) >> 1) & 1), abort_flag, p);
                     if (!ok)
                         break;
                     // Does the piece end with tile k?  (itp runs one tile ahead.)
@@ -483,31 +554,42 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                         piece_ends = itp.seg0 != segp;
                         segp = itp.seg0;
                     }
-                    tc_fence_after_sync();
-                    const uint32_t va_off = (uint32_t)(L::V_RING_OFF + s * L::SLOT_BYTES);
-                    const uint32_t va = ring_a + va_off;
-                    // V^T rows 64..127: the slot's upper half, or the zero block at D = 64.
-                    const uint32_t vlbo = HALVES == 2 ? (uint32_t)C::BOX_BYTES : (uint32_t)L::ZERO_OFF - va_off;
                     const uint32_t pa = p_a + (uint32_t)(b * C::PBUF_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < T / KSTEP; ++kk) {
-                        if constexpr (F8) {
-                            // 32 tokens per instruction: 4 KB of V rows, four 8-token groups of P.
-                            umma_e4m3(tbase + (uint32_t)(OC + (u & 1) * NO),
-                                      umma_smem_desc(va + (uint32_t)(kk * 4096), C::BOX_BYTES, 1024,
-                                                     SMEM_LAYOUT_SW128),
-                                      umma_smem_desc(pa + (uint32_t)(4 * kk * P8_LBO), P8_LBO, 128,
-                                                     SMEM_LAYOUT_NONE),
-                                      idesc2, kk > 0 || !fresh);
-                        } else {
-                            umma_bf16(tbase + (uint32_t)(OC + (u & 1) * NO),
-                                      umma_smem_desc(va + (uint32_t)(kk * 2048), vlbo, 1024, SMEM_LAYOUT_SW128),
-                                      umma_smem_desc(pa + (uint32_t)(2 * kk * C::P_LBO), C::P_LBO, 128, SMEM_LAYOUT_NONE),
-                                      idesc2, kk > 0 || !fresh);
+                    for (int sub = 0; sub < SUB && ok; ++sub) {
+                        // O^T rows of head-dimension half `sub` (D = 256) in their own columns.
+                        const int ks = k * SUB + sub, s = ks % S;
+                        ok = bounded_wait(&v_full[s], (uint32_t)((ks / S) & 1), abort_flag, p);
+                        if (!ok)
+                            break;
+                        tc_fence_after_sync();
+                        const uint32_t va_off = (uint32_t)(L::V_RING_OFF + s * L::SLOT_BYTES);
+                        const uint32_t va = ring_a + va_off;
+                        // V^T rows 64..127: the slot's upper half, or the zero block at D = 64.
+                        const uint32_t vlbo = HALVES == 2 ? (uint32_t)C::BOX_BYTES : (uint32_t)L::ZERO_OFF - va_off;
+                        const uint32_t ocol = tbase + (uint32_t)(OC + (u & 1) * NO * SUB + sub * NO);
+#pragma unroll
+                        for (int kk = 0; kk < T / KSTEP; ++kk) {
+                            if constexpr (F8) {
+                                // 32 tokens per instruction: 4 KB of V rows, four 8-token groups of P.
+                                umma_e4m3(ocol,
+                                          umma_smem_desc(va + (uint32_t)(kk * 4096), C::BOX_BYTES, 1024,
+                                                         SMEM_LAYOUT_SW128),
+                                          umma_smem_desc(pa + (uint32_t)(4 * kk * P8_LBO), P8_LBO, 128,
+                                                         SMEM_LAYOUT_NONE),
+                                          idesc2, kk > 0 || !fresh);
+                            } else {
+                                umma_bf16(ocol,
+                                          umma_smem_desc(va + (uint32_t)(kk * 2048), vlbo, 1024, SMEM_LAYOUT_SW128),
+                                          umma_smem_desc(pa + (uint32_t)(2 * kk * C::P_LBO), C::P_LBO, 128, SMEM_LAYOUT_NONE),
+                                          idesc2, kk > 0 || !fresh);
+                            }
                         }
+                        umma_commit(&v_empty[s]);
                     }
+                    if (!ok)
+                        break;
                     fresh = false;
-                    umma_commit(&v_empty[s]);
                     umma_commit(&p_free[b]);
                     if (piece_ends) {
                         umma_commit(&o_full[u & 1]);
@@ -593,7 +675,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         };
         // acc holds the closed O buffers, relative to the current reference m_ref
         // (the open TMEM buffer shares that reference).
-        float m_ref[NV], l_t[NV], acc[NV];
+        float m_ref[NV], l_t[NV], acc[SUB][NV];
         PendingPiece pending[2];  // a run has at most a first and a last partial piece
         int npending = 0;
         bool poisoned = false;
@@ -607,38 +689,45 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
         // Fold closed O buffer use u (scaled by w[g]) into acc and hand it back.
         auto fold = [&](const float (&w)[NV]) {
             const int bc = u & 1;
-            float o[NV];
+            float o[SUB][NV];
             if (ok && bounded_wait(&o_full[bc], (uint32_t)((u >> 1) & 1), abort_flag, p)) {
-                float olo[NV];
                 tc_fence_after_sync();
-                tmem_load<NV>(tlane + (uint32_t)(OC + bc * NO), o);
-                tmem_load<NV>(tlane + (uint32_t)(OC + bc * NO + NP), olo);
-                if constexpr (F8) {
-                    // P terms 2 and 3 carry x16 and x256.
-                    float o3[NV];
-                    tmem_load<NV>(tlane + (uint32_t)(OC + bc * NO + 2 * NP), o3);
 #pragma unroll
-                    for (int g = 0; g < NV; ++g)
-                        o[g] = fmaf(fmaf(o3[g], 1.f / 16.f, olo[g]), 1.f / 16.f, o[g]);
+                for (int sub = 0; sub < SUB; ++sub) {
+                    float olo[NV];
+                    const uint32_t oc = tlane + (uint32_t)(OC + bc * NO * SUB + sub * NO);
+                    tmem_load<NV>(oc, o[sub]);
+                    tmem_load<NV>(oc + NP, olo);
+                    if constexpr (F8) {
+                        // P terms 2 and 3 carry x16 and x256.
+                        float o3[NV];
+                        tmem_load<NV>(oc + 2 * NP, o3);
+#pragma unroll
+                        for (int g = 0; g < NV; ++g)
+                            o[sub][g] = fmaf(fmaf(o3[g], 1.f / 16.f, olo[g]), 1.f / 16.f, o[sub][g]);
+                    } else {
+#pragma unroll
+                        for (int g = 0; g < NV; ++g)
+                            o[sub][g] += olo[g];
+                    }
                 }
                 tc_fence_before_sync();
-                if constexpr (!F8) {
-#pragma unroll
-                    for (int g = 0; g < NV; ++g)
-                        o[g] += olo[g];
-                }
             } else {
                 ok = false;
                 poisoned = true;
 #pragma unroll
-                for (int g = 0; g < NV; ++g)
-                    o[g] = 0.f;
+                for (int sub = 0; sub < SUB; ++sub)
+#pragma unroll
+                    for (int g = 0; g < NV; ++g)
+                        o[sub][g] = 0.f;
             }
             mbar_arrive(&o_free[bc]);
             ++u;
 #pragma unroll
-            for (int g = 0; g < NV; ++g)
-                acc[g] = fmaf(o[g], w[g], acc[g]);
+            for (int sub = 0; sub < SUB; ++sub)
+#pragma unroll
+                for (int g = 0; g < NV; ++g)
+                    acc[sub][g] = fmaf(o[sub][g], w[g], acc[sub][g]);
         };
 
         auto epilogue = [&](int64_t last_excl) {
@@ -671,15 +760,19 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             float *slot = p.slots + (p.nsplit ? c : 2 * c + (piece_first == start ? 0 : 1)) * (int64_t)SLOT;
             if (complete) {
 #pragma unroll
-                for (int g = 0; g < NV; ++g)
-                    if (g < rows && ti < D)
-                        write_result<false>(p, MQ ? out_row(p, cur.b, cur.kvh, r0 + g) : out_row_q1(p, cur.b, cur.kvh, r0 + g), ti, D, acc[g], m_ref[g],
-                                            lsum[g], pois);
+                for (int sub = 0; sub < SUB; ++sub)
+#pragma unroll
+                    for (int g = 0; g < NV; ++g)
+                        if (g < rows && ti + 128 * sub < D)
+                            write_result<false>(p, MQ ? out_row(p, cur.b, cur.kvh, r0 + g) : out_row_q1(p, cur.b, cur.kvh, r0 + g),
+                                                ti + 128 * sub, D, acc[sub][g], m_ref[g], lsum[g], pois);
             } else {
 #pragma unroll
-                for (int g = 0; g < NV; ++g)
-                    if (ti < D)
-                        slot[g * D + ti] = acc[g];
+                for (int sub = 0; sub < SUB; ++sub)
+#pragma unroll
+                    for (int g = 0; g < NV; ++g)
+                        if (ti + 128 * sub < D)
+                            slot[g * D + ti + 128 * sub] = acc[sub][g];
                 if (ti < NV) {
                     float mv = m_ref[0], lvv = lsum[0];
 #pragma unroll
@@ -733,12 +826,13 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 // 128-byte-swizzled K-major form the tensor cores read (row g,
                 // 16-byte chunk cc of a 64-column half at chunk position cc ^ (g & 7)).
                 ++piece;
-                unsigned char *qd = qbuf + ((piece - 1) & 1) * C::QBUF_BYTES;
+                const int qb = QBUFS == 2 ? (piece - 1) & 1 : 0;
+                unsigned char *qd = qbuf + qb * L::QBUF;
                 if constexpr (F8) {
                     load_q_e4m3(qd, it);
                 } else {
 #pragma unroll
-                for (int r = 0; r < HALVES; ++r) {
+                for (int r = 0; r < QH; ++r) {
                     const int x = stid + 128 * r;
                     const int half = x >> 7, g = (x & 127) >> 3, cc = x & 7;
                     uint4 w = make_uint4(0, 0, 0, 0);
@@ -749,7 +843,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 }
                 }
                 fence_proxy_async_smem();
-                mbar_arrive(&q_full[(piece - 1) & 1]);
+                mbar_arrive(&q_full[qb]);
                 if constexpr (F8) {
                     named_barrier_sync(1, 128);  // the rows' range factors are in red
 #pragma unroll
@@ -771,15 +865,21 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 for (int g = 0; g < NV; ++g) {
                     m_ref[g] = -INFINITY;
                     l_t[g] = 0.f;
-                    acc[g] = 0.f;
+#pragma unroll
+                    for (int sub = 0; sub < SUB; ++sub)
+                        acc[sub][g] = 0.f;
                 }
             }
 
-            const int s = k % S, b = k & 1;
+            const int s = (k * SUB) % S, b = k & 1;  // the tile's (first) V slot
             float sc[NV];
             int n = 0;
-            if (ok && bounded_wait(&v_full[s], (uint32_t)((k / S) & 1), abort_flag, p) &&
-                bounded_wait(&s_full[b], (uint32_t)((k >> 1) & 1), abort_flag, p)) {
+            bool have_v = ok;
+#pragma unroll
+            for (int sub = 0; sub < SUB; ++sub)
+                have_v = have_v && bounded_wait(&v_full[(k * SUB + sub) % S],
+                                                (uint32_t)(((k * SUB + sub) / S) & 1), abort_flag, p);
+            if (have_v && bounded_wait(&s_full[b], (uint32_t)((k >> 1) & 1), abort_flag, p)) {
                 n = stage_n[s];
                 poisoned |= stage_bad[s] != 0;
                 tc_fence_after_sync();
@@ -855,7 +955,9 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                     m_ref[g] = m_new;
                     x[g] = (see[g] && m_new != -INFINITY) ? fmaf(sc[g], qsc(g), -m_new) : -INFINITY;
                     l_t[g] *= alpha[g];
-                    acc[g] *= alpha[g];
+#pragma unroll
+                    for (int sub = 0; sub < SUB; ++sub)
+                        acc[sub][g] *= alpha[g];
                 }
             }
             // This P buffer was last read by BMM2 two tiles ago.
@@ -931,12 +1033,15 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             // Rows past the valid tokens may hold anything (stale tiles, poison):
             // zero this token's V row so that 0-weight rows add exact zeros.
             if (!valid) {
-                unsigned char *vr = ring + L::V_RING_OFF + (size_t)s * L::SLOT_BYTES + ti * 128;
 #pragma unroll
-                for (int h = 0; h < HALVES; ++h)
+                for (int sub = 0; sub < SUB; ++sub) {
+                    unsigned char *vr = ring + L::V_RING_OFF + (size_t)((k * SUB + sub) % S) * L::SLOT_BYTES + ti * 128;
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc)
-                        *reinterpret_cast<uint4 *>(vr + h * C::BOX_BYTES + cc * 16) = make_uint4(0, 0, 0, 0);
+                    for (int h = 0; h < HALVES; ++h)
+#pragma unroll
+                        for (int cc = 0; cc < 8; ++cc)
+                            *reinterpret_cast<uint4 *>(vr + h * C::BOX_BYTES + cc * 16) = make_uint4(0, 0, 0, 0);
+                }
             }
             // A moved reference closes the open O buffer (unless this tile opens a
             // piece, whose buffer is fresh anyway).

@@ -79,6 +79,11 @@ SMALL = [
     (4, 64, 2, 128, [5000, 1, 0, 777], None),           # contiguous, an empty request
     (1, 64, 1, 128, [150000], 64),                      # one long segment over every CTA
     (2, 32, 1, 128, [130, 9000], 8),                    # G = 32, 8-token pages
+    # tensor-core path at D = 256 (two ring slots per tile)
+    (2, 16, 4, 256, [3000, 129], 16),                   # G = 4, 16-token pages
+    (2, 32, 2, 256, [700, 1], None),                    # G = 16, contiguous
+    (3, 24, 2, 256, [128, 127, 4097], 64),              # G = 12: padded head chunk
+    (1, 8, 1, 256, [100000], 64),                       # one long segment over every CTA
     # tensor-core path at D = 64
     (2, 32, 4, 64, [3001, 77], 32),                     # G = 8
     (2, 16, 2, 64, [1000, 999], None),                  # contiguous
@@ -110,6 +115,8 @@ OUTLIER = [
     (4, 16, 4, 64, [5000, 3000, 1, 700], 16, 16.0),
     (4, 64, 1, 128, [6000, 3000, 1, 900], 16, 16.0),    # 64-head passes
     (1, 64, 1, 128, [100000], 64, 24.0),                # 64-head passes, split segment
+    (4, 16, 4, 256, [5000, 3000, 1, 700], 16, 16.0),    # D = 256
+    (1, 16, 2, 256, [60000], 64, 24.0),                 # D = 256, split segment
 ]
 
 
@@ -222,7 +229,7 @@ def test_deterministic_repeat():
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
 
 
-@pytest.mark.parametrize("name", ["long_256k", "one_segment_200k", "varlen_small", "mqa_200k"])
+@pytest.mark.parametrize("name", ["long_256k", "one_segment_200k", "varlen_small", "mqa_200k", "d256_100k"])
 def test_split_segments_bitwise_repeat(name):
     """Segments split over many CTAs are merged in a fixed order, so repeated calls
     give bit-identical outputs whatever the CTAs' timing (other work and an L2
@@ -231,6 +238,8 @@ def test_split_segments_bitwise_repeat(name):
         p = workloads.workload(name)
     elif name == "one_segment_200k":
         p = make_problem(name, 1, 16, 1, 128, [200000], seed=21, block_size=64)
+    elif name == "d256_100k":  # D = 256 on the tensor cores
+        p = make_problem(name, 1, 16, 2, 256, [100000], seed=24, block_size=64)
     elif name == "mqa_200k":   # the 64-heads-per-pass kernel
         p = make_problem(name, 2, 64, 1, 128, [200000, 31000], seed=23, block_size=64)
     else:

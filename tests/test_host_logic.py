@@ -46,7 +46,10 @@ def test_plan_reports_the_dispatch():
     assert _plan(1, 32, 32, 128)["kernel"] == cc                      # G = 1
     d64 = _plan(1, 32, 8, 64)
     assert d64["kernel"] == tc and d64["ring_stages"] == 5            # D = 64, deep ring
-    assert _plan(1, 32, 8, 256)["kernel"] == cc                       # D = 256
+    d256 = _plan(1, 32, 8, 256)                                       # D = 256: two slots per tile
+    assert d256["kernel"] == tc and d256["kernel_name"] == "gqa_decode_tc_kernel<NV=4,MQ=0,D=256,F8=0>"
+    assert d256["ring_stages"] == 3
+    assert _plan(1, 32, 16, 256)["kernel"] == cc                      # D = 256, G = 2
     assert _plan(1, 32, 8, 128, bs=48, paged=True, nb=10)["kernel"] == cc  # page size
     assert _plan(1, 32, 8, 128, bs=64, paged=True, nb=10)["box_rows"] == 64
     f8 = _plan(1, 32, 8, 128, kv_fp8=True)
@@ -74,7 +77,10 @@ def test_plan_reports_the_dispatch():
 
 def test_plan_errors():
     with pytest.raises(gq.GqaError) as e:
-        _plan(2, 32, 8, 256, num_splits=2)        # fixed split needs the tensor-core kernel
+        _plan(2, 32, 16, 256, num_splits=2)       # fixed split needs the tensor-core kernel
+    assert e.value.code == 2
+    with pytest.raises(gq.GqaError) as e:
+        _plan(2, 32, 8, 256, qlen=2)              # several query tokens at D = 256: not built
     assert e.value.code == 2
     with pytest.raises(gq.GqaError) as e:
         _plan(2, 32, 8, 128, num_splits=-1)       # auto needs lengths and a device

@@ -30,10 +30,13 @@ def test_selector_estimates_scale_with_work():
 
 
 def test_selector_fixed_split_not_applicable_off_the_tensor_core_shapes():
-    n, (sk, fs) = gq.select_schedule([4096] * 4, 32, 8, 256, 148)  # D = 256
+    n, (sk, fs) = gq.select_schedule([4096] * 4, 32, 16, 256, 148)  # D = 256, G = 2
     assert n == 0 and fs == -1.0 and sk > 0
     n, (_, fs) = gq.select_schedule([4096] * 4, 32, 32, 128, 148)  # G = 1
     assert n == 0 and fs == -1.0
+    # D = 256 with G >= 4 runs on the tensor cores (two ring slots per tile).
+    _, (sk, fs) = gq.select_schedule([4096] * 4, 32, 8, 256, 148)
+    assert sk > 0 and fs > 0
 
 
 def test_selector_covers_head_dim_64_on_the_tensor_cores():
