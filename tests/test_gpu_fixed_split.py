@@ -19,6 +19,10 @@ CASES = [
     (2, 64, 2, [4000, 999], 32, 4),             # G = 32: two head chunks
     (5, 8, 1, [0, 17, 0, 2500, 64], 16, 5),     # empty requests
     (2, 32, 4, [9000, 130], 16, 5, 64),         # D = 64
+    (2, 64, 1, [6000, 999], 32, 1),             # G = 64, one CTA per segment: the 64-head kernel
+    (2, 64, 1, [6000, 999], 32, 4),             # G = 64 split in 4: 16-head passes
+    (2, 16, 4, [9000, 130], 16, 5, 256),        # D = 256
+    (3, 16, 4, [2000, 1, 4100], None, 1, 256),  # D = 256, one CTA per segment
 ]
 
 
@@ -48,13 +52,16 @@ def test_fixed_split_rejects_cuda_core_shapes():
                                   scale=p.scale)
 
 
-@pytest.mark.parametrize("lens,hq,hkv,bs", [
-    ([3000] * 16, 32, 8, None),          # uniform, many segments: one CTA per segment
-    ([40000], 32, 2, 64),                # long context: stream-K
-    ([100, 7000, 1, 2500], 32, 8, 16),   # uneven: stream-K
+@pytest.mark.parametrize("lens,hq,hkv,bs,D", [
+    ([3000] * 16, 32, 8, None, 128),     # uniform, many segments: one CTA per segment
+    ([40000], 32, 2, 64, 128),           # long context: stream-K
+    ([100, 7000, 1, 2500], 32, 8, 16, 128),  # uneven: stream-K
+    ([9000, 3000], 64, 1, 32, 128),      # MQA: the 64-head kernel
+    ([3000] * 40, 64, 2, 16, 128),       # MQA, many segments: one CTA per segment
+    ([20000, 1, 5000], 16, 4, 16, 256),  # D = 256
 ])
-def test_auto_matches_oracle(lens, hq, hkv, bs):
-    p = make_problem("auto", len(lens), hq, hkv, 128, lens, seed=900 + sum(lens), block_size=bs)
+def test_auto_matches_oracle(lens, hq, hkv, bs, D):
+    p = make_problem("auto", len(lens), hq, hkv, D, lens, seed=900 + sum(lens), block_size=bs)
     d = p.to("cuda")
     ws = gq.Workspace(d.q.device)
     out = gq.gqa_decode_auto(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,

@@ -44,7 +44,10 @@ def test_noalloc_matches_gqa_decode_on_consecutive_calls():
     # the scratch are exercised) and a contiguous case with a different shape.
     cases = [make_problem("paged", 4, 32, 8, 128, [20000, 3, 9000, 4097], seed=77,
                           block_size=16, spare_blocks=4),
-             make_problem("contig", 2, 16, 4, 64, [30000, 1000], seed=78)]
+             make_problem("contig", 2, 16, 4, 64, [30000, 1000], seed=78),
+             # the 64-head kernel's larger partial-state slots, and D = 256
+             make_problem("mqa", 2, 64, 1, 128, [30000, 777], seed=81, block_size=64),
+             make_problem("d256", 2, 16, 4, 256, [20000, 300], seed=82, block_size=16)]
     for p in cases:
         d = p.to("cuda")
         expect = gq.gqa_decode(d.q, d.k_cache, d.v_cache, d.block_table, d.seq_lens,
