@@ -1,5 +1,6 @@
 // decode_tc.cuh -- persistent stream-K decode attention on the 5th-generation
-// tensor cores (tcgen05), for groups of G >= 4 query heads per KV head (D = 128 or 64).
+// tensor cores (tcgen05), for groups of G >= 4 query heads per KV head (D = 64, 128 or
+// 256; decode_tc_wide.cuh takes more than 16 heads per KV head at D = 128).
 // The MMAs run M = 128 tokens by N = 16 heads; the softmax threads carry only
 // the NV <= 16 heads that exist.
 //
@@ -163,10 +164,11 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[NV], int lane)
 // never read (zero Q rows in, P left as is: an O column depends on its P column only).
 // MQ: several query tokens per request (causal mask inside them); the one-token
 // decode instantiation carries no mask code.
-// DH: head dimension, 128 or 64.  At 64, BMM1 takes 4 K-steps over the one
+// DH: head dimension, 64, 128 or 256.  At 64, BMM1 takes 4 K-steps over the one
 // 64-column half that is loaded, and BMM2 still runs M = 128 over V^T with rows
 // 64..127 read from a block of zeros (written once, never loaded), so the O rows
-// 64..127 are zero and are not read back.
+// 64..127 are zero and are not read back.  At 256 (one query token, bf16) each
+// tile's two 128-column halves come through two ring slots (TcGeom::SUB).
 // F8: the cache holds FP8 E4M3 (D = 128): the MMAs run kind::f8f6f4 (K = 32) on
 // the cache bytes as loaded.  Q enters as two E4M3 terms, t1 + t2 / 16 (exact for
 // bf16 q after the row's power-of-two scaling), side by side in N = 32 (one term

@@ -96,8 +96,9 @@ GQA_API int gqa_decode_workspace_size(int B, int Hq, int Hkv, int D, int device,
  * requests spread over many SMs (LeanAttention decode tiles digest, sections
  * "Exact softmax that merges piece by piece" and "Hardware-sized work units").
  * A (request, KV head) split across CTAs is merged exactly from the partial
- * states.  On the tensor-core kernel (D = 64 or 128, at least 4 query heads per KV head,
- * pages of 8..128 tokens dividing 128 or multiples of 128, B <= 1024) the launch
+ * states.  On the tensor-core kernels (D = 64, 128 or 256, at least 4 query heads
+ * per KV head -- more than 16 at D = 128 run 64 heads per pass -- pages of 8..128
+ * tokens dividing 128 or multiples of 128, B <= 1024) the launch
  * is cooperative: every CTA is resident, and the owners of a split segment wait
  * (bounded, GQA_DEV_TIMEOUT on expiry) for one another and merge one slice of its
  * outputs each; the launch fails with GQA_ERR_CUDA rather than run when the grid
