@@ -318,7 +318,10 @@ class Runner:
         self.stream = torch.cuda.current_stream(dev)
         self.lens_host = p.seq_lens.to(torch.int32).contiguous()
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        self.mode = "stream-K" if self.fp8 else args.schedule
+        # FP8 caches: gqa_decode_fp8_auto, or gqa_decode_fp8 (stream-K) for any other
+        # --schedule (the fixed-split comparator has no FP8 form).
+        self.mode = ("auto" if args.schedule == "auto" else "streamk") if self.fp8 \
+            else args.schedule
         if self.mode == "fixed":
             segs = p.B * p.Hkv * -(-p.G // 16)
             self.splits = args.splits if args.splits > 0 else max(1, -(-sms // segs))
@@ -337,7 +340,10 @@ class Runner:
     def step(self):
         gq, d, p = self.gq, self.d, self.p
         kw = dict(out=self.out, scale=p.scale, workspace=self.ws, stream=self.stream)
-        if self.fp8:
+        if self.fp8 and self.mode == "auto":
+            gq.gqa_decode_fp8_auto(d.q, d.k_cache, d.v_cache, self.k_scale, self.v_scale,
+                                   d.block_table, d.seq_lens, self.lens_host, **kw)
+        elif self.fp8:
             gq.gqa_decode_fp8(d.q, d.k_cache, d.v_cache, self.k_scale, self.v_scale,
                               d.block_table, d.seq_lens, **kw)
         elif self.mode == "fixed":

@@ -34,8 +34,8 @@ EXPORTED = ("gqa_decode_workspace_size", "gqa_decode", "gqa_decode_states", "gqa
             "gqa_status", "gqa_decode_host_buffer_bytes", "gqa_decode_host", "gqa_error_string",
             "gqa_decode_noalloc", "gqa_decode_fixed_split_workspace_size",
             "gqa_decode_fixed_split", "gqa_select_schedule", "gqa_decode_auto",
-            "gqa_decode_multi", "gqa_decode_fp8", "gqa_decode_timeline", "gqa_decode_plan",
-            "gqa_set_wait_limit", "gqa_stream_floor")
+            "gqa_decode_multi", "gqa_decode_fp8", "gqa_decode_fp8_auto", "gqa_decode_timeline",
+            "gqa_decode_plan", "gqa_set_wait_limit", "gqa_stream_floor")
 GQA_ERR_SCRATCH_LIMIT = 6
 TIMELINE_COLS = 8  # values per CTA row of gqa_decode_timeline
 KERNEL_TENSOR_CORE = 1
@@ -86,6 +86,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_decode_auto.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, SZ, P]
     lib.gqa_decode_multi.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, P, SZ, P]
     lib.gqa_decode_fp8.argtypes = [P, P, P, F, F, P, P, P, I, I, I, I, I, F, I, I, P, SZ, P]
+    lib.gqa_decode_fp8_auto.argtypes = [P, P, P, F, F, P, P, P, P, I, I, I, I, I, F, I, I, P, SZ,
+                                        P]
     lib.gqa_decode_timeline.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, I, P, I,
                                         ctypes.POINTER(I), P, SZ, P]
     lib.gqa_decode_plan.argtypes = [I, I, I, I, I, I, I, I, I, I, P, I, ctypes.POINTER(_Plan)]
@@ -98,7 +100,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                  "gqa_merge_states", "gqa_status", "gqa_decode_host",
                  "gqa_decode_fixed_split_workspace_size", "gqa_decode_fixed_split",
                  "gqa_select_schedule", "gqa_decode_auto", "gqa_decode_multi",
-                 "gqa_decode_fp8", "gqa_decode_plan", "gqa_decode_noalloc",
+                 "gqa_decode_fp8", "gqa_decode_fp8_auto", "gqa_decode_plan", "gqa_decode_noalloc",
                  "gqa_decode_timeline", "gqa_set_wait_limit", "gqa_stream_floor"):
         getattr(lib, name).restype = I
     _lib = lib
@@ -423,6 +425,43 @@ def gqa_decode_fp8(q, k8, v8, k_scale: float, v_scale: float, block_table, seq_l
                                 _ptr(block_table), _ptr(seq_lens), _ptr(out), B, Hq, Hkv, D, bs,
                                 scale, mb, nb, _ptr(buf), buf.numel(), _stream_ptr(stream))
     _check("gqa_decode_fp8", rc)
+    return out
+
+
+def gqa_decode_fp8_auto(q, k8, v8, k_scale: float, v_scale: float, block_table, seq_lens,
+                        seq_lens_host=None, out=None, scale=None,
+                        workspace: Optional[Workspace] = None, stream=None) -> torch.Tensor:
+    """gqa_decode_fp8 with the runtime schedule selection of gqa_decode_auto;
+    seq_lens_host: int32 CPU tensor (a copy of seq_lens; taken from the device, with a
+    sync, when omitted)."""
+    lib = load_library()
+    k8 = k8.view(torch.uint8) if k8.dtype != torch.uint8 else k8
+    v8 = v8.view(torch.uint8) if v8.dtype != torch.uint8 else v8
+    B, Hq, Hkv, D, bs, mb, nb = _shape(q, k8, block_table)
+    dev = q.device
+    _require(q, "q", torch.bfloat16, dev)
+    _require(k8, "k_cache", torch.uint8, dev)
+    _require(v8, "v_cache", torch.uint8, dev)
+    _require(seq_lens, "seq_lens", torch.int32, dev)
+    if block_table is not None:
+        _require(block_table, "block_table", torch.int32, dev)
+    host = seq_lens.cpu() if seq_lens_host is None else seq_lens_host
+    if host.device.type != "cpu" or host.dtype != torch.int32 or not host.is_contiguous() \
+            or host.numel() != B:
+        raise ValueError("seq_lens_host must be a contiguous int32 CPU tensor of length B")
+    if out is None:
+        out = torch.empty_like(q)
+    _require(out, "out", torch.bfloat16, dev)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    ws = default_workspace(dev) if workspace is None else workspace
+    buf = ws.get(workspace_size(B, Hq, Hkv, D, dev.index))
+    with torch.cuda.device(dev):
+        rc = lib.gqa_decode_fp8_auto(_ptr(q), _ptr(k8), _ptr(v8), float(k_scale),
+                                     float(v_scale), _ptr(block_table), _ptr(seq_lens),
+                                     ctypes.c_void_p(host.data_ptr()), _ptr(out), B, Hq, Hkv, D,
+                                     bs, scale, mb, nb, _ptr(buf), buf.numel(),
+                                     _stream_ptr(stream))
+    _check("gqa_decode_fp8_auto", rc)
     return out
 
 

@@ -600,9 +600,10 @@ int run_decode(bool states, const void *q, const void *k_cache, const void *v_ca
 using namespace gqa;
 
 // The schedule selector (gqa_select_schedule, gqa_decode_auto): fixed split
-// with 1, 2, 4, ..., max_splits chunks against stream-K.
+// with 1, 2, 4, ..., max_splits chunks against stream-K.  kv_fp8: an FP8 cache,
+// whose tiles are half the bytes and which runs 16-head passes only.
 int select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int num_sms,
-                    int max_splits, int *num_splits, float *est_us)
+                    int max_splits, int *num_splits, float *est_us, bool kv_fp8 = false)
 {
     if (!num_splits || num_sms <= 0 || (B > 0 && !seq_lens))
         return GQA_ERR_INVALID_ARG;
@@ -619,10 +620,10 @@ int select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int 
     // several chunks runs 16-head passes.
     const int64_t units16 = (int64_t)Hkv * (tc ? (G + TcCfg::NP - 1) / TcCfg::NP
                                                : (G + head_chunk(G) - 1) / head_chunk(G));
-    const int64_t units = tc && tc_wide(G, D, false, false, 0)
+    const int64_t units = tc && tc_wide(G, D, false, kv_fp8, 0)
                               ? (int64_t)Hkv * ((G + TcWide::NP - 1) / TcWide::NP) : units16;
     // Microseconds per 128-token K+V tile for a CTA while `active` CTAs stream.
-    const double tile_bytes = 4.0 * TcCfg::T * D;
+    const double tile_bytes = (kv_fp8 ? 2.0 : 4.0) * TcCfg::T * D;
     auto tile_us = [&](int64_t active) {
         const double gbs = std::min(SCHED_SM_GBS, SCHED_HBM_GBS / (double)std::max<int64_t>(active, 1));
         return tile_bytes / (gbs * 1e3);
@@ -705,13 +706,15 @@ int select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int 
 // kernel does not take (a page size its TMA boxes cannot tile, too many rows
 // for a tensor map, a small group) stays on stream-K.
 static int auto_splits(int B, int Hq, int Hkv, int D, int block_size, bool paged, int num_blocks,
-                       const int32_t *seq_lens_host, int sms, int &ns)
+                       const int32_t *seq_lens_host, int sms, int &ns, bool kv_fp8 = false)
 {
     ns = 0;
-    int rc = select_schedule(B, Hq, Hkv, D, seq_lens_host, sms, 1, &ns, nullptr);
+    int rc = select_schedule(B, Hq, Hkv, D, seq_lens_host, sms, 1, &ns, nullptr, kv_fp8);
     if (rc)
         return rc;
     if (ns && !tc_applicable(false, B, Hkv, D, block_size, paged, num_blocks, Hq / Hkv))
+        ns = 0;
+    if (kv_fp8 && D != 128)  // FP8 runs on the tensor cores at D = 128 only; elsewhere stream-K
         ns = 0;
     return GQA_OK;
 }
@@ -866,7 +869,7 @@ int gqa_decode_plan(int B, int Hq, int Hkv, int D, int block_size, int paged, in
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
             return GQA_ERR_CUDA;
         if ((rc = auto_splits(B, Hq, Hkv, D, block_size, paged != 0, num_blocks, seq_lens_host, sms,
-                              ns)))
+                              ns, kv_fp8 != 0)))
             return rc;
     }
     ns = ns < 0 ? 0 : ns;
@@ -935,6 +938,29 @@ int gqa_decode_fp8(const void *q, const void *k_cache, const void *v_cache, floa
     return run_decode(false, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, out,
                       nullptr, nullptr, nullptr, B, Hq, Hkv, D, block_size, scale,
                       max_blocks_per_seq, num_blocks, workspace, workspace_bytes, stream, 0, 1,
+                      true, k_scale, v_scale);
+}
+
+int gqa_decode_fp8_auto(const void *q, const void *k_cache, const void *v_cache, float k_scale,
+                        float v_scale, const int32_t *block_table, const int32_t *seq_lens,
+                        const int32_t *seq_lens_host, void *out, int B, int Hq, int Hkv, int D,
+                        int block_size, float scale, int max_blocks_per_seq, int num_blocks,
+                        void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || k_scale <= 0.f || v_scale <= 0.f)
+        return GQA_ERR_INVALID_ARG;
+    int dev = 0, sms = 0, rc;
+    if ((rc = current_device(dev)))
+        return rc;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    int ns = 0;
+    if ((rc = auto_splits(B, Hq, Hkv, D, block_size, block_table != nullptr, num_blocks,
+                          seq_lens_host, sms, ns, true)))
+        return rc;
+    return run_decode(false, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, out,
+                      nullptr, nullptr, nullptr, B, Hq, Hkv, D, block_size, scale,
+                      max_blocks_per_seq, num_blocks, workspace, workspace_bytes, stream, ns, 1,
                       true, k_scale, v_scale);
 }
 

@@ -207,8 +207,9 @@ GQA_API int gqa_decode_auto(const void *q, const void *k_cache, const void *v_ca
  *                  0: a contiguous cache (block_size = per-request capacity)
  *   qlen           query tokens per request (1: gqa_decode; > 1: gqa_decode_multi)
  *   kv_fp8         1: an FP8 E4M3 cache (gqa_decode_fp8; qlen must be 1)
- *   num_splits     -1: the choice gqa_decode_auto makes (needs seq_lens_host and
- *                  a device); 0: gqa_decode (stream-K); n > 0: gqa_decode_fixed_split
+ *   num_splits     -1: the choice gqa_decode_auto (gqa_decode_fp8_auto) makes (needs
+ *                  seq_lens_host and a device); 0: stream-K; n > 0:
+ *                  gqa_decode_fixed_split
  *   seq_lens_host  HOST int32 [B] or NULL; with it, plan->tiles is filled in
  *   device         CUDA device for the grid and workspace size; < 0: no device
  *                  query (grid = -1 for stream-K, workspace_bytes = 0)
@@ -222,7 +223,7 @@ GQA_API int gqa_decode_auto(const void *q, const void *k_cache, const void *v_ca
 #define GQA_KERNEL_CUDA_CORE 2    /* gqa_decode_simt_kernel: packed FMAs on CUDA cores */
 typedef struct gqa_plan {
     int kernel;              /* GQA_KERNEL_*, 0 when nothing is launched */
-    int heads_per_pass;      /* query rows one pass carries (tensor cores: 4, 8, 16) */
+    int heads_per_pass;      /* query rows one pass carries (tensor cores: 4, 8, 16, 64) */
     int head_chunks;         /* passes per KV head */
     int num_splits;          /* 0: stream-K; n > 0: fixed split into n chunks */
     int grid;                /* CTAs of the decode kernel (-1: no device given) */
@@ -281,6 +282,21 @@ GQA_API int gqa_decode_fp8(const void *q, const void *k_cache, const void *v_cac
                            void *out, int B, int Hq, int Hkv, int D, int block_size, float scale,
                            int max_blocks_per_seq, int num_blocks, void *workspace,
                            size_t workspace_bytes, void *stream);
+
+/*
+ * gqa_decode_fp8 with gqa_decode_auto's runtime selection (stream-K, or one CTA
+ * per (request, KV head) when that already fills the GPU), given a HOST copy of
+ * the lengths, seq_lens_host int32 [B] (read during the call only).  The cost
+ * model takes the FP8 tile size (one byte per element) and the FP8 kernel's
+ * 16-head passes.  FP8 caches off the tensor cores (D != 128) always take
+ * stream-K.  Arguments, workspace, results and errors otherwise as gqa_decode_fp8.
+ */
+GQA_API int gqa_decode_fp8_auto(const void *q, const void *k_cache, const void *v_cache,
+                                float k_scale, float v_scale, const int32_t *block_table,
+                                const int32_t *seq_lens, const int32_t *seq_lens_host, void *out,
+                                int B, int Hq, int Hkv, int D, int block_size, float scale,
+                                int max_blocks_per_seq, int num_blocks, void *workspace,
+                                size_t workspace_bytes, void *stream);
 
 /*
  * Partial softmax states of every query row over the key range

@@ -1,6 +1,6 @@
-"""GPU parity of the FP8 E4M3 cache path (gqa_decode_fp8) against the fp64 oracle
-on the same E4M3 bytes and scales: the tensor-core kernel (D = 128, G >= 4) and
-the CUDA-core kernel (the other shapes)."""
+"""GPU parity of the FP8 E4M3 cache path (gqa_decode_fp8, gqa_decode_fp8_auto)
+against the fp64 oracle on the same E4M3 bytes and scales: the tensor-core kernel
+(D = 128, G >= 4) and the CUDA-core kernel (the other shapes)."""
 import pytest
 import torch
 
@@ -50,3 +50,55 @@ def test_fp8_llama3_shape_full():
                             scale=p.scale).cpu()
     ref = oracle.gqa_decode_fp8(p.q, k8, v8, ks, vs, p.block_table, p.seq_lens, p.scale)
     parity(out, ref, "llama3_8b_fp8", bf16_scaled=True)
+
+
+AUTO_CASES = [
+    # B, Hq, Hkv, D, lens, block_size
+    (4, 32, 8, 128, [3000, 129, 2048, 7], 16),  # G = 4, uneven lengths
+    (1, 32, 2, 128, [40000], 64),           # one long request: stream-K, segments merged
+    (2, 64, 1, 128, [30000, 500], 64),      # G = 64: four 16-head passes (no wide kernel)
+    (3, 4, 2, 64, [128, 127, 900], 8),      # D = 64: the CUDA-core kernel, stream-K
+]
+
+
+@pytest.mark.parametrize("case", AUTO_CASES, ids=lambda c: f"B{c[0]}_Hq{c[1]}_Hkv{c[2]}_D{c[3]}")
+def test_fp8_auto_matches_oracle_and_its_plan(case):
+    """gqa_decode_fp8_auto: the schedule gqa_decode_plan reports for the FP8 cache
+    (kv_fp8, num_splits = -1) and the oracle's result on the same E4M3 bytes."""
+    B, Hq, Hkv, D, lens, bs = case
+    p = make_problem("fp8a", B, Hq, Hkv, D, lens, seed=900 + sum(lens) % 97 + D, block_size=bs,
+                     spare_blocks=2, key_outlier_frac=0.01)
+    k8, v8, ks, vs = fp8_caches(p)
+    d = p.to("cuda")
+    host = p.seq_lens.to(torch.int32).contiguous()
+    plan = gq.decode_plan(B, Hq, Hkv, D, bs, True, p.num_blocks, kv_fp8=True, num_splits=-1,
+                          seq_lens_host=host, device=0)
+    if D == 128:
+        assert plan["kernel"] == gq.KERNEL_TENSOR_CORE and plan["heads_per_pass"] == min(16, Hq // Hkv)
+    else:
+        assert plan["kernel"] == gq.KERNEL_CUDA_CORE and plan["num_splits"] == 0
+    if B == 1:  # two segments on 148 SMs: stream-K
+        assert plan["num_splits"] == 0
+    ws = gq.Workspace(d.q.device)
+    out = gq.gqa_decode_fp8_auto(d.q, k8.cuda(), v8.cuda(), ks, vs, d.block_table, d.seq_lens,
+                                 host, scale=p.scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    ref = oracle.gqa_decode_fp8(p.q, k8, v8, ks, vs, p.block_table, p.seq_lens, p.scale)
+    parity(out.cpu(), ref, f"auto {case}", bf16_scaled=True)
+
+
+def test_fp8_auto_llama3_shape_full():
+    """The full-size FP8 step through gqa_decode_fp8_auto (one CTA per (request, KV
+    head), the schedule the bench times): all 512 query rows against the oracle."""
+    p = workloads.workload("llama3_8b_fp8")
+    k8, v8, ks, vs = fp8_caches(p)
+    d = p.to("cuda")
+    host = p.seq_lens.to(torch.int32).contiguous()
+    plan = gq.decode_plan(p.B, p.Hq, p.Hkv, p.D, p.block_size, p.paged, p.num_blocks,
+                          kv_fp8=True, num_splits=-1, seq_lens_host=host, device=0)
+    assert plan["num_splits"] == 1 and plan["kernel_name"].endswith("F8=1>")
+    out = gq.gqa_decode_fp8_auto(d.q, k8.cuda(), v8.cuda(), ks, vs, d.block_table, d.seq_lens,
+                                 host, scale=p.scale).cpu()
+    ref = oracle.gqa_decode_fp8(p.q, k8, v8, ks, vs, p.block_table, p.seq_lens, p.scale)
+    parity(out, ref, "llama3_8b_fp8 auto", bf16_scaled=True)
