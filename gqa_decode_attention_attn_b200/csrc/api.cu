@@ -423,7 +423,7 @@ int make_plan(bool states, int B, int Hq, int Hkv, int D, int block_size, bool p
         pl.hch = (pl.R + TcCfg::NP - 1) / TcCfg::NP;
         pl.nv = pl.R <= 4 ? 4 : (pl.R <= 8 ? 8 : 16);
         pl.threads = TcCfg::THREADS;
-        pl.tile_tokens = TcCfg::T;
+        pl.tile_tokens = fp8 ? TcGeom<128, true>::TILE : TcCfg::T;
         pl.stages = fp8 ? TcGeom<128, true>::STAGES
                         : (D == 64 ? TcGeom<64>::STAGES : D == 256 ? TcGeom<256>::STAGES : TcGeom<128>::STAGES);
         pl.smem = tc_smem_bytes(D, B, fp8);
@@ -601,7 +601,8 @@ using namespace gqa;
 
 // The schedule selector (gqa_select_schedule, gqa_decode_auto): fixed split
 // with 1, 2, 4, ..., max_splits chunks against stream-K.  kv_fp8: an FP8 cache,
-// whose tiles are half the bytes and which runs 16-head passes only.
+// whose tensor-core tiles are 256 tokens of one byte per element and which runs
+// 16-head passes only.
 int select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int num_sms,
                     int max_splits, int *num_splits, float *est_us, bool kv_fp8 = false)
 {
@@ -623,7 +624,8 @@ int select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int 
     const int64_t units = tc && tc_wide(G, D, false, kv_fp8, 0)
                               ? (int64_t)Hkv * ((G + TcWide::NP - 1) / TcWide::NP) : units16;
     // Microseconds per 128-token K+V tile for a CTA while `active` CTAs stream.
-    const double tile_bytes = (kv_fp8 ? 2.0 : 4.0) * TcCfg::T * D;
+    const int Tt = kv_fp8 ? TcGeom<128, true>::TILE : TcCfg::T;  // tokens per LeanTile
+    const double tile_bytes = (kv_fp8 ? 2.0 : 4.0) * Tt * D;
     auto tile_us = [&](int64_t active) {
         const double gbs = std::min(SCHED_SM_GBS, SCHED_HBM_GBS / (double)std::max<int64_t>(active, 1));
         return tile_bytes / (gbs * 1e3);
@@ -631,7 +633,7 @@ int select_schedule(int B, int Hq, int Hkv, int D, const int32_t *seq_lens, int 
     std::vector<int64_t> nb(B);
     int64_t W = 0;
     for (int b = 0; b < B; ++b) {
-        nb[b] = ((int64_t)seq_lens[b] + TcCfg::T - 1) / TcCfg::T;
+        nb[b] = ((int64_t)seq_lens[b] + Tt - 1) / Tt;
         W += units * nb[b];
     }
     const int64_t P = num_sms;

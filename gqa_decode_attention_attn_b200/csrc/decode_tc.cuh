@@ -62,11 +62,15 @@ static_assert(TcCfg::O_COL + 2 * TcCfg::NO <= TcCfg::TMEM_COLS, "tensor memory c
 
 // Shared-memory layout for head dimension D (F8: an FP8 E4M3 cache, D = 128).  A
 // ring slot holds one K or V tile of 128-byte boxes (one box row per token):
-// two boxes at bf16 D = 128 (32 KB, three slots per ring), one at bf16 D = 64 and
-// at FP8 D = 128 (16 KB, five slots per ring, so that as many bytes stay in
-// flight).  At bf16 D = 64 BMM2 still runs M = 128 over V^T; its rows 64..127
-// come from one 16 KB block of zeros shared by every V slot (the operand's
-// leading-byte offset points there).  At 8 bits one box row spans all 128 rows
+// two boxes at bf16 D = 128 (32 KB, three slots per ring), one at bf16 D = 64
+// (16 KB, five slots per ring, so that as many bytes stay in flight).  FP8 tiles
+// are 256 tokens (TH = 2 halves of 128): one box row per token, 32 KB, three
+// slots per ring, so that a pipeline step moves 64 KB as at bf16 D = 128; BMM1
+// writes each half's scores to its own TMEM columns, BMM2 runs K = 256 tokens,
+// each softmax thread carries two token rows, and Q has one buffer (the rings and
+// the 12 KB P buffers then fit).  At bf16 D = 64 BMM2 still runs M = 128 over
+// V^T; its rows 64..127 come from one 16 KB block of zeros shared by every V slot
+// (the operand's leading-byte offset points there).  At 8 bits one box row spans all 128 rows
 // of V^T.  At bf16 D = 256 a tile's two 128-column halves are two consecutive
 // slots of the 32 KB rings (SUB = 2): BMM1 accumulates S over both, BMM2 writes
 // each half's O rows to its own TMEM columns; Q (8 KB) has one buffer, so that the
@@ -75,17 +79,24 @@ template <int D, bool F8 = false>
 struct TcGeom {
     static_assert(!F8 || D == 128, "FP8 tiles are built for D = 128");
     static constexpr int SUB = D == 256 ? 2 : 1;           // ring slots per tile
+    // 128-token halves per tile: FP8 tiles are 256 tokens (64 KB of K and V, as a
+    // bf16 tile at D = 128), so that each pipeline step moves as many bytes.
+    static constexpr int TH = F8 ? 2 : 1;
+    static constexpr int TILE = TcCfg::T * TH;             // tokens per tile
     static constexpr int BOXES = (F8 ? D : 2 * D / SUB) / 128;  // 128-byte boxes per token row of a slot
     static constexpr bool NEED_ZERO = !F8 && D == 64;
-    static constexpr int STAGES = BOXES == 1 ? 5 : 3;      // slots per ring (K ring, V ring)
-    static constexpr int SLOT_BYTES = BOXES * TcCfg::BOX_BYTES;
-    static constexpr int QBUFS = D == 256 ? 1 : 2;         // Q buffers
+    static constexpr int STAGES = (BOXES == 1 && !F8) ? 5 : 3;  // slots per ring (K ring, V ring)
+    static constexpr int SLOT_BYTES = BOXES * TcCfg::BOX_BYTES * TH;
+    static constexpr int QBUFS = (D == 256 || F8) ? 1 : 2;  // Q buffers
+    // P buffer: bf16 hi | lo for 16 heads per 128 tokens, or FP8's three E4M3 terms
+    // (three 128-byte core matrices per 8 tokens) for a 256-token tile.
+    static constexpr int PBUF = F8 ? (TILE / 8) * 3 * 128 : TcCfg::PBUF_BYTES;
     static constexpr int QBUF = (D == 256 ? 2 : 1) * TcCfg::QBUF_BYTES;
     static constexpr size_t V_RING_OFF = (size_t)STAGES * SLOT_BYTES;
     static constexpr size_t ZERO_OFF = 2 * V_RING_OFF;                 // NEED_ZERO only
     static constexpr size_t Q_OFF = ZERO_OFF + (NEED_ZERO ? TcCfg::BOX_BYTES : 0);
     static constexpr size_t P_OFF = Q_OFF + QBUFS * QBUF;
-    static constexpr size_t BAR_OFF = P_OFF + 2 * TcCfg::PBUF_BYTES;
+    static constexpr size_t BAR_OFF = P_OFF + 2 * PBUF;
     static constexpr int NBAR = 4 * STAGES + 16;
     static constexpr size_t MISC_OFF = BAR_OFF + NBAR * 8;
     // floats: tile maxima [2][4][NP], piece sums [4][NP], merge maxima [NP], then
@@ -97,7 +108,7 @@ struct TcGeom {
     // Segment merge: the owner list (<= 512 ints) in the P buffers; the gathered
     // slices, at most E + 4 no + 3 no (E / D + 2) + 2 NP floats (E <= NP x D
     // outputs, no <= 512 owners, slices rounded to 4 elements), in the rings.
-    static_assert(512 * 4 <= 2 * TcCfg::PBUF_BYTES, "owner list must fit in the P buffers");
+    static_assert(512 * 4 <= 2 * PBUF, "owner list must fit in the P buffers");
     static_assert((16 * D + 4 * 512 + 3 * 512 * (16 + 2) + 32) * 4 <= 2 * V_RING_OFF,
                   "gathered slices must fit in the rings");
     static_assert(STAGES <= 8, "stage_n and stage_bad hold 8 slots");
@@ -169,8 +180,8 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[NV], int lane)
 // 64..127 read from a block of zeros (written once, never loaded), so the O rows
 // 64..127 are zero and are not read back.  At 256 (one query token, bf16) each
 // tile's two 128-column halves come through two ring slots (TcGeom::SUB).
-// F8: the cache holds FP8 E4M3 (D = 128): the MMAs run kind::f8f6f4 (K = 32) on
-// the cache bytes as loaded.  Q enters as two E4M3 terms, t1 + t2 / 16 (exact for
+// F8: the cache holds FP8 E4M3 (D = 128), in 256-token tiles (TcGeom::TH): the
+// MMAs run kind::f8f6f4 (K = 32) on the cache bytes as loaded.  Q enters as two E4M3 terms, t1 + t2 / 16 (exact for
 // bf16 q after the row's power-of-two scaling), side by side in N = 32 (one term
 // per 16 columns); P as three, t1 + t2 / 16 + t3 / 256, in N = 48: two terms
 // leave the weights of the keys that dominate a row 8 significant bits, whose
@@ -184,13 +195,15 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
 {
     using C = TcCfg;
     using L = TcGeom<DH, F8>;
-    constexpr int S = L::STAGES, NP = C::NP, D = DH, T = C::T;
+    constexpr int TH = L::TH;                       // 128-token halves per tile
+    constexpr int S = L::STAGES, NP = C::NP, D = DH, T = L::TILE;
     constexpr int HALVES = L::BOXES;  // 128-byte boxes loaded per token row of a slot
     constexpr int SUB = L::SUB;       // ring slots per tile (2 at D = 256)
     constexpr int QH = D / 64;        // 64-column halves of a bf16 Q row
     constexpr int QBUFS = L::QBUFS;
     constexpr int SW = F8 ? 2 * NP : NP;            // S columns per buffer
-    constexpr int OC = F8 ? 4 * NP : C::O_COL;      // first O column
+    constexpr int SWB = SW * TH;                     // S columns per buffer, all halves
+    constexpr int OC = F8 ? 2 * SWB : C::O_COL;     // first O column
     constexpr int KSTEP = F8 ? 32 : 16;             // MMA K per instruction
     // FP8 P: per 8-token group, two 128-byte core matrices along N (16 E4M3 heads
     // per 16-byte row: term 1, then term 2).
@@ -198,7 +211,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
     constexpr int P8_LBO = 3 * 128;                 // FP8 P: three core matrices per 8 tokens
     constexpr int TMEM_COLS = (F8 || SUB == 2) ? 256 : C::TMEM_COLS;
     static_assert(OC + 2 * NO * SUB <= TMEM_COLS, "tensor memory columns");
-    static_assert(!F8 || (T / 8) * P8_LBO <= C::PBUF_BYTES, "FP8 P buffer");
+    static_assert(!F8 || (T / 8) * P8_LBO <= L::PBUF, "FP8 P buffer");
     static_assert(D == 64 || D == 128 || (D == 256 && !MQ && !F8), "head dimension");
     constexpr int SLOT = slot_floats(NV, D);
     constexpr int LPH = 32 / NV;  // lanes per head after a transposed warp reduction
@@ -506,16 +519,20 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                         tc_fence_after_sync();
                         const uint32_t ka = ring_a + (uint32_t)(s * L::SLOT_BYTES);
 #pragma unroll
-                        for (int kk = 0; kk < D / SUB / KSTEP; ++kk) {
-                            // 32 bytes of every row per instruction: 16 bf16 or 32 E4M3 elements.
-                            const uint32_t off = (uint32_t)((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32);
-                            const uint32_t qoff = (uint32_t)((2 * sub + (kk >> 2)) * NP * 128 + (kk & 3) * 32);
-                            const uint64_t ad = umma_smem_desc(ka + off, 16, 1024, SMEM_LAYOUT_SW128);
-                            const uint64_t bd = umma_smem_desc(qa + qoff, 16, 1024, SMEM_LAYOUT_SW128);
-                            if constexpr (F8)
-                                umma_e4m3(tbase + (uint32_t)(C::S_COL + b * SW), ad, bd, idesc1, kk > 0);
-                            else
-                                umma_bf16(tbase + (uint32_t)(C::S_COL + b * SW), ad, bd, idesc1, sub > 0 || kk > 0);
+                        for (int th = 0; th < TH; ++th) {
+                            // token half th: rows 128 th .. of the slot, into its own S columns
+#pragma unroll
+                            for (int kk = 0; kk < D / SUB / KSTEP; ++kk) {
+                                // 32 bytes of every row per instruction: 16 bf16 or 32 E4M3 elements.
+                                const uint32_t off = (uint32_t)(th * C::BOX_BYTES + (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32);
+                                const uint32_t qoff = (uint32_t)((2 * sub + (kk >> 2)) * NP * 128 + (kk & 3) * 32);
+                                const uint64_t ad = umma_smem_desc(ka + off, 16, 1024, SMEM_LAYOUT_SW128);
+                                const uint64_t bd = umma_smem_desc(qa + qoff, 16, 1024, SMEM_LAYOUT_SW128);
+                                if constexpr (F8)
+                                    umma_e4m3(tbase + (uint32_t)(C::S_COL + b * SWB + th * SW), ad, bd, idesc1, kk > 0);
+                                else
+                                    umma_bf16(tbase + (uint32_t)(C::S_COL + b * SWB), ad, bd, idesc1, sub > 0 || kk > 0);
+                            }
                         }
                         if (sub == SUB - 1)
                             umma_commit(&s_full[b]);
@@ -556,7 +573,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                         piece_ends = itp.seg0 != segp;
                         segp = itp.seg0;
                     }
-                    const uint32_t pa = p_a + (uint32_t)(b * C::PBUF_BYTES);
+                    const uint32_t pa = p_a + (uint32_t)(b * L::PBUF);
 #pragma unroll
                     for (int sub = 0; sub < SUB && ok; ++sub) {
                         // O^T rows of head-dimension half `sub` (D = 256) in their own columns.
@@ -874,7 +891,7 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             }
 
             const int s = (k * SUB) % S, b = k & 1;  // the tile's (first) V slot
-            float sc[NV];
+            float sc[TH][NV];
             int n = 0;
             bool have_v = ok;
 #pragma unroll
@@ -886,14 +903,17 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 poisoned |= stage_bad[s] != 0;
                 tc_fence_after_sync();
                 if constexpr (F8) {
-                    float s2[NV];
-                    tmem_load<NV>(tlane + (uint32_t)(C::S_COL + b * SW), sc);
-                    tmem_load<NV>(tlane + (uint32_t)(C::S_COL + b * SW + NP), s2);
 #pragma unroll
-                    for (int g = 0; g < NV; ++g)
-                        sc[g] = fmaf(s2[g], 1.f / 16.f, sc[g]);  // the second Q term carries x16
+                    for (int th = 0; th < TH; ++th) {
+                        float s2[NV];
+                        tmem_load<NV>(tlane + (uint32_t)(C::S_COL + b * SWB + th * SW), sc[th]);
+                        tmem_load<NV>(tlane + (uint32_t)(C::S_COL + b * SWB + th * SW + NP), s2);
+#pragma unroll
+                        for (int g = 0; g < NV; ++g)
+                            sc[th][g] = fmaf(s2[g], 1.f / 16.f, sc[th][g]);  // the second Q term carries x16
+                    }
                 } else {
-                    tmem_load<NV>(tlane + (uint32_t)(C::S_COL + b * SW), sc);
+                    tmem_load<NV>(tlane + (uint32_t)(C::S_COL + b * SWB), sc[0]);
                 }
                 tc_fence_before_sync();
                 if (k == 0 && stid == 0 && p.timeline)
@@ -904,14 +924,19 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             }
             mbar_arrive(&s_free[b]);
             flush_fold();  // before this tile may rescale acc again
-            const bool valid = ti < n;
+            bool valid[TH];
+#pragma unroll
+            for (int th = 0; th < TH; ++th)
+                valid[th] = ti + 128 * th < n;
             // Several query tokens (qlen > 1): query row r is token r / G at position
             // L - qlen + r / G and sees keys up to its own position, so a key `past`
             // places beyond L - qlen is hidden from the rows of tokens before it.
-            bool see[NV];
+            bool see[TH][NV];
 #pragma unroll
-            for (int g = 0; g < NV; ++g)
-                see[g] = valid;
+            for (int th = 0; th < TH; ++th)
+#pragma unroll
+                for (int g = 0; g < NV; ++g)
+                    see[th][g] = valid[th];
             if (MQ) {
                 if (it.b != len_b) {
                     len_b = it.b;
@@ -923,27 +948,33 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 if (past > 0) {  // only the last qlen - 1 keys of a request
 #pragma unroll
                     for (int g = 0; g < NV; ++g)
-                        see[g] = see[g] && past <= (it.hc * NP + g) / G;
+                        see[0][g] = see[0][g] && past <= (it.hc * NP + g) / G;
                 }
             }
             // x = scaled score relative to the reference.  While no score of the tile
             // exceeds its reference by more than 2^LAZY, P = 2^x <= 2^LAZY is used as
             // is and nothing is rescaled: one barrier-OR decides that for the CTA.
-            float x[NV];
+            float x[TH][NV];
             float xmax = -INFINITY;
 #pragma unroll
-            for (int g = 0; g < NV; ++g) {
-                x[g] = see[g] ? fmaf(sc[g], qsc(g), -m_ref[g]) : -INFINITY;
-                xmax = fmaxf(xmax, x[g]);
-            }
+            for (int th = 0; th < TH; ++th)
+#pragma unroll
+                for (int g = 0; g < NV; ++g) {
+                    x[th][g] = see[th][g] ? fmaf(sc[th][g], qsc(g), -m_ref[g]) : -INFINITY;
+                    xmax = fmaxf(xmax, x[th][g]);
+                }
             const bool moved = named_barrier_or(1, 128, !(xmax <= C::LAZY));
             float alpha[NV];
             if (moved) {
                 // Tile maximum per head over the 128 tokens: warp, then the 4 warps.
                 float mx[NV];
 #pragma unroll
-                for (int g = 0; g < NV; ++g)
-                    mx[g] = see[g] ? sc[g] * qsc(g) : -INFINITY;
+                for (int g = 0; g < NV; ++g) {
+                    mx[g] = see[0][g] ? sc[0][g] * qsc(g) : -INFINITY;
+#pragma unroll
+                    for (int th = 1; th < TH; ++th)
+                        mx[g] = fmaxf(mx[g], see[th][g] ? sc[th][g] * qsc(g) : -INFINITY);
+                }
                 const float wmax = warp_transpose_reduce<NV, true>(mx, lane);
                 float *tred = red + (k & 1) * 4 * NP;
                 if (lane % LPH == 0)
@@ -955,7 +986,9 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                     const float m_new = tm > m_ref[g] + C::LAZY ? tm : m_ref[g];
                     alpha[g] = m_new == m_ref[g] ? 1.f : fast_exp2(m_ref[g] - m_new);
                     m_ref[g] = m_new;
-                    x[g] = (see[g] && m_new != -INFINITY) ? fmaf(sc[g], qsc(g), -m_new) : -INFINITY;
+#pragma unroll
+                    for (int th = 0; th < TH; ++th)
+                        x[th][g] = (see[th][g] && m_new != -INFINITY) ? fmaf(sc[th][g], qsc(g), -m_new) : -INFINITY;
                     l_t[g] *= alpha[g];
 #pragma unroll
                     for (int sub = 0; sub < SUB; ++sub)
@@ -967,12 +1000,14 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 ok = false;
                 poisoned = true;
             }
-            float pr[NV];
+            float prh[TH][NV];
 #pragma unroll
-            for (int g = 0; g < NV; ++g) {
-                pr[g] = fast_exp2(x[g]);
-                l_t[g] += pr[g];
-            }
+            for (int th = 0; th < TH; ++th)
+#pragma unroll
+                for (int g = 0; g < NV; ++g) {
+                    prh[th][g] = fast_exp2(x[th][g]);
+                    l_t[g] += prh[th][g];
+                }
             // P = hi + lo, both bf16, as one N = 32 operand (hi heads in columns
             // 0..NP-1, lo heads in NP..2NP-1) in the no-swizzle MN-major layout:
             // token ti's 8-head groups are 16-byte rows of 8x8 core matrices.
@@ -980,7 +1015,11 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 // P = t1 + t2 / 16 + t3 / 256, all E4M3, as one N = 48 operand (term
                 // i of the heads in bytes 0..NP-1 of the token's 16-byte row of core
                 // matrix i), no-swizzle MN-major.
-                unsigned char *pd8 = pbuf + b * C::PBUF_BYTES + (ti >> 3) * P8_LBO + (ti & 7) * 16;
+#pragma unroll
+              for (int th = 0; th < TH; ++th) {
+                const float (&pr)[NV] = prh[th];
+                const int tt = ti + 128 * th;  // the token of this half
+                unsigned char *pd8 = pbuf + b * L::PBUF + (tt >> 3) * P8_LBO + (tt & 7) * 16;
                 uint32_t w1[(NV + 3) / 4], w2[(NV + 3) / 4], w3[(NV + 3) / 4];
 #pragma unroll
                 for (int j = 0; j < (NV + 3) / 4; ++j)
@@ -1006,8 +1045,10 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                     *reinterpret_cast<uint4 *>(pd8 + 128) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
                     *reinterpret_cast<uint4 *>(pd8 + 256) = make_uint4(w3[0], w3[1], w3[2], w3[3]);
                 }
+              }
             } else {
-                unsigned char *pd = pbuf + b * C::PBUF_BYTES + (ti >> 3) * C::P_LBO + (ti & 7) * 16;
+                const float (&pr)[NV] = prh[0];
+                unsigned char *pd = pbuf + b * L::PBUF + (ti >> 3) * C::P_LBO + (ti & 7) * 16;
                 constexpr int NW = NV / 2;  // bf16 pairs per term
                 uint32_t whi[NW], wlo[NW];
 #pragma unroll
@@ -1034,16 +1075,20 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             }
             // Rows past the valid tokens may hold anything (stale tiles, poison):
             // zero this token's V row so that 0-weight rows add exact zeros.
-            if (!valid) {
+#pragma unroll
+            for (int th = 0; th < TH; ++th) {
+              if (!valid[th]) {
 #pragma unroll
                 for (int sub = 0; sub < SUB; ++sub) {
-                    unsigned char *vr = ring + L::V_RING_OFF + (size_t)((k * SUB + sub) % S) * L::SLOT_BYTES + ti * 128;
+                    unsigned char *vr = ring + L::V_RING_OFF + (size_t)((k * SUB + sub) % S) * L::SLOT_BYTES +
+                                        (ti + 128 * th) * 128;
 #pragma unroll
                     for (int h = 0; h < HALVES; ++h)
 #pragma unroll
                         for (int cc = 0; cc < 8; ++cc)
                             *reinterpret_cast<uint4 *>(vr + h * C::BOX_BYTES + cc * 16) = make_uint4(0, 0, 0, 0);
                 }
+              }
             }
             // A moved reference closes the open O buffer (unless this tile opens a
             // piece, whose buffer is fresh anyway).

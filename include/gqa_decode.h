@@ -230,7 +230,7 @@ typedef struct gqa_plan {
     int threads_per_cta;
     int cooperative;         /* 1: cooperative launch (every CTA resident) */
     int merge_launch;        /* 1: a second kernel merges the fixed-split chunks */
-    int tile_tokens;         /* tokens per LeanTile */
+    int tile_tokens;         /* tokens per LeanTile (256 on the FP8 tensor-core kernel) */
     int ring_stages;         /* shared-memory ring slots per K (and per V) stream */
     int box_rows;            /* tensor cores: tokens per TMA box (0 on CUDA cores) */
     long long tiles;         /* LeanTiles of the step (-1 without seq_lens_host) */
@@ -270,10 +270,12 @@ GQA_API int gqa_decode_multi(const void *q, const void *k_cache, const void *v_c
  * and e4m3(byte) * v_scale (one scale per tensor, > 0).  q and out stay bf16.  A
  * decode step reads half the bytes.  At D = 128 with at least 4 query heads per
  * KV head (and the tensor-core kernel's page sizes, B <= 1024) it runs on the
- * tensor cores: kind::f8f6f4 MMAs read the cache bytes as loaded; q enters as
- * two E4M3 terms (t1 + t2 / 16, each q row first scaled by a power of two) and
- * the softmax weights as three (t1 + t2 / 16 + t3 / 256); accumulation in fp32.  Other shapes run on the
- * CUDA-core kernel, the E4M3 bytes widened exactly in registers.  k_scale is
+ * tensor cores over 256-token LeanTiles (64 KB of K and V per step, as a bf16
+ * tile of 128 tokens): kind::f8f6f4 MMAs read the cache bytes as loaded; q
+ * enters as two E4M3 terms (t1 + t2 / 16, each q row first scaled by a power of
+ * two) and the softmax weights as three (t1 + t2 / 16 + t3 / 256); accumulation
+ * in fp32.  Other shapes run on the CUDA-core kernel, the E4M3 bytes widened
+ * exactly in registers.  k_scale is
  * folded into the scores, v_scale applied to the output.  Workspace:
  * gqa_decode_workspace_size.  Errors as gqa_decode.
  */
@@ -287,7 +289,7 @@ GQA_API int gqa_decode_fp8(const void *q, const void *k_cache, const void *v_cac
  * gqa_decode_fp8 with gqa_decode_auto's runtime selection (stream-K, or one CTA
  * per (request, KV head) when that already fills the GPU), given a HOST copy of
  * the lengths, seq_lens_host int32 [B] (read during the call only).  The cost
- * model takes the FP8 tile size (one byte per element) and the FP8 kernel's
+ * model takes the FP8 kernel's tiles (256 tokens, one byte per element) and its
  * 16-head passes.  FP8 caches off the tensor cores (D != 128) always take
  * stream-K.  Arguments, workspace, results and errors otherwise as gqa_decode_fp8.
  */

@@ -23,6 +23,13 @@ CASES = [
     (1, 4, 1, 128, [60000], None),          # one long segment over every CTA
     (2, 16, 2, 128, [5000, 300], 32),       # G = 8
     (1, 32, 2, 128, [40000], 64),           # G = 16, long: split segments merged
+    # 256-token LeanTiles on the tensor cores: lengths around tile and half-tile
+    # edges, 8-token pages (32 TMA boxes per tile, a full warp of them), pages of a
+    # whole tile, a contiguous cache
+    (4, 16, 4, 128, [255, 256, 257, 129], 8),
+    (3, 8, 2, 128, [511, 513, 128], 256),
+    (2, 32, 8, 128, [384, 1], None),
+    (2, 64, 4, 128, [3000, 700], 32),       # G = 16: two head chunks per KV head
 ]
 
 
@@ -75,6 +82,9 @@ def test_fp8_auto_matches_oracle_and_its_plan(case):
                           seq_lens_host=host, device=0)
     if D == 128:
         assert plan["kernel"] == gq.KERNEL_TENSOR_CORE and plan["heads_per_pass"] == min(16, Hq // Hkv)
+        # 256-token LeanTiles: tiles = head passes x KV heads x sum of ceil(L / 256)
+        assert plan["tile_tokens"] == 256
+        assert plan["tiles"] == plan["head_chunks"] * Hkv * sum(-(-L // 256) for L in lens)
     else:
         assert plan["kernel"] == gq.KERNEL_CUDA_CORE and plan["num_splits"] == 0
     if B == 1:  # two segments on 148 SMs: stream-K

@@ -52,8 +52,9 @@ def test_plan_reports_the_dispatch():
     assert _plan(1, 32, 16, 256)["kernel"] == cc                      # D = 256, G = 2
     assert _plan(1, 32, 8, 128, bs=48, paged=True, nb=10)["kernel"] == cc  # page size
     assert _plan(1, 32, 8, 128, bs=64, paged=True, nb=10)["box_rows"] == 64
-    f8 = _plan(1, 32, 8, 128, kv_fp8=True)
+    f8 = _plan(1, 32, 8, 128, kv_fp8=True, seq_lens_host=[1000])
     assert f8["kernel"] == tc and f8["kernel_name"].endswith("F8=1>")
+    assert f8["tile_tokens"] == 256 and f8["ring_stages"] == 3 and f8["tiles"] == 8 * 4  # 256-token tiles
     assert _plan(1, 32, 8, 64, kv_fp8=True)["kernel"] == cc           # FP8 at D = 64
     mqa = _plan(8, 64, 1, 128, seq_lens_host=[100] * 8)   # G = 64: one 64-head pass per tile
     assert mqa["heads_per_pass"] == 64 and mqa["head_chunks"] == 1 and mqa["tiles"] == 8
