@@ -520,11 +520,11 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                         const uint32_t ka = ring_a + (uint32_t)(s * L::SLOT_BYTES);
 #pragma unroll
                         for (int th = 0; th < TH; ++th) {
-                            // token half th: rows 128 th .. of the slot, into its own S columns
+                            // token half th (FP8): slot rows 128 th .., into its own S columns
 #pragma unroll
                             for (int kk = 0; kk < D / SUB / KSTEP; ++kk) {
                                 // 32 bytes of every row per instruction: 16 bf16 or 32 E4M3 elements.
-                                const uint32_t off = (uint32_t)(th * C::BOX_BYTES + (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32);
+                                const uint32_t off = (uint32_t)((th + (kk >> 2)) * C::BOX_BYTES + (kk & 3) * 32);
                                 const uint32_t qoff = (uint32_t)((2 * sub + (kk >> 2)) * NP * 128 + (kk & 3) * 32);
                                 const uint64_t ad = umma_smem_desc(ka + off, 16, 1024, SMEM_LAYOUT_SW128);
                                 const uint64_t bd = umma_smem_desc(qa + qoff, 16, 1024, SMEM_LAYOUT_SW128);
@@ -1016,36 +1016,36 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                 // i of the heads in bytes 0..NP-1 of the token's 16-byte row of core
                 // matrix i), no-swizzle MN-major.
 #pragma unroll
-              for (int th = 0; th < TH; ++th) {
-                const float (&pr)[NV] = prh[th];
-                const int tt = ti + 128 * th;  // the token of this half
-                unsigned char *pd8 = pbuf + b * L::PBUF + (tt >> 3) * P8_LBO + (tt & 7) * 16;
-                uint32_t w1[(NV + 3) / 4], w2[(NV + 3) / 4], w3[(NV + 3) / 4];
+                for (int th = 0; th < TH; ++th) {
+                    const float (&pr)[NV] = prh[th];
+                    const int tt = ti + 128 * th;  // the token of this half
+                    unsigned char *pd8 = pbuf + b * L::PBUF + (tt >> 3) * P8_LBO + (tt & 7) * 16;
+                    uint32_t w1[(NV + 3) / 4], w2[(NV + 3) / 4], w3[(NV + 3) / 4];
 #pragma unroll
-                for (int j = 0; j < (NV + 3) / 4; ++j)
-                    w1[j] = w2[j] = w3[j] = 0u;
+                    for (int j = 0; j < (NV + 3) / 4; ++j)
+                        w1[j] = w2[j] = w3[j] = 0u;
 #pragma unroll
-                for (int g = 0; g < NV; ++g) {
-                    uint32_t t1, t2, t3;
-                    split3_e4m3(pr[g], t1, t2, t3);
-                    w1[g >> 2] |= t1 << (8 * (g & 3));
-                    w2[g >> 2] |= t2 << (8 * (g & 3));
-                    w3[g >> 2] |= t3 << (8 * (g & 3));
+                    for (int g = 0; g < NV; ++g) {
+                        uint32_t t1, t2, t3;
+                        split3_e4m3(pr[g], t1, t2, t3);
+                        w1[g >> 2] |= t1 << (8 * (g & 3));
+                        w2[g >> 2] |= t2 << (8 * (g & 3));
+                        w3[g >> 2] |= t3 << (8 * (g & 3));
+                    }
+                    if constexpr (NV == 4) {
+                        *reinterpret_cast<uint32_t *>(pd8) = w1[0];
+                        *reinterpret_cast<uint32_t *>(pd8 + 128) = w2[0];
+                        *reinterpret_cast<uint32_t *>(pd8 + 256) = w3[0];
+                    } else if constexpr (NV == 8) {
+                        *reinterpret_cast<uint2 *>(pd8) = make_uint2(w1[0], w1[1]);
+                        *reinterpret_cast<uint2 *>(pd8 + 128) = make_uint2(w2[0], w2[1]);
+                        *reinterpret_cast<uint2 *>(pd8 + 256) = make_uint2(w3[0], w3[1]);
+                    } else {
+                        *reinterpret_cast<uint4 *>(pd8) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+                        *reinterpret_cast<uint4 *>(pd8 + 128) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+                        *reinterpret_cast<uint4 *>(pd8 + 256) = make_uint4(w3[0], w3[1], w3[2], w3[3]);
+                    }
                 }
-                if constexpr (NV == 4) {
-                    *reinterpret_cast<uint32_t *>(pd8) = w1[0];
-                    *reinterpret_cast<uint32_t *>(pd8 + 128) = w2[0];
-                    *reinterpret_cast<uint32_t *>(pd8 + 256) = w3[0];
-                } else if constexpr (NV == 8) {
-                    *reinterpret_cast<uint2 *>(pd8) = make_uint2(w1[0], w1[1]);
-                    *reinterpret_cast<uint2 *>(pd8 + 128) = make_uint2(w2[0], w2[1]);
-                    *reinterpret_cast<uint2 *>(pd8 + 256) = make_uint2(w3[0], w3[1]);
-                } else {
-                    *reinterpret_cast<uint4 *>(pd8) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-                    *reinterpret_cast<uint4 *>(pd8 + 128) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
-                    *reinterpret_cast<uint4 *>(pd8 + 256) = make_uint4(w3[0], w3[1], w3[2], w3[3]);
-                }
-              }
             } else {
                 const float (&pr)[NV] = prh[0];
                 unsigned char *pd = pbuf + b * L::PBUF + (ti >> 3) * C::P_LBO + (ti & 7) * 16;
@@ -1077,7 +1077,8 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
             // zero this token's V row so that 0-weight rows add exact zeros.
 #pragma unroll
             for (int th = 0; th < TH; ++th) {
-              if (!valid[th]) {
+                if (valid[th])
+                    continue;
 #pragma unroll
                 for (int sub = 0; sub < SUB; ++sub) {
                     unsigned char *vr = ring + L::V_RING_OFF + (size_t)((k * SUB + sub) % S) * L::SLOT_BYTES +
@@ -1088,7 +1089,6 @@ __global__ void __launch_bounds__(TcCfg::THREADS, 1)
                         for (int cc = 0; cc < 8; ++cc)
                             *reinterpret_cast<uint4 *>(vr + h * C::BOX_BYTES + cc * 16) = make_uint4(0, 0, 0, 0);
                 }
-              }
             }
             // A moved reference closes the open O buffer (unless this tile opens a
             // piece, whose buffer is fresh anyway).
